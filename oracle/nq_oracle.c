@@ -1,0 +1,292 @@
+/*
+ * nq_oracle.c -- plain, slow, single-threaded CPU oracle for the low-rank binary (LRB)
+ * matmul of NanoQuant.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may call, link or load this
+ * file: only the tests, the package smoke check and the CPU-baseline leg of bench.py use
+ * it.  It shares no code, header, table or helper with the CUDA library.
+ *
+ * What it computes, and where each piece comes from
+ * (page "NanoQuant: Efficient Sub-1-Bit Quantization of Large Language Models",
+ *  research.samsung.com blog, unless stated otherwise):
+ *
+ *   - Section 2, "Low-Rank Binary Factorization", first display equation:
+ *         W ~= s1 (.) (U V^T) (.) s2^T,   U in {-1,+1}^{d_out x r},  V in {-1,+1}^{d_in x r},
+ *         s1 in R^{d_out},  s2 in R^{d_in}.
+ *     Read elementwise: W_ij = s1_i * (sum_k U_ik V_jk) * s2_j.  The oracle materialises
+ *     W in fp64 and returns y[b][i] = sum_j W_ij x[b][j], plus
+ *     S[b][i] = sum_j |W_ij x[b][j]| (the magnitude of the terms of that sum).
+ *   - Same section, the sentence after the equation: the representation holds
+ *     r (d_out + d_in) binary values plus (d_out + d_in) floating-point values.
+ *   - Section 3, "Step 3: Factorized Component Refinement", objective: binary factors are
+ *     sign(U), sign(V) of latent real matrices.  sign(0) is not stated; the reading taken
+ *     is +1 iff latent >= 0 (so +0, -0 -> +1; NaN -> -1).
+ *   - Section 3, "Phase 3: Scale-Only Model Reconstruction": frozen binary factors are
+ *     "packed into efficient integer formats"; no layout is given.  The reading taken:
+ *     32 signs per uint32 along r, element k of a row in word k/32 at bit k%32
+ *     (least significant bit first), bit = 1 for +1.  Words of a row beyond r/32 (row
+ *     padding up to the leading dimension) are written as 0 and never read as data.
+ *
+ * Precision: fp16 scales and bf16 activations convert exactly to fp64; the integer Gram
+ * entry G_ij = sum_k U_ik V_jk is exact; W_ij = s1_i G_ij s2_j needs 11+11+13 significant
+ * bits and each product W_ij x_j another 8, all below fp64's 53, so only the final sums
+ * round.  The oracle is therefore the exact result up to one fp64 summation.
+ *
+ * Two evaluation orders are provided on purpose:
+ *   nq_oracle_dense_*     materialise W (the definition);
+ *   nq_oracle_factored_*  y = s1 (.) (U (V^T (s2 (.) x))) in fp64 (the same product, with
+ *                         the associativity the factorisation exists for).
+ * Tests pin each against closed forms, invariants, brute force and integer matmul.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_API __attribute__((visibility("default")))
+
+/* ---------------------------------------------------------------------------------
+ * Number formats, written from the IEEE 754 binary16 definition and from bfloat16 being
+ * the upper half of an IEEE binary32.
+ * --------------------------------------------------------------------------------- */
+
+/* binary16: 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits. */
+ORACLE_API double nq_oracle_f16_to_double(uint16_t h) {
+    int sign = (h >> 15) & 1;
+    int e = (h >> 10) & 0x1F;
+    int f = h & 0x3FF;
+    double v;
+    if (e == 0) {
+        v = ldexp((double)f, -24); /* subnormal: f * 2^-24 */
+    } else if (e == 31) {
+        v = (f == 0) ? INFINITY : NAN;
+    } else {
+        v = ldexp((double)(1024 + f), e - 25); /* (1 + f/1024) * 2^(e-15) */
+    }
+    return sign ? -v : v;
+}
+
+/* bfloat16: the 16 most significant bits of an IEEE binary32. */
+ORACLE_API double nq_oracle_bf16_to_double(uint16_t b) {
+    uint32_t u = ((uint32_t)b) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* fp64 -> bfloat16, round to nearest, ties to even, directly from the real value (no
+ * intermediate binary32 rounding).  bfloat16 keeps 8 significant bits; its smallest normal
+ * is 2^-126 and its quantum below that is 2^-133. */
+ORACLE_API uint16_t nq_oracle_double_to_bf16(double v) {
+    if (isnan(v)) return 0x7FC0;
+    uint16_t sign = signbit(v) ? 0x8000 : 0;
+    double a = fabs(v);
+    if (isinf(a)) return sign | 0x7F80;
+    if (a == 0.0) return sign;
+    int e;
+    frexp(a, &e); /* a = m * 2^e, 0.5 <= m < 1 */
+    int qexp = e - 8;
+    if (qexp < -133) qexp = -133;
+    double q = nearbyint(ldexp(a, -qexp)); /* default rounding mode: to nearest, ties even */
+    double rv = ldexp(q, qexp);
+    if (rv >= ldexp(1.0, 128)) return sign | 0x7F80;
+    float f = (float)rv; /* exact: rv has at most 8 significant bits and is in range */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return sign | (uint16_t)(u >> 16);
+}
+
+/* Array forms of the two conversions above. */
+ORACLE_API void nq_oracle_f16_array_to_double(const uint16_t* h, int64_t n, double* out) {
+    for (int64_t e = 0; e < n; ++e) out[e] = nq_oracle_f16_to_double(h[e]);
+}
+
+ORACLE_API void nq_oracle_bf16_array_to_double(const uint16_t* b, int64_t n, double* out) {
+    for (int64_t e = 0; e < n; ++e) out[e] = nq_oracle_bf16_to_double(b[e]);
+}
+
+/* ---------------------------------------------------------------------------------
+ * sign() and packing.
+ * --------------------------------------------------------------------------------- */
+
+/* Packs sign(latent) of a [rows][ld_latent] fp32 matrix (first r columns) into
+ * [rows][ld_words] uint32 words.  Returns 0, or -1 on bad sizes. */
+ORACLE_API int nq_oracle_pack(const float* latent, int64_t rows, int64_t r, int64_t ld_latent,
+                              uint32_t* packed, int64_t ld_words) {
+    if (rows < 0 || r < 0 || r % 32 != 0 || ld_latent < r || ld_words < r / 32) return -1;
+    for (int64_t i = 0; i < rows; ++i) {
+        uint32_t* row = packed + i * ld_words;
+        for (int64_t w = 0; w < ld_words; ++w) row[w] = 0u;
+        for (int64_t k = 0; k < r; ++k) {
+            float v = latent[i * ld_latent + k];
+            if (v >= 0.0f) row[k / 32] |= 1u << (k % 32);
+        }
+    }
+    return 0;
+}
+
+/* Unpacks [rows][ld_words] words to int8 signs [rows][r] (+1 for bit 1, -1 for bit 0). */
+ORACLE_API int nq_oracle_unpack(const uint32_t* packed, int64_t rows, int64_t r, int64_t ld_words,
+                                int8_t* signs) {
+    if (rows < 0 || r < 0 || r % 32 != 0 || ld_words < r / 32) return -1;
+    for (int64_t i = 0; i < rows; ++i)
+        for (int64_t k = 0; k < r; ++k) {
+            uint32_t bit = (packed[i * ld_words + k / 32] >> (k % 32)) & 1u;
+            signs[i * r + k] = bit ? (int8_t)1 : (int8_t)-1;
+        }
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------------
+ * Gram matrix G = U V^T of the sign factors (exact integers).
+ * --------------------------------------------------------------------------------- */
+
+/* Literal triple loop on unpacked signs: G[i][j] = sum_k U[i][k] V[j][k]. */
+ORACLE_API void nq_oracle_gram_signs(const int8_t* U, const int8_t* V, int64_t d_out, int64_t d_in,
+                                     int64_t r, int32_t* G) {
+    for (int64_t i = 0; i < d_out; ++i)
+        for (int64_t j = 0; j < d_in; ++j) {
+            int32_t acc = 0;
+            for (int64_t k = 0; k < r; ++k) acc += (int32_t)U[i * r + k] * (int32_t)V[j * r + k];
+            G[i * d_in + j] = acc;
+        }
+}
+
+/* One Gram entry from packed rows: matching bits contribute +1, differing bits -1, so
+ * G_ij = r - 2 * (number of differing bits). */
+static int32_t gram_entry_packed(const uint32_t* u_row, const uint32_t* v_row, int64_t r) {
+    int64_t differ = 0;
+    for (int64_t w = 0; w < r / 32; ++w) differ += __builtin_popcount(u_row[w] ^ v_row[w]);
+    return (int32_t)(r - 2 * differ);
+}
+
+ORACLE_API void nq_oracle_gram_packed(const uint32_t* U, int64_t ldu, const uint32_t* V, int64_t ldv,
+                                      int64_t d_out, int64_t d_in, int64_t r, int32_t* G) {
+    for (int64_t i = 0; i < d_out; ++i)
+        for (int64_t j = 0; j < d_in; ++j)
+            G[i * d_in + j] = gram_entry_packed(U + i * ldu, V + j * ldv, r);
+}
+
+/* ---------------------------------------------------------------------------------
+ * Forward products.
+ * --------------------------------------------------------------------------------- */
+
+/* The definition on unpacked signs and fp64 values:
+ *   W_ij = s1_i * G_ij * s2_j,  y[b][i] = sum_j W_ij x[b][j],  S[b][i] = sum_j |W_ij x[b][j]|.
+ * U int8 [d_out][r], V int8 [d_in][r], x [B][d_in]; y, S [B][d_out].  S may be NULL. */
+ORACLE_API void nq_oracle_dense_signs(const int8_t* U, const int8_t* V, const double* s1,
+                                      const double* s2, int64_t d_out, int64_t d_in, int64_t r,
+                                      const double* x, int64_t B, double* y, double* S) {
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t i = 0; i < d_out; ++i) {
+            y[b * d_out + i] = 0.0;
+            if (S) S[b * d_out + i] = 0.0;
+        }
+    for (int64_t i = 0; i < d_out; ++i)
+        for (int64_t j = 0; j < d_in; ++j) {
+            int64_t g = 0;
+            for (int64_t k = 0; k < r; ++k) g += (int64_t)U[i * r + k] * (int64_t)V[j * r + k];
+            double w = s1[i] * (double)g * s2[j];
+            for (int64_t b = 0; b < B; ++b) {
+                double term = w * x[b * d_in + j];
+                y[b * d_out + i] += term;
+                if (S) S[b * d_out + i] += fabs(term);
+            }
+        }
+}
+
+/* The definition on the packed layout with fp16 scales and bf16 activations given as raw
+ * bit patterns, for a chosen subset of output rows (rows == NULL means all d_out rows, in
+ * order).  y and S are [B][n_rows]. */
+ORACLE_API int nq_oracle_dense_packed(const uint32_t* U, int64_t ldu, const uint32_t* V, int64_t ldv,
+                                      const uint16_t* s1_f16, const uint16_t* s2_f16, int64_t d_out,
+                                      int64_t d_in, int64_t r, const uint16_t* x_bf16, int64_t B,
+                                      const int64_t* rows, int64_t n_rows, double* y, double* S) {
+    if (r % 32 != 0 || ldu < r / 32 || ldv < r / 32) return -1;
+    if (rows == NULL) n_rows = d_out;
+    double* s2 = (double*)malloc(sizeof(double) * (size_t)(d_in > 0 ? d_in : 1));
+    double* x = (double*)malloc(sizeof(double) * (size_t)(B * d_in > 0 ? B * d_in : 1));
+    if (!s2 || !x) {
+        free(s2);
+        free(x);
+        return -2;
+    }
+    for (int64_t j = 0; j < d_in; ++j) s2[j] = nq_oracle_f16_to_double(s2_f16[j]);
+    for (int64_t e = 0; e < B * d_in; ++e) x[e] = nq_oracle_bf16_to_double(x_bf16[e]);
+    for (int64_t n = 0; n < n_rows; ++n) {
+        int64_t i = rows ? rows[n] : n;
+        if (i < 0 || i >= d_out) {
+            free(s2);
+            free(x);
+            return -1;
+        }
+        double s1 = nq_oracle_f16_to_double(s1_f16[i]);
+        for (int64_t b = 0; b < B; ++b) {
+            y[b * n_rows + n] = 0.0;
+            if (S) S[b * n_rows + n] = 0.0;
+        }
+        for (int64_t j = 0; j < d_in; ++j) {
+            double w = s1 * (double)gram_entry_packed(U + i * ldu, V + j * ldv, r) * s2[j];
+            for (int64_t b = 0; b < B; ++b) {
+                double term = w * x[b * d_in + j];
+                y[b * n_rows + n] += term;
+                if (S) S[b * n_rows + n] += fabs(term);
+            }
+        }
+    }
+    free(s2);
+    free(x);
+    return 0;
+}
+
+/* The factored evaluation order, in fp64, on the packed layout:
+ *   z[b][j] = s2_j x[b][j];  t[b][k] = sum_j V_jk z[b][j];  y[b][i] = s1_i sum_k U_ik t[b][k].
+ * y is [B][d_out]. */
+ORACLE_API int nq_oracle_factored_packed(const uint32_t* U, int64_t ldu, const uint32_t* V, int64_t ldv,
+                                         const uint16_t* s1_f16, const uint16_t* s2_f16, int64_t d_out,
+                                         int64_t d_in, int64_t r, const uint16_t* x_bf16, int64_t B,
+                                         double* y) {
+    if (r % 32 != 0 || ldu < r / 32 || ldv < r / 32) return -1;
+    double* t = (double*)malloc(sizeof(double) * (size_t)(r > 0 ? r : 1));
+    if (!t) return -2;
+    for (int64_t b = 0; b < B; ++b) {
+        for (int64_t k = 0; k < r; ++k) t[k] = 0.0;
+        for (int64_t j = 0; j < d_in; ++j) {
+            double z = nq_oracle_f16_to_double(s2_f16[j]) * nq_oracle_bf16_to_double(x_bf16[b * d_in + j]);
+            const uint32_t* vrow = V + j * ldv;
+            for (int64_t k = 0; k < r; ++k) {
+                uint32_t bit = (vrow[k / 32] >> (k % 32)) & 1u;
+                t[k] += bit ? z : -z;
+            }
+        }
+        for (int64_t i = 0; i < d_out; ++i) {
+            const uint32_t* urow = U + i * ldu;
+            double acc = 0.0;
+            for (int64_t k = 0; k < r; ++k) {
+                uint32_t bit = (urow[k / 32] >> (k % 32)) & 1u;
+                acc += bit ? t[k] : -t[k];
+            }
+            y[b * d_out + i] = nq_oracle_f16_to_double(s1_f16[i]) * acc;
+        }
+    }
+    free(t);
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------------
+ * SiLU-gated product between the gate/up and down projections of a Llama MLP block.  This
+ * is not on the pages; it is the MLP composition of the 7B/70B workloads:
+ *   h = bf16( silu(g) * u ),  silu(g) = g / (1 + exp(-g)),  in fp64 before the rounding.
+ * g, u given as fp64; h returned as bf16 bit patterns.
+ * --------------------------------------------------------------------------------- */
+ORACLE_API void nq_oracle_silu_mul(const double* g, const double* u, int64_t n, uint16_t* h_bf16) {
+    for (int64_t e = 0; e < n; ++e) {
+        double s = g[e] / (1.0 + exp(-g[e]));
+        h_bf16[e] = nq_oracle_double_to_bf16(s * u[e]);
+    }
+}
+
+/* Rounds n fp64 values to bf16 bit patterns (round to nearest, ties to even). */
+ORACLE_API void nq_oracle_round_bf16(const double* v, int64_t n, uint16_t* out) {
+    for (int64_t e = 0; e < n; ++e) out[e] = nq_oracle_double_to_bf16(v[e]);
+}

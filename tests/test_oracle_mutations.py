@@ -1,0 +1,49 @@
+"""The oracle pins must bite: each planted mistake in a copy of the oracle fails them.
+
+Mistakes are planted in a temporary copy of ``oracle/nq_oracle.c`` on the CPU (never in the
+CUDA path); the pin suite then runs against that copy in a subprocess and must fail.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "nq_oracle.c")
+
+MUTATIONS = [
+    # Gram from popcount: a dropped factor of 2
+    ("return (int32_t)(r - 2 * differ);", "return (int32_t)(r - differ);"),
+    # a dropped s2 term in the materialised weight
+    ("double w = s1 * (double)gram_entry_packed(U + i * ldu, V + j * ldv, r) * s2[j];",
+     "double w = s1 * (double)gram_entry_packed(U + i * ldu, V + j * ldv, r);"),
+    # a wrong sign in the factored stage 1
+    ("t[k] += bit ? z : -z;", "t[k] += bit ? z : z;"),
+    # a transposed operand: V indexed by the output row
+    ("double w = s1 * (double)gram_entry_packed(U + i * ldu, V + j * ldv, r) * s2[j];",
+     "double w = s1 * (double)gram_entry_packed(U + (j % d_out) * ldu, V + (i % d_in) * ldv, r) * s2[j];"),
+    # sign(0) read as -1
+    ("if (v >= 0.0f) row", "if (v > 0.0f) row"),
+    # MSB-first bit order
+    ("row[k / 32] |= 1u << (k % 32);", "row[k / 32] |= 1u << (31 - k % 32);"),
+    # bf16 rounding keeps one bit too few
+    ("int qexp = e - 8;", "int qexp = e - 9;"),
+    # fp16 decode with the wrong exponent bias
+    ("v = ldexp((double)(1024 + f), e - 25);", "v = ldexp((double)(1024 + f), e - 24);"),
+]
+
+
+@pytest.mark.parametrize("old,new", MUTATIONS)
+def test_pins_fail_on_planted_mistake(tmp_path, old, new):
+    src = open(SRC).read()
+    assert old in src, "mutation anchor not found"
+    mutant = tmp_path / "mutant.c"
+    mutant.write_text(src.replace(old, new, 1))
+    so = tmp_path / "libmutant.so"
+    subprocess.check_call(["gcc", "-std=c11", "-O2", "-fPIC", "-shared", "-o", str(so), str(mutant), "-lm"])
+    env = dict(os.environ, NQ_ORACLE_SO=str(so))
+    proc = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
+                           os.path.join(ROOT, "tests", "test_oracle.py")],
+                          cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
+    assert proc.returncode != 0, "pins passed on a planted mistake: " + new
