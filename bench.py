@@ -1,0 +1,490 @@
+#!/usr/bin/env python
+"""Benchmark of the LRB (low-rank binary) matmul path on B200.
+
+Headline: batch-1 decode of the Llama-2-7B attention projection (d_out = d_in = 4096,
+r = 2048, 1.0 bit/weight).  One step is one pass of a chain of distinct layer instances
+(y of one layer is x of the next), enough of them that the weights (>= 3x the L2 size)
+stream from HBM on every step; the chain is captured once as a CUDA graph of the public
+API calls and replayed.  Reported: microseconds per layer (whole job), achieved HBM GB/s
+of the layer forward against the measured copy bandwidth, the CPU oracle on the host cores,
+and an end-to-end figure with host<->device copies inside the timed region.
+
+Launch: ``python bench.py [--gpus N --steps K --warmup W]``; for N > 1 one process per GPU
+(torchrun), each an independent replica (the path has no cross-GPU exchange).
+``--impl reference`` times the CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from rank_binary_factorized_b200 import synth  # noqa: E402
+
+HEADLINE = "attn7b"
+METRIC = "binary low-rank matmul µs/layer + achieved HBM GB/s (% roofline), batch 1"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["nq", "reference"], default="nq")
+    ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--headline-only", action="store_true", help="skip the other workloads")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU oracle sample budget")
+    return ap.parse_args()
+
+
+# --------------------------------------------------------------------------- plumbing
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def profile_traffic(kernel_key: str):
+    """DRAM bytes per launch recorded from an ncu capture in profiles/ (None if absent or
+    if the kernel source changed since: the summary records the source hash)."""
+    import hashlib
+    for path in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
+        text = open(path).read()
+        tag = "traffic[%s]:" % kernel_key
+        if tag not in text:
+            continue
+        line = [ln for ln in text.splitlines() if ln.startswith(tag)][0]
+        fields = dict(kv.split("=") for kv in line[len(tag):].split())
+        src = os.path.join(ROOT, fields["source"])
+        if not os.path.exists(src):
+            return None
+        if hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] != fields["sha"]:
+            return None
+        return float(fields["bytes"])
+    return None
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index: int, period_s: float = 0.01):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                bits = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for b, name in self.REASONS.items():
+                    if bits & b and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"]}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------- GPU arm
+class Chain:
+    """n distinct instances of one projection shape on the device, chained y -> x."""
+
+    def __init__(self, torch, nq, d_out, d_in, r, M, n, seed, ws=None):
+        self.M, self.n = M, n
+        self.layers = []
+        for i in range(n):
+            p = synth.make_projection("chain", d_out, d_in, r, seed=seed, key=i)
+            self.layers.append(nq.Layer.from_host(p.U, p.V, p.s1, p.s2, r))
+        need = max(L.workspace_bytes(M) for L in self.layers)
+        self.ws = ws if ws is not None and ws.numel() >= need else torch.zeros(need, dtype=torch.uint8, device="cuda")
+        xb = synth.acts_bf16(synth.rng_for(seed, 999), (M, d_in))
+        self.x0 = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
+        self.bufs = [torch.empty((M, d_out), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+        self.chained = d_in == d_out
+
+    def run(self, nq, stream):
+        x = self.x0
+        for i, L in enumerate(self.layers):
+            y = self.bufs[i % 2]
+            nq.layer_forward(L, x, y, ws=self.ws, stream=stream)
+            x = y if self.chained else self.x0
+        return x
+
+    @property
+    def weight_bytes(self):
+        return sum(L.storage_bytes for L in self.layers)
+
+
+def graph_of(torch, fn, stream):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        fn()  # warm (attribute setup, lazy loads) outside the capture
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def timed_replays(torch, g, stream, steps, warmup, dist=None, sampler=None):
+    """Device time of `steps` replays (ms), bracketed by barrier + sync, max over ranks."""
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            g.replay()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ctx = sampler if sampler is not None else _null()
+    with ctx:
+        start.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(steps):
+                g.replay()
+        end.record(stream)
+        torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end)
+    if dist is not None:
+        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return ms
+
+
+class _null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
+
+
+def decode_bytes(d_out, d_in, r, M):
+    """Algorithmic bytes of one projection: packed signs + fp16 scales + bf16 in/out."""
+    return r * (d_in + d_out) // 8 + 2 * (d_in + d_out) + 2 * M * (d_in + d_out)
+
+
+def n_instances(layer_bytes):
+    return max(8, int(np.ceil(3 * L2_BYTES / layer_bytes)))
+
+
+def gpu_arm(args, rank, world, local):
+    import torch
+    from rank_binary_factorized_b200 import nq
+
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as tdist
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+        dist = tdist
+    hbm_gbs, bf16_tf, bf16_tf_sus, peak_src = measured_peaks()
+    stream = torch.cuda.Stream()
+
+    # ---- headline: 7B attention projection, batch M, chain of distinct instances
+    (_, d_out, d_in, r), = synth.WORKLOADS[HEADLINE]
+    M = args.batch
+    lbytes = decode_bytes(d_out, d_in, r, M)
+    n = n_instances(lbytes)
+    chain = Chain(torch, nq, d_out, d_in, r, M, n, seed=synth.workload_seed(HEADLINE))
+    g = graph_of(torch, lambda: chain.run(nq, stream), stream)
+    sampler = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                           int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local]))
+    ms = timed_replays(torch, g, stream, args.steps, args.warmup, dist, sampler)
+    nq.sync_status(stream)
+    layers_total = args.steps * n * world
+    us_per_layer_job = ms * 1e3 / layers_total  # whole job: all ranks' layers in the max time
+    us_per_layer_gpu = ms * 1e3 / (args.steps * n)  # one GPU's layer forward
+    achieved = lbytes / (us_per_layer_gpu * 1e-6) / 1e9
+    del g
+
+    result = {
+        "metric": METRIC,
+        "value": round(us_per_layer_job, 4),
+        "unit": "us/layer",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms / args.steps, 4),
+        "higher_is_better": False,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic (seeded iid +-1 signs, fp16 0.02|N(0,1)| scales, bf16 N(0,1) activations)",
+        "config": {
+            "workload": "Llama-2-7B attention projection d_out=d_in=4096 r=2048 (1.0 bit/weight), decode batch %d" % M,
+            "batch": M,
+            "operands": "1-bit packed U, V (uint32 words); fp16 s1, s2; bf16 x, y; fp32 accumulate",
+            "layers_per_step": n,
+            "chain": "y of each layer is x of the next (distinct weights per layer)",
+            "l2": "no flush: %d distinct layers = %.0f MB of weights per step > 3x L2" % (n, chain.weight_bytes / 1e6),
+            "parallelism": "replicas" if world > 1 else "single GPU",
+        },
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "decode layer forward (stage-1 + stage-2 kernels, PDL-chained)",
+            "achieved": round(achieved, 1),
+            "peak": hbm_gbs,
+            "peak_source": peak_src + " (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else peak_src,
+            "unit": "GB/s",
+            "frac": round(achieved / hbm_gbs, 4),
+            "traffic": profile_traffic("decode_attn7b_b%d" % M),
+            "algorithmic_bytes_per_launch": lbytes,
+        },
+        "clocks": sampler.summary(),
+        "gpu_launches": 2 * n * args.steps,
+    }
+
+    # ---- end to end through the public API: H2D of the step's input from pinned memory,
+    # the chain of layer_forward calls (captured once as a graph), D2H of the result
+    result["e2e"] = e2e_measure(torch, nq, chain, stream, args, dist, world)
+
+    if not args.headline_only:
+        result["extra"] = extras(torch, nq, stream, args, hbm_gbs, bf16_tf, bf16_tf_sus, peak_src)
+
+    if rank == 0 and world == 1:
+        result["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    elif rank == 0:
+        result["cpu_baseline"] = None
+
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result
+
+
+def e2e_measure(torch, nq, chain, stream, args, dist, world):
+    M = chain.M
+    d_in = chain.layers[0].d_in
+    d_out = chain.layers[0].d_out
+    host_x = torch.from_numpy(synth.acts_bf16(synth.rng_for(77), (M, d_in)).view(np.int16)).pin_memory()
+    host_y = torch.empty((M, d_out), dtype=torch.int16).pin_memory()
+    x_dev = chain.x0
+
+    def step():
+        x_dev.view(torch.int16).copy_(host_x, non_blocking=True)
+        y = chain.run(nq, stream)
+        host_y.copy_(y.view(torch.int16), non_blocking=True)
+
+    g = graph_of(torch, step, stream)
+    ms = timed_replays(torch, g, stream, args.steps, args.warmup, dist)
+    del g
+    return {"value": round(ms * 1e3 / (args.steps * chain.n * world), 4), "unit": "us/layer",
+            "h2d_bytes_per_step": int(host_x.numel() * 2), "d2h_bytes_per_step": int(host_y.numel() * 2),
+            "note": "graph of public-API layer_forward calls with a pinned-host H2D of x and D2H of y per step"}
+
+
+def extras(torch, nq, stream, args, hbm_gbs, bf16_tf, bf16_tf_sus, peak_src):
+    out = {}
+    steps = max(5, args.steps // 5)
+    warm = max(3, args.warmup)
+
+    # decode batch 8 of the headline shape
+    (_, d_out, d_in, r), = synth.WORKLOADS[HEADLINE]
+    lb = decode_bytes(d_out, d_in, r, 8)
+    ch = Chain(torch, nq, d_out, d_in, r, 8, n_instances(lb), seed=synth.workload_seed(HEADLINE) + 50)
+    g = graph_of(torch, lambda: ch.run(nq, stream), stream)
+    ms = timed_replays(torch, g, stream, steps, warm)
+    us = ms * 1e3 / (steps * ch.n)
+    out["attn7b_b8"] = {"us_per_layer": round(us, 3), "GB_s": round(lb / us / 1e3, 1),
+                        "frac_hbm": round(lb / us / 1e3 / hbm_gbs, 4)}
+    del g, ch
+
+    # MLP block (7B) and 70B decoder layer: one block = all its projections (+ SiLU.mul)
+    for wl in ("mlp7b", "layer70b"):
+        shapes = synth.WORKLOADS[wl]
+        block_bytes = sum(decode_bytes(do, di, r, 1) for (_, do, di, r) in shapes)
+        reps = max(2, int(np.ceil(3 * L2_BYTES / block_bytes)))
+        blocks = []
+        for b in range(reps):
+            projs = {}
+            for idx, (name, do, di, rr) in enumerate(shapes):
+                p = synth.make_projection(name, do, di, rr, seed=synth.workload_seed(wl), key=1000 * b + idx)
+                projs[name] = nq.Layer.from_host(p.U, p.V, p.s1, p.s2, rr)
+            blocks.append(projs)
+        need = max(L.workspace_bytes(1) for bl in blocks for L in bl.values())
+        ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+        dmodel = shapes[0][2]
+        x = torch.zeros((1, dmodel), dtype=torch.bfloat16, device="cuda").normal_()
+        bufs = {name: torch.empty((1, do), dtype=torch.bfloat16, device="cuda") for (name, do, di, rr) in shapes}
+        h = torch.empty((1, blocks[0]["gate"].d_out), dtype=torch.bfloat16, device="cuda")
+        attn_in = torch.zeros((1, shapes[0][1]), dtype=torch.bfloat16, device="cuda").normal_()
+
+        def run_blocks():
+            xx = x
+            for bl in blocks:
+                if "q" in bl:
+                    for name in ("q", "k", "v"):
+                        nq.layer_forward(bl[name], xx, bufs[name], ws=ws, stream=stream)
+                    nq.layer_forward(bl["o"], attn_in, bufs["o"], ws=ws, stream=stream)
+                    xin = bufs["o"]
+                else:
+                    xin = xx
+                nq.layer_forward(bl["gate"], xin, bufs["gate"], ws=ws, stream=stream)
+                nq.layer_forward(bl["up"], xin, bufs["up"], ws=ws, stream=stream)
+                nq.silu_mul(bufs["gate"], bufs["up"], h, stream=stream)
+                nq.layer_forward(bl["down"], h, bufs["down"], ws=ws, stream=stream)
+                xx = bufs["down"]
+
+        g = graph_of(torch, run_blocks, stream)
+        ms = timed_replays(torch, g, stream, steps, warm)
+        us = ms * 1e3 / (steps * reps)
+        out[wl] = {"us_per_block": round(us, 3), "block_bytes": block_bytes, "GB_s": round(block_bytes / us / 1e3, 1),
+                   "frac_hbm": round(block_bytes / us / 1e3 / hbm_gbs, 4), "blocks_per_step": reps,
+                   "block": "+".join(n for (n, *_r) in shapes) + " + silu_mul"}
+        del g, blocks
+
+    # prefill, 70B gate projection
+    (_, do, di, r), = synth.WORKLOADS["prefill70b"]
+    p = synth.make_projection("gate", do, di, r, seed=synth.workload_seed("prefill70b"))
+    L = nq.Layer.from_host(p.U, p.V, p.s1, p.s2, r)
+    pre = {}
+    for M in (64, 512, 2048):
+        x = torch.zeros((M, di), dtype=torch.bfloat16, device="cuda").normal_()
+        y = torch.empty((M, do), dtype=torch.bfloat16, device="cuda")
+        ws = L.workspace(M)
+        g = graph_of(torch, lambda: nq.lrb_matmul(L, x, y, ws=ws, stream=stream), stream)
+        psteps = 3 if M >= 512 else steps
+        ms = timed_replays(torch, g, stream, psteps, 2)
+        us = ms * 1e3 / psteps
+        flops = 2.0 * M * r * (di + do)
+        pre["M%d" % M] = {"us": round(us, 2), "TFLOP_s": round(flops / us / 1e6, 2),
+                          "frac_bf16": round(flops / us / 1e6 / bf16_tf, 4)}
+        del g
+    out["prefill70b_gate"] = pre
+
+    # pack: the 70B gate U, 28672 x 3520 fp32 -> packed words
+    rows, rr = 28672, 3520
+    lat = torch.randn((rows, rr), dtype=torch.float32, device="cuda")
+    pk = torch.empty((rows, rr // 32), dtype=torch.int32, device="cuda")
+    g = graph_of(torch, lambda: nq.pack_signs(lat, r=rr, out=pk, stream=stream), stream)
+    ms = timed_replays(torch, g, stream, steps, warm)
+    us = ms * 1e3 / steps
+    pbytes = 4 * rows * rr + rows * rr // 8
+    out["pack_70b_gate_U"] = {"us": round(us, 2), "GB_s": round(pbytes / us / 1e3, 1),
+                              "frac_hbm": round(pbytes / us / 1e3 / hbm_gbs, 4)}
+    nq.sync_status(stream)
+    return out
+
+
+# --------------------------------------------------------------------------- CPU oracle
+def cpu_baseline(budget_s: float):
+    """The oracle (plain single-threaded C, fp64, factored order) on the headline layer."""
+    import oracle
+    (_, d_out, d_in, r), = synth.WORKLOADS[HEADLINE]
+    p = synth.make_projection("cpu", d_out, d_in, r, seed=synth.workload_seed(HEADLINE))
+    xb = synth.acts_bf16(synth.rng_for(5), (1, d_in))
+    times = []
+    t_end = time.perf_counter() + budget_s
+    while time.perf_counter() < t_end or len(times) < 3:
+        t0 = time.perf_counter()
+        oracle.factored_packed(p.U, p.V, p.s1, p.s2, r, xb)
+        times.append(time.perf_counter() - t0)
+    us = statistics.median(times) * 1e6
+    return {"value": round(us, 1), "unit": "us/layer", "cores": 1, "kind": "oracle",
+            "sample": "%d forwards of the factored fp64 oracle (s1 (.) U (V^T (s2 (.) x))) on one 4096x4096 r=2048 "
+                      "layer at batch 1, single thread, median" % len(times)}
+
+
+def reference_arm(args):
+    rank, world, local = dist_env()
+    if rank != 0:
+        return None
+    base = cpu_baseline(max(1.0, min(args.cpu_seconds, 60.0)))
+    steps_us = []
+    import oracle
+    (_, d_out, d_in, r), = synth.WORKLOADS[HEADLINE]
+    p = synth.make_projection("cpu", d_out, d_in, r, seed=synth.workload_seed(HEADLINE))
+    xb = synth.acts_bf16(synth.rng_for(6), (args.batch, d_in))
+    for _ in range(args.warmup):
+        oracle.factored_packed(p.U, p.V, p.s1, p.s2, r, xb)
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.factored_packed(p.U, p.V, p.s1, p.s2, r, xb)
+        steps_us.append((time.perf_counter() - t0) * 1e6)
+    v = statistics.median(steps_us)
+    return {"impl": "reference", "metric": METRIC, "value": round(v, 1), "unit": "us/layer", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(v / 1e3, 3), "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "Llama-2-7B attention projection d_out=d_in=4096 r=2048, decode batch %d" % args.batch,
+                       "batch": args.batch, "layers_per_step": 1},
+            "cpu_baseline": {**base, "value": round(v, 1)},
+            "e2e": {"value": round(v, 1), "unit": "us/layer", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse_args()
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        res = reference_arm(args)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return 0
+    res = gpu_arm(args, rank, world, local)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

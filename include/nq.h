@@ -1,0 +1,162 @@
+/*
+ * nq.h -- C ABI of the B200 (sm_100a) low-rank binary (LRB) matmul library, libnq.so.
+ *
+ * The operation (page "NanoQuant: Efficient Sub-1-Bit Quantization of Large Language
+ * Models", research.samsung.com blog, section 2 "Low-Rank Binary Factorization",
+ * factorisation equation):
+ *
+ *     W ~= s1 (.) (U V^T) (.) s2^T,   U in {-1,+1}^{d_out x r},  V in {-1,+1}^{d_in x r}
+ *
+ * and the library evaluates, without ever forming W,
+ *
+ *     y[m][i] = s1_i * sum_k U_ik * ( sum_j V_jk * s2_j * x[m][j] )
+ *
+ * for M rows of activations x.  The sign factors are stored as packed bits (section 3,
+ * "Phase 3: Scale-Only Model Reconstruction": frozen binary factors packed into integer
+ * formats).
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ * - Tensor pointers are DEVICE pointers on the current CUDA device, owned by the caller.
+ *   The library never allocates or frees device memory, never synchronises the stream
+ *   (except nq_sync_status) and keeps no state between calls besides one device error word
+ *   per device.  Calls on different streams may run concurrently as long as they do not
+ *   share a workspace.
+ * - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ * - Packed sign layout: row i of a [rows][ld] uint32 matrix holds element k of that row at
+ *   bit (k % 32) of word (k / 32), least significant bit first; bit 1 means +1, bit 0
+ *   means -1.  r must be a multiple of 32.  Words r/32 .. ld-1 of a row are padding: pack
+ *   writes them as 0 and no reader looks at them.
+ * - fp16 values (s1, s2) and bf16 values (x, y) are passed as uint16_t bit patterns.
+ * - Activations are row-major: x is [M][d_in], y is [M][d_out], contiguous.
+ * - Alignment: every pointer must be 16-byte aligned (NQ_ERR_ALIGN otherwise).
+ * - Arguments are validated on the host before anything is launched; on an error nothing
+ *   is launched and outputs are untouched.
+ * - Kernels read the weights (U, V, s1, s2) before they wait for the work queued ahead of
+ *   them on the stream (programmatic dependent launch): the caller must not write a
+ *   layer's weights in the kernel launched immediately before a call that reads them
+ *   without a stream/event synchronisation in between.  Activations and workspace are
+ *   only touched after that wait.
+ */
+#ifndef NQ_H_
+#define NQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Exported from libnq.so (the library is built with hidden default visibility). */
+#if defined(__GNUC__)
+#define NQ_API __attribute__((visibility("default")))
+#else
+#define NQ_API
+#endif
+
+typedef enum nq_status {
+    NQ_OK = 0,
+    NQ_ERR_NULL = 1,      /* a required pointer is NULL */
+    NQ_ERR_SHAPE = 2,     /* non-positive size, r % 32 != 0, ld too small, M out of range */
+    NQ_ERR_ALIGN = 3,     /* a pointer is not 16-byte aligned */
+    NQ_ERR_WORKSPACE = 4, /* workspace NULL or smaller than nq_workspace_bytes() */
+    NQ_ERR_DEVICE = 5,    /* current device is not compute capability 10.0 (B200) */
+    NQ_ERR_LAUNCH = 6,    /* a kernel launch failed */
+    NQ_ERR_TIMEOUT = 7    /* a bounded device-side wait gave up (seen by nq_sync_status) */
+} nq_status;
+
+/* One LRB linear layer.  All pointers are device pointers; the struct itself is host
+ * memory and is read only during the call. */
+typedef struct nq_lrb_layer {
+    int64_t d_out;      /* output features (rows of U, length of s1) */
+    int64_t d_in;       /* input features (rows of V, length of s2) */
+    int64_t r;          /* rank, a multiple of 32, at most NQ_MAX_RANK_LIMIT */
+    const uint32_t* U;  /* [d_out][ldu] packed signs of U */
+    int64_t ldu;        /* words per row of U, >= r/32 */
+    const uint32_t* V;  /* [d_in][ldv] packed signs of V */
+    int64_t ldv;        /* words per row of V, >= r/32 */
+    const uint16_t* s1; /* [d_out] fp16 */
+    const uint16_t* s2; /* [d_in] fp16 */
+} nq_lrb_layer;
+
+/* Largest rank any entry point accepts. */
+#define NQ_MAX_RANK_LIMIT 262144
+
+/* Largest row count nq_lrb_matvec accepts (the decode path). */
+#define NQ_MATVEC_MAX_M 8
+
+/*
+ * nq_pack_signs -- sign extraction and bit packing of latent factors.
+ * Section 3 "Step 3: Factorized Component Refinement" (the binary factors are sign(U),
+ * sign(V) of latent matrices) and "Phase 3" (frozen signs packed into integers).
+ *   latent    [rows][ld_latent] fp32, device; columns 0..r-1 are read.
+ *   packed    [rows][ld_words] uint32, device; written in full (pad words = 0).
+ *   bit(i,k) = (latent[i][k] >= 0): +0 and -0 give 1, NaN gives 0, +-inf by sign.
+ * Requires rows >= 0, r >= 0, r % 32 == 0, ld_latent >= r, ld_words >= r/32.  rows == 0
+ * or r == 0 with ld_words == 0 is a no-op.  Bit-exact and deterministic.
+ */
+NQ_API nq_status nq_pack_signs(const float* latent, int64_t rows, int64_t r, int64_t ld_latent, uint32_t* packed,
+                        int64_t ld_words, void* stream);
+
+/*
+ * nq_workspace_bytes -- device scratch a call with M activation rows needs (for both
+ * nq_lrb_matvec and nq_lrb_matmul through nq_layer_forward).  Returns 0 for an invalid
+ * layer or M.  The workspace must stay untouched by other work while the call runs.  Its
+ * first 4096 bytes hold counters that read zero between calls (the library restores them
+ * before each call ends); the rest is scratch.  So one workspace can be reused by
+ * consecutive calls of any shape on the same stream, provided it was zero-filled once
+ * before its first use (and again after a call reported NQ_ERR_TIMEOUT).
+ */
+NQ_API size_t nq_workspace_bytes(const nq_lrb_layer* L, int64_t M);
+
+/*
+ * nq_lrb_matvec -- decode path, 1 <= M <= NQ_MATVEC_MAX_M.
+ * Section 2 factorisation equation, evaluated as two streaming stages over the packed
+ * words: t[m][k] = sum_j V_jk s2_j x[m][j] (fp32), then y[m][i] = bf16(s1_i sum_k U_ik t[m][k]).
+ *   x [M][d_in] bf16, y [M][d_out] bf16 (round to nearest even), ws = workspace of at
+ *   least nq_workspace_bytes(L, M) bytes (16-byte aligned, zero-filled before first use).
+ * Accumulation is fp32; results are run-to-run deterministic.
+ */
+NQ_API nq_status nq_lrb_matvec(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y, int64_t M, void* ws,
+                        size_t ws_bytes, void* stream);
+
+/*
+ * nq_lrb_matmul -- prefill path on the tensor cores (tcgen05), any M >= 1 (tuned for
+ * M >= 64).  Same operation as nq_lrb_matvec.  The activations are scaled by s2 and
+ * rounded to fp16, the packed signs are expanded to fp16 +-1 on chip, both products
+ * accumulate in fp32 (TMEM), the intermediate t is rounded to fp16, and y is rounded to
+ * bf16.  Finite results require |x_j s2_j| and |t_k| below the fp16 range (65504).
+ */
+NQ_API nq_status nq_lrb_matmul(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y, int64_t M, void* ws,
+                        size_t ws_bytes, void* stream);
+
+/* nq_layer_forward -- M <= NQ_MATVEC_MAX_M: nq_lrb_matvec; otherwise nq_lrb_matmul. */
+NQ_API nq_status nq_layer_forward(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y, int64_t M, void* ws,
+                           size_t ws_bytes, void* stream);
+
+/*
+ * nq_silu_mul -- h[e] = bf16( silu(g[e]) * u[e] ), silu(g) = g / (1 + exp(-g)), fp32 math,
+ * for the Llama MLP block built from LRB projections (gate, up -> h -> down).  Not part of
+ * the factorisation itself.  g, u, h: n bf16 values each, device.
+ */
+NQ_API nq_status nq_silu_mul(const uint16_t* g, const uint16_t* u, uint16_t* h, int64_t n, void* stream);
+
+/*
+ * nq_sync_status -- synchronises `stream`, then reports and clears this device's error
+ * word: NQ_ERR_TIMEOUT if a bounded device-side wait gave up since the last check,
+ * NQ_ERR_LAUNCH if the stream reported an asynchronous CUDA error, NQ_OK otherwise.
+ */
+NQ_API nq_status nq_sync_status(void* stream);
+
+/* Human-readable name of a status code (static storage). */
+NQ_API const char* nq_status_string(nq_status s);
+
+/* Library build identification (static storage): target architecture and version. */
+NQ_API const char* nq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NQ_H_ */

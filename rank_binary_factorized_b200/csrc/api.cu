@@ -1,0 +1,202 @@
+// api.cu -- the C ABI declared in include/nq.h: argument validation, device checks,
+// workspace planning and dispatch to the kernels.  No allocation, no synchronisation (except
+// nq_sync_status), no fallback: a device that is not sm_100 gets NQ_ERR_DEVICE.
+#include <mutex>
+
+#include "nq_common.cuh"
+
+namespace nq {
+__device__ unsigned int g_error_word = 0u;
+}
+
+// kernels' host launchers (defined next to each kernel)
+nq_status nq_launch_pack(const float*, int64_t, int64_t, int64_t, uint32_t*, int64_t, cudaStream_t);
+nq_status nq_launch_decode(const nq_lrb_layer*, const uint16_t*, uint16_t*, int64_t, void*, cudaStream_t, bool);
+size_t nq_decode_workspace_bytes(int64_t d_in, int64_t r, int64_t M);
+size_t nq_decode_stage2_smem(int64_t r, int64_t M);
+nq_status nq_launch_silu_mul(const uint16_t*, const uint16_t*, uint16_t*, int64_t, cudaStream_t, bool);
+nq_status nq_launch_prefill(const nq_lrb_layer*, const uint16_t*, uint16_t*, int64_t, void*, cudaStream_t, bool);
+size_t nq_prefill_workspace_bytes(const nq_lrb_layer*, int64_t M);
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr size_t kMaxDecodeSmem = 200 * 1024;
+
+struct DeviceInfo {
+    std::once_flag once;
+    bool ok = false;
+    int sms = 0;
+    unsigned int* err = nullptr;
+};
+DeviceInfo g_dev[kMaxDevices];
+
+// Returns the current device's info, probing it once.  ok == false: not sm_100.
+DeviceInfo* current_device() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    DeviceInfo* d = &g_dev[dev];
+    std::call_once(d->once, [d, dev]() {
+        int major = 0, minor = 0, sms = 0;
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        d->sms = sms;
+        d->ok = (major == 10 && minor == 0 && sms > 0);
+        void* p = nullptr;
+        if (d->ok && cudaGetSymbolAddress(&p, nq::g_error_word) == cudaSuccess) d->err = static_cast<unsigned int*>(p);
+        d->ok = d->ok && d->err != nullptr;
+    });
+    return d;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool pdl_enabled() {
+    static const bool on = [] {
+        const char* e = getenv("NQ_DISABLE_PDL");
+        return !(e && e[0] == '1');
+    }();
+    return on;
+}
+
+nq_status check_layer(const nq_lrb_layer* L) {
+    if (!L || !L->U || !L->V || !L->s1 || !L->s2) return NQ_ERR_NULL;
+    if (L->d_out <= 0 || L->d_in <= 0 || L->r <= 0 || (L->r % 32) != 0) return NQ_ERR_SHAPE;
+    if (L->ldu < L->r / 32 || L->ldv < L->r / 32 || L->r > NQ_MAX_RANK) return NQ_ERR_SHAPE;
+    if (!aligned16(L->U) || !aligned16(L->V) || !aligned16(L->s1) || !aligned16(L->s2)) return NQ_ERR_ALIGN;
+    return NQ_OK;
+}
+
+nq_status check_io(const uint16_t* x, const uint16_t* y, void* ws) {
+    if (!x || !y || !ws) return NQ_ERR_NULL;
+    if (!aligned16(x) || !aligned16(y) || !aligned16(ws)) return NQ_ERR_ALIGN;
+    return NQ_OK;
+}
+
+}  // namespace
+
+namespace nq_host {
+
+int sm_count() {
+    DeviceInfo* d = current_device();
+    return (d && d->sms > 0) ? d->sms : 148;
+}
+
+unsigned int* error_word() {
+    DeviceInfo* d = current_device();
+    return d ? d->err : nullptr;
+}
+
+cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem, cudaStream_t s, void** args, bool pdl) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    cudaError_t e = cudaLaunchKernelExC(&cfg, fn, args);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+}  // namespace nq_host
+
+extern "C" {
+
+const char* nq_status_string(nq_status s) {
+    switch (s) {
+        case NQ_OK: return "NQ_OK";
+        case NQ_ERR_NULL: return "NQ_ERR_NULL: a required pointer is NULL";
+        case NQ_ERR_SHAPE: return "NQ_ERR_SHAPE: invalid size, rank or leading dimension";
+        case NQ_ERR_ALIGN: return "NQ_ERR_ALIGN: a pointer is not 16-byte aligned";
+        case NQ_ERR_WORKSPACE: return "NQ_ERR_WORKSPACE: workspace missing or too small";
+        case NQ_ERR_DEVICE: return "NQ_ERR_DEVICE: current device is not sm_100 (B200)";
+        case NQ_ERR_LAUNCH: return "NQ_ERR_LAUNCH: kernel launch or asynchronous CUDA error";
+        case NQ_ERR_TIMEOUT: return "NQ_ERR_TIMEOUT: a bounded device-side wait gave up";
+    }
+    return "unknown nq_status";
+}
+
+const char* nq_version(void) { return "libnq 0.1 sm_100a"; }
+
+nq_status nq_pack_signs(const float* latent, int64_t rows, int64_t r, int64_t ld_latent, uint32_t* packed,
+                        int64_t ld_words, void* stream) {
+    if (rows < 0 || r < 0 || (r % 32) != 0 || ld_latent < r || ld_words < r / 32) return NQ_ERR_SHAPE;
+    if (rows == 0 || ld_words == 0) return NQ_OK;
+    if (!packed || (r > 0 && !latent)) return NQ_ERR_NULL;
+    if (!aligned16(packed) || (latent && !aligned16(latent))) return NQ_ERR_ALIGN;
+    DeviceInfo* d = current_device();
+    if (!d || !d->ok) return NQ_ERR_DEVICE;
+    return nq_launch_pack(latent, rows, r, ld_latent, packed, ld_words, static_cast<cudaStream_t>(stream));
+}
+
+size_t nq_workspace_bytes(const nq_lrb_layer* L, int64_t M) {
+    if (check_layer(L) != NQ_OK || M < 1) return 0;
+    size_t bytes = nq_prefill_workspace_bytes(L, M);
+    if (M <= NQ_MATVEC_MAX_M) {
+        const size_t dec = nq_decode_workspace_bytes(L->d_in, L->r, M);
+        if (dec > bytes) bytes = dec;
+    }
+    return bytes;
+}
+
+nq_status nq_lrb_matvec(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y, int64_t M, void* ws,
+                        size_t ws_bytes, void* stream) {
+    nq_status st = check_layer(L);
+    if (st != NQ_OK) return st;
+    if (M < 1 || M > NQ_MATVEC_MAX_M) return NQ_ERR_SHAPE;
+    if (nq_decode_stage2_smem(L->r, M) > kMaxDecodeSmem) return NQ_ERR_SHAPE;
+    if ((st = check_io(x, y, ws)) != NQ_OK) return st;
+    if (ws_bytes < nq_decode_workspace_bytes(L->d_in, L->r, M)) return NQ_ERR_WORKSPACE;
+    DeviceInfo* d = current_device();
+    if (!d || !d->ok) return NQ_ERR_DEVICE;
+    return nq_launch_decode(L, x, y, M, ws, static_cast<cudaStream_t>(stream), pdl_enabled());
+}
+
+nq_status nq_lrb_matmul(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y, int64_t M, void* ws,
+                        size_t ws_bytes, void* stream) {
+    nq_status st = check_layer(L);
+    if (st != NQ_OK) return st;
+    if (M < 1) return NQ_ERR_SHAPE;
+    if ((st = check_io(x, y, ws)) != NQ_OK) return st;
+    if (ws_bytes < nq_prefill_workspace_bytes(L, M)) return NQ_ERR_WORKSPACE;
+    DeviceInfo* d = current_device();
+    if (!d || !d->ok) return NQ_ERR_DEVICE;
+    return nq_launch_prefill(L, x, y, M, ws, static_cast<cudaStream_t>(stream), pdl_enabled());
+}
+
+nq_status nq_layer_forward(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y, int64_t M, void* ws,
+                           size_t ws_bytes, void* stream) {
+    if (M >= 1 && M <= NQ_MATVEC_MAX_M) return nq_lrb_matvec(L, x, y, M, ws, ws_bytes, stream);
+    return nq_lrb_matmul(L, x, y, M, ws, ws_bytes, stream);
+}
+
+nq_status nq_silu_mul(const uint16_t* g, const uint16_t* u, uint16_t* h, int64_t n, void* stream) {
+    if (n < 0) return NQ_ERR_SHAPE;
+    if (n == 0) return NQ_OK;
+    if (!g || !u || !h) return NQ_ERR_NULL;
+    if (!aligned16(g) || !aligned16(u) || !aligned16(h)) return NQ_ERR_ALIGN;
+    DeviceInfo* d = current_device();
+    if (!d || !d->ok) return NQ_ERR_DEVICE;
+    return nq_launch_silu_mul(g, u, h, n, static_cast<cudaStream_t>(stream), pdl_enabled());
+}
+
+nq_status nq_sync_status(void* stream) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return NQ_ERR_LAUNCH;
+    unsigned int word = 0u;
+    if (cudaMemcpyFromSymbol(&word, nq::g_error_word, sizeof word) != cudaSuccess) return NQ_ERR_LAUNCH;
+    if (word != 0u) {
+        const unsigned int zero = 0u;
+        cudaMemcpyToSymbol(nq::g_error_word, &zero, sizeof zero);
+        if (word & nq::kErrTimeout) return NQ_ERR_TIMEOUT;
+    }
+    return NQ_OK;
+}
+
+}  // extern "C"

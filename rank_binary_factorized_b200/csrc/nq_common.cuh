@@ -1,0 +1,63 @@
+// nq_common.cuh -- device-side helpers shared by the libnq kernels (sm_100a only).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "nq.h"
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ != 1000)
+#error "libnq is written for sm_100a (B200) only"
+#endif
+
+// Every workspace starts with this many bytes of counters owned by the decode path (zero
+// between calls); the rest is per-call scratch.  Bounds the word-chunk count of stage 1.
+#define NQ_WS_HEADER_BYTES 4096
+#define NQ_MAX_RANK (NQ_WS_HEADER_BYTES / 4 * 8 * 32)
+static_assert(NQ_MAX_RANK == NQ_MAX_RANK_LIMIT, "rank limit of nq.h and the ticket header disagree");
+
+namespace nq {
+
+// Device error word (one per device that loads the library, defined in api.cu; kernels get
+// its address as an argument).  Set with atomicOr by a kernel whose bounded wait gave up,
+// read and cleared by nq_sync_status.
+constexpr unsigned int kErrTimeout = 1u;
+
+// Iteration cap for every spin-wait on device (each iteration sleeps ~128 ns with
+// __nanosleep after the first few polls; 2^22 polls is well over a second).
+constexpr unsigned int kSpinLimit = 1u << 22;
+
+__device__ __forceinline__ void flag_error(unsigned int* word, unsigned int bits) { atomicOr(word, bits); }
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
+    return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+__device__ __forceinline__ float f16_bits_to_float(uint16_t h) {
+    return __half2float(__ushort_as_half(h));
+}
+
+// fp32 -> bf16, round to nearest even (the CUDA intrinsic).
+__device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
+    return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+
+// Programmatic dependent launch: wait for the grid queued before this one to finish and
+// publish its memory, and let the next grid start its prologue.  Both are no-ops when the
+// kernel was launched without the programmatic-serialisation attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+}  // namespace nq
+
+// Host-side launch plumbing shared by the translation units (defined in api.cu).
+namespace nq_host {
+int sm_count();                                   // multiprocessors of the current device
+unsigned int* error_word();                       // device address of the error word
+cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem, cudaStream_t s, void** args,
+                       bool pdl);
+}  // namespace nq_host

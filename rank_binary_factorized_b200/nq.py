@@ -1,0 +1,181 @@
+"""Thin Python binding of libnq.so (include/nq.h) -- argument marshalling only.
+
+Every step of the LRB path runs in the CUDA library; this module turns torch tensors into
+device pointers and the current torch stream into a ``cudaStream_t``.  PyTorch provides
+device memory and streams, nothing else.  If ``libnq.so`` is missing the import fails: there
+is no other implementation to fall back to.
+
+Tensor conventions (device tensors, contiguous):
+  packed signs  int32 [rows][ld] (the bits of uint32 words)
+  s1, s2        float16 [d_out], [d_in]
+  x, y          bfloat16 [M][d_in], [M][d_out]
+  latent        float32 [rows][ld_latent]
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libnq.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError("libnq.so is not built (python -m rank_binary_factorized_b200.build): " + LIB_PATH)
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+NQ_OK = 0
+STATUS_NAMES = {0: "NQ_OK", 1: "NQ_ERR_NULL", 2: "NQ_ERR_SHAPE", 3: "NQ_ERR_ALIGN", 4: "NQ_ERR_WORKSPACE",
+                5: "NQ_ERR_DEVICE", 6: "NQ_ERR_LAUNCH", 7: "NQ_ERR_TIMEOUT"}
+MATVEC_MAX_M = 8
+
+_i64 = ctypes.c_int64
+_p = ctypes.c_void_p
+
+
+class nq_lrb_layer(ctypes.Structure):
+    _fields_ = [("d_out", _i64), ("d_in", _i64), ("r", _i64), ("U", _p), ("ldu", _i64), ("V", _p), ("ldv", _i64),
+                ("s1", _p), ("s2", _p)]
+
+
+_lib.nq_pack_signs.restype = ctypes.c_int
+_lib.nq_pack_signs.argtypes = [_p, _i64, _i64, _i64, _p, _i64, _p]
+_lib.nq_workspace_bytes.restype = ctypes.c_size_t
+_lib.nq_workspace_bytes.argtypes = [ctypes.POINTER(nq_lrb_layer), _i64]
+for _name in ("nq_lrb_matvec", "nq_lrb_matmul", "nq_layer_forward"):
+    getattr(_lib, _name).restype = ctypes.c_int
+    getattr(_lib, _name).argtypes = [ctypes.POINTER(nq_lrb_layer), _p, _p, _i64, _p, ctypes.c_size_t, _p]
+_lib.nq_silu_mul.restype = ctypes.c_int
+_lib.nq_silu_mul.argtypes = [_p, _p, _p, _i64, _p]
+_lib.nq_sync_status.restype = ctypes.c_int
+_lib.nq_sync_status.argtypes = [_p]
+_lib.nq_status_string.restype = ctypes.c_char_p
+_lib.nq_status_string.argtypes = [ctypes.c_int]
+_lib.nq_version.restype = ctypes.c_char_p
+_lib.nq_version.argtypes = []
+
+
+class NQError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__("%s: %s" % (fn, _lib.nq_status_string(status).decode()))
+
+
+def _check(fn: str, status: int) -> None:
+    if status != NQ_OK:
+        raise NQError(fn, status)
+
+
+def version() -> str:
+    return _lib.nq_version().decode()
+
+
+def status_string(status: int) -> str:
+    return _lib.nq_status_string(status).decode()
+
+
+def _stream_ptr(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def _ptr(t) -> int:
+    return 0 if t is None else int(t.data_ptr())
+
+
+class Layer:
+    """A device-resident LRB layer: packed U, V (int32 words), fp16 s1, s2."""
+
+    def __init__(self, U: torch.Tensor, V: torch.Tensor, s1: torch.Tensor, s2: torch.Tensor, r: int):
+        self.U, self.V, self.s1, self.s2 = U, V, s1, s2
+        self.d_out, self.ldu = int(U.shape[0]), int(U.shape[1])
+        self.d_in, self.ldv = int(V.shape[0]), int(V.shape[1])
+        self.r = int(r)
+        self.struct = nq_lrb_layer(self.d_out, self.d_in, self.r, _ptr(U), self.ldu, _ptr(V), self.ldv, _ptr(s1),
+                                   _ptr(s2))
+        self._ws = {}
+
+    @classmethod
+    def from_host(cls, U, V, s1_bits, s2_bits, r: int, device="cuda") -> "Layer":
+        """From numpy arrays: uint32 words and fp16 bit patterns (uint16)."""
+        import numpy as np
+
+        def dev(a, dt):
+            return torch.from_numpy(np.ascontiguousarray(a).view(dt)).to(device)
+
+        return cls(dev(U, np.int32), dev(V, np.int32), dev(s1_bits, np.float16), dev(s2_bits, np.float16), r)
+
+    def workspace_bytes(self, M: int) -> int:
+        return int(_lib.nq_workspace_bytes(ctypes.byref(self.struct), M))
+
+    def workspace(self, M: int) -> torch.Tensor:
+        """A zero-filled workspace large enough for M rows (cached per size)."""
+        need = self.workspace_bytes(M)
+        if need == 0:
+            raise NQError("nq_workspace_bytes", 2)
+        ws = self._ws.get("ws")
+        if ws is None or ws.numel() < need:
+            ws = torch.zeros(max(need, 256), dtype=torch.uint8, device=self.U.device)
+            self._ws["ws"] = ws
+        return ws
+
+    @property
+    def storage_bytes(self) -> int:
+        return 4 * (self.d_out + self.d_in) * self.r // 32 + 2 * (self.d_out + self.d_in)
+
+
+def pack_signs(latent: torch.Tensor, r: int | None = None, ld_words: int | None = None, out=None,
+               stream=None) -> torch.Tensor:
+    """sign(latent) >= 0 packed 32 per word along r (bit k%32 of word k/32)."""
+    if latent.dim() != 2 or latent.stride(1) != 1 or latent.dtype != torch.float32:
+        raise ValueError("latent must be a 2-D float32 tensor with unit column stride")
+    rows, ld_latent = int(latent.shape[0]), int(latent.stride(0))
+    r = int(latent.shape[1]) if r is None else int(r)
+    ld_words = r // 32 if ld_words is None else int(ld_words)
+    if out is None:
+        out = torch.empty((rows, ld_words), dtype=torch.int32, device=latent.device)
+    _check("nq_pack_signs", _lib.nq_pack_signs(_ptr(latent), rows, r, ld_latent, _ptr(out), ld_words,
+                                               _stream_ptr(stream)))
+    return out
+
+
+def _forward(fn_name: str, layer: Layer, x: torch.Tensor, y=None, ws=None, stream=None) -> torch.Tensor:
+    M = int(x.shape[0])
+    if y is None:
+        y = torch.empty((M, layer.d_out), dtype=torch.bfloat16, device=x.device)
+    if ws is None:
+        ws = layer.workspace(M)
+    fn = getattr(_lib, fn_name)
+    _check(fn_name, fn(ctypes.byref(layer.struct), _ptr(x), _ptr(y), M, _ptr(ws), ws.numel(), _stream_ptr(stream)))
+    return y
+
+
+def lrb_matvec(layer: Layer, x: torch.Tensor, y=None, ws=None, stream=None) -> torch.Tensor:
+    return _forward("nq_lrb_matvec", layer, x, y, ws, stream)
+
+
+def lrb_matmul(layer: Layer, x: torch.Tensor, y=None, ws=None, stream=None) -> torch.Tensor:
+    return _forward("nq_lrb_matmul", layer, x, y, ws, stream)
+
+
+def layer_forward(layer: Layer, x: torch.Tensor, y=None, ws=None, stream=None) -> torch.Tensor:
+    return _forward("nq_layer_forward", layer, x, y, ws, stream)
+
+
+def silu_mul(g: torch.Tensor, u: torch.Tensor, h=None, stream=None) -> torch.Tensor:
+    if h is None:
+        h = torch.empty_like(g)
+    _check("nq_silu_mul", _lib.nq_silu_mul(_ptr(g), _ptr(u), _ptr(h), g.numel(), _stream_ptr(stream)))
+    return h
+
+
+def sync_status(stream=None) -> None:
+    _check("nq_sync_status", _lib.nq_sync_status(_stream_ptr(stream)))
+
+
+def raw_lib() -> ctypes.CDLL:
+    """The loaded libnq.so (for callers that marshal arguments themselves)."""
+    return _lib

@@ -1,0 +1,121 @@
+"""The C ABI: libnq.so loads, exports every entry point include/nq.h declares, and rejects
+bad arguments on the host with the documented status before anything is launched.
+
+No compute call runs here: every call below fails validation (or, on a machine without a
+GPU, the device check), so no pointer is ever dereferenced.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "nq.h")
+
+NQ = dict(OK=0, NULL=1, SHAPE=2, ALIGN=3, WORKSPACE=4, DEVICE=5, LAUNCH=6, TIMEOUT=7)
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"NQ_API\s+[\w\s\*]+?\b(nq_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def nq():
+    from rank_binary_factorized_b200 import nq as mod
+    return mod
+
+
+def test_header_declares_the_entry_points():
+    syms = declared_symbols()
+    for name in ["nq_pack_signs", "nq_lrb_matvec", "nq_lrb_matmul", "nq_layer_forward", "nq_workspace_bytes",
+                 "nq_silu_mul", "nq_sync_status", "nq_status_string"]:
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol(nq):
+    lib = ctypes.CDLL(nq.LIB_PATH)
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    # and nothing else with the nq_ prefix leaks out undocumented
+    out = os.popen("nm -D --defined-only %s" % nq.LIB_PATH).read()
+    exported = set(re.findall(r" T (nq_\w+)", out))
+    assert exported == set(declared_symbols())
+
+
+def test_status_strings_and_version(nq):
+    for code, name in nq.STATUS_NAMES.items():
+        assert nq.status_string(code).startswith(name)
+    assert "sm_100a" in nq.version()
+
+
+def _layer(nq, d_out=64, d_in=96, r=64, ldu=None, ldv=None, U=0x10000, V=0x20000, s1=0x30000, s2=0x40000):
+    return nq.nq_lrb_layer(d_out, d_in, r, U, ldu if ldu is not None else r // 32, V,
+                           ldv if ldv is not None else r // 32, s1, s2)
+
+
+def _call(nq, fn, L, x=0x50000, y=0x60000, M=1, ws=0x70000, ws_bytes=1 << 30):
+    lib = nq.raw_lib()
+    return getattr(lib, fn)(ctypes.byref(L) if L is not None else None, x, y, M, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("fn", ["nq_lrb_matvec", "nq_lrb_matmul", "nq_layer_forward"])
+def test_forward_argument_errors(nq, fn):
+    assert _call(nq, fn, None) == NQ["NULL"]
+    assert _call(nq, fn, _layer(nq, U=0)) == NQ["NULL"]
+    assert _call(nq, fn, _layer(nq), x=0) == NQ["NULL"]
+    assert _call(nq, fn, _layer(nq), ws=0) == NQ["NULL"]
+    assert _call(nq, fn, _layer(nq, r=48)) == NQ["SHAPE"]  # r % 32 != 0
+    assert _call(nq, fn, _layer(nq, r=0)) == NQ["SHAPE"]
+    assert _call(nq, fn, _layer(nq, d_out=0)) == NQ["SHAPE"]
+    assert _call(nq, fn, _layer(nq, d_in=-3)) == NQ["SHAPE"]
+    assert _call(nq, fn, _layer(nq, ldu=1)) == NQ["SHAPE"]  # ld below r/32
+    assert _call(nq, fn, _layer(nq, ldv=1)) == NQ["SHAPE"]
+    assert _call(nq, fn, _layer(nq, r=262144 + 32, ldu=8193, ldv=8193)) == NQ["SHAPE"]  # above NQ_MAX_RANK_LIMIT
+    assert _call(nq, fn, _layer(nq), M=0) == NQ["SHAPE"]
+    assert _call(nq, fn, _layer(nq, V=0x20004)) == NQ["ALIGN"]
+    assert _call(nq, fn, _layer(nq), x=0x50002) == NQ["ALIGN"]
+    assert _call(nq, fn, _layer(nq), ws_bytes=16) == NQ["WORKSPACE"]
+
+
+def test_matvec_rejects_large_batch(nq):
+    assert _call(nq, "nq_lrb_matvec", _layer(nq), M=nq.MATVEC_MAX_M + 1) == NQ["SHAPE"]
+
+
+def test_workspace_bytes(nq):
+    lib = nq.raw_lib()
+    L = _layer(nq)
+    for M in (1, 8, 9, 64, 2048):
+        assert lib.nq_workspace_bytes(ctypes.byref(L), M) > 0
+    assert lib.nq_workspace_bytes(ctypes.byref(L), 0) == 0
+    assert lib.nq_workspace_bytes(ctypes.byref(_layer(nq, r=40)), 1) == 0
+
+
+def test_pack_argument_errors(nq):
+    lib = nq.raw_lib()
+    assert lib.nq_pack_signs(0x1000, 4, 48, 48, 0x2000, 2, None) == NQ["SHAPE"]  # r % 32
+    assert lib.nq_pack_signs(0x1000, 4, 64, 32, 0x2000, 2, None) == NQ["SHAPE"]  # ld_latent < r
+    assert lib.nq_pack_signs(0x1000, 4, 64, 64, 0x2000, 1, None) == NQ["SHAPE"]  # ld_words < r/32
+    assert lib.nq_pack_signs(0x1000, -1, 64, 64, 0x2000, 2, None) == NQ["SHAPE"]
+    assert lib.nq_pack_signs(0x1000, 0, 64, 64, 0x2000, 2, None) == NQ["OK"]  # empty: no-op
+    assert lib.nq_pack_signs(0, 4, 64, 64, 0x2000, 2, None) == NQ["NULL"]
+    assert lib.nq_pack_signs(0x1000, 4, 64, 64, 0, 2, None) == NQ["NULL"]
+    assert lib.nq_pack_signs(0x1004, 4, 64, 64, 0x2000, 2, None) == NQ["ALIGN"]
+
+
+def test_silu_argument_errors(nq):
+    lib = nq.raw_lib()
+    assert lib.nq_silu_mul(0x1000, 0x2000, 0x3000, -1, None) == NQ["SHAPE"]
+    assert lib.nq_silu_mul(0x1000, 0x2000, 0x3000, 0, None) == NQ["OK"]
+    assert lib.nq_silu_mul(0, 0x2000, 0x3000, 8, None) == NQ["NULL"]
+    assert lib.nq_silu_mul(0x1000, 0x2002, 0x3000, 8, None) == NQ["ALIGN"]
+
+
+def test_no_gpu_gives_device_error(nq):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present; this checks the CPU-only path")
+    # valid arguments, no device: the call must refuse, not fall back to anything
+    assert _call(nq, "nq_lrb_matvec", _layer(nq)) == NQ["DEVICE"]
+    assert nq.raw_lib().nq_pack_signs(0x1000, 4, 64, 64, 0x2000, 2, None) == NQ["DEVICE"]

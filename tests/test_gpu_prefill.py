@@ -1,0 +1,118 @@
+"""Prefill path (nq_lrb_matmul, tcgen05 tensor cores) against the CPU oracle.
+
+- floating parity at the stated tolerance on ragged shapes (d_out, r, d_in and M not
+  multiples of the 128 x 64 x 256 tiles) and on the 70B gate projection at M = 64, 512,
+  2048 (sampled outputs, the launch the benchmark times);
+- integer-exact regime: s1 = s2 = 1, x in {-1, 0, 1} and |t| <= 2048, where every fp16
+  operand and intermediate is an exact integer, so the GPU must equal bf16(y_ref) bitwise;
+- every 4 x 2 sign pattern (stacked, r = 32 with cancelling pad columns), bitwise.
+"""
+import itertools
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from rank_binary_factorized_b200 import synth
+from tests.gpu_util import (check_tolerance, download_bf16_bits, need_gpu, nq, upload_bf16, upload_projection)
+
+pytestmark = pytest.mark.gpu
+
+
+def gpu_matmul(p, xb, fn="lrb_matmul"):
+    L = upload_projection(p)
+    y = getattr(nq(), fn)(L, upload_bf16(xb))
+    nq().sync_status()
+    return download_bf16_bits(y)
+
+
+@pytest.mark.parametrize("M", [9, 16, 64, 100, 256, 300])
+def test_tiny_layer_token_counts(M):
+    need_gpu()
+    p = synth.make_workload("tiny")[0]
+    xb = synth.make_input("tiny", p.d_in, M, key=100 + M)
+    y = gpu_matmul(p, xb)
+    y_ref, S = oracle.dense_packed(p.U, p.V, p.s1, p.s2, p.r, xb)
+    check_tolerance(y, y_ref, S, "prefill tiny M=%d" % M)
+
+
+@pytest.mark.parametrize("d_out,d_in,r,ldu,ldv,M", [
+    (77, 1000, 96, 3, 3, 20),
+    (300, 2049, 320, 10, 11, 70),
+    (129, 64, 160, 5, 8, 257),
+    (1, 8, 32, 1, 1, 9),
+    (640, 200, 2048, 64, 66, 33),
+])
+def test_ragged_and_padded(d_out, d_in, r, ldu, ldv, M):
+    need_gpu()
+    p = synth.make_projection("ragged", d_out, d_in, r, seed=402, key=d_out + 3 * d_in, ldu=ldu, ldv=ldv)
+    xb = synth.acts_bf16(synth.rng_for(403, d_in, M), (M, d_in))
+    y = gpu_matmul(p, xb)
+    y_ref, S = oracle.dense_packed(p.U, p.V, p.s1, p.s2, p.r, xb)
+    check_tolerance(y, y_ref, S, "prefill ragged %r" % ((d_out, d_in, r, ldu, ldv, M),))
+
+
+@pytest.mark.parametrize("d_out,d_in,r,M", [(256, 512, 128, 64), (1024, 2048, 512, 300), (4096, 1024, 1024, 40)])
+def test_integer_exact_bitwise(d_out, d_in, r, M):
+    need_gpu()
+    p = synth.make_projection("int", d_out, d_in, r, seed=404, key=d_out + M)
+    p.s1 = np.full(d_out, 0x3C00, dtype=np.uint16)
+    p.s2 = np.full(d_in, 0x3C00, dtype=np.uint16)
+    xi = synth.rng_for(405, d_out, M).integers(-1, 2, size=(M, d_in)).astype(np.float32)
+    xb = synth.f32_to_bf16_bits(xi)
+    y = gpu_matmul(p, xb)
+    rows = np.arange(d_out) if d_out <= 1024 else np.linspace(0, d_out - 1, 300).astype(np.int64)
+    y_ref, _ = oracle.dense_packed(p.U, p.V, p.s1, p.s2, p.r, xb, rows=rows)
+    np.testing.assert_array_equal(y[:, rows], oracle.round_bf16(y_ref))
+
+
+def test_every_sign_pattern_4x2_bitwise():
+    need_gpu()
+    pats = np.array(list(itertools.product([-1, 1], repeat=8)), dtype=np.int8).reshape(256 * 4, 2)
+
+    def words(S, pad):
+        w = np.zeros(S.shape[0], dtype=np.uint32)
+        for k in range(2):
+            w |= (S[:, k] > 0).astype(np.uint32) << np.uint32(k)
+        return (w | np.uint32(pad)).reshape(-1, 1)
+
+    p = synth.Projection("patterns", 1024, 1024, 32, words(pats, 0xFFFFFFFC), words(pats, 0x0001FFFC),
+                         np.full(1024, 0x3C00, dtype=np.uint16), np.full(1024, 0x3C00, dtype=np.uint16))
+    xi = synth.rng_for(406).integers(-1, 2, size=(24, 1024)).astype(np.float32)
+    xb = synth.f32_to_bf16_bits(xi)
+    y = gpu_matmul(p, xb)
+    y_ref, _ = oracle.dense_packed(p.U, p.V, p.s1, p.s2, 32, xb)
+    np.testing.assert_array_equal(y, oracle.round_bf16(y_ref))
+
+
+@pytest.mark.parametrize("M", [64, 512, 2048])
+def test_full_size_70b_gate_sampled(M):
+    """The 70B gate projection (28672 x 8192, r = 3520) at the benchmark's token counts;
+    sampled output features for every token."""
+    need_gpu()
+    p = synth.make_workload("prefill70b")[0]
+    xb = synth.make_input("prefill70b", p.d_in, M, key=M)
+    y = gpu_matmul(p, xb)
+    rows = np.unique(np.concatenate([[0, 127, 128, p.d_out - 1], np.linspace(0, p.d_out - 1, 40).astype(np.int64)]))
+    y_ref, S = oracle.dense_packed(p.U, p.V, p.s1, p.s2, p.r, xb, rows=rows)
+    check_tolerance(y[:, rows], y_ref, S, "prefill 70B gate M=%d" % M)
+
+
+def test_layer_forward_dispatches_to_matmul_and_is_deterministic():
+    need_gpu()
+    p = synth.make_workload("tiny")[0]
+    xb = synth.make_input("tiny", p.d_in, 33, key=7)
+    y1 = gpu_matmul(p, xb, fn="layer_forward")
+    y2 = gpu_matmul(p, xb, fn="lrb_matmul")
+    np.testing.assert_array_equal(y1, y2)
+
+
+def test_matmul_small_m_matches_matvec_tolerance():
+    """nq_lrb_matmul accepts M <= 8 too (the tensor-core path with a 16-token tile)."""
+    need_gpu()
+    p = synth.make_workload("tiny")[0]
+    xb = synth.make_input("tiny", p.d_in, 3, key=8)
+    y = gpu_matmul(p, xb)
+    y_ref, S = oracle.dense_packed(p.U, p.V, p.s1, p.s2, p.r, xb)
+    check_tolerance(y, y_ref, S, "prefill M=3")
