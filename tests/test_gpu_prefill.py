@@ -116,3 +116,21 @@ def test_matmul_small_m_matches_matvec_tolerance():
     y = gpu_matmul(p, xb)
     y_ref, S = oracle.dense_packed(p.U, p.V, p.s1, p.s2, p.r, xb)
     check_tolerance(y, y_ref, S, "prefill M=3")
+
+
+def test_one_workspace_shared_by_decode_and_prefill():
+    """Decode and prefill calls of different shapes share one zero-initialised workspace."""
+    need_gpu()
+    p = synth.make_projection("shared", 640, 1536, 256, seed=407, key=1)
+    L = upload_projection(p)
+    need = max(L.workspace_bytes(M) for M in (1, 8, 300))
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    outs = []
+    for M in (1, 300, 8, 77, 3, 300, 1):
+        xb = synth.acts_bf16(synth.rng_for(408, M), (M, p.d_in))
+        y = nq().layer_forward(L, upload_bf16(xb), ws=ws)
+        outs.append((xb, y))
+    nq().sync_status()
+    for xb, y in outs:
+        y_ref, S = oracle.dense_packed(p.U, p.V, p.s1, p.s2, p.r, xb)
+        check_tolerance(download_bf16_bits(y), y_ref, S, "shared workspace M=%d" % xb.shape[0])
