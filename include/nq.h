@@ -63,7 +63,8 @@ typedef enum nq_status {
     NQ_ERR_WORKSPACE = 4, /* workspace NULL or smaller than nq_workspace_bytes() */
     NQ_ERR_DEVICE = 5,    /* current device is not compute capability 10.0 (B200) */
     NQ_ERR_LAUNCH = 6,    /* a kernel launch failed */
-    NQ_ERR_TIMEOUT = 7    /* a bounded device-side wait gave up (seen by nq_sync_status) */
+    NQ_ERR_TIMEOUT = 7,   /* a bounded device-side wait gave up (seen by nq_sync_status) */
+    NQ_ERR_SCRATCH_LIMIT = 8 /* nq_lrb_matvec_noalloc: the call needs more than NQ_NOALLOC_SCRATCH_BYTES */
 } nq_status;
 
 /* One LRB linear layer.  All pointers are device pointers; the struct itself is host
@@ -148,6 +149,29 @@ NQ_API nq_status nq_silu_mul(const uint16_t* g, const uint16_t* u, uint16_t* h, 
  * NQ_ERR_LAUNCH if the stream reported an asynchronous CUDA error, NQ_OK otherwise.
  */
 NQ_API nq_status nq_sync_status(void* stream);
+
+/*
+ * nq_lrb_matvec_noalloc -- nq_lrb_matvec for callers that cannot allocate device memory.
+ * The pages have no counterpart to this entry point; it exists for deployment.  Callers
+ * that cannot hand over a workspace: plug-ins that an inference engine gives only their
+ * input and output tensors, code issued while a stream is being captured into a CUDA graph
+ * (cudaMalloc is not a stream operation and may synchronise the device), latency-critical
+ * loops that cannot take an allocator round trip, plain C callers without an allocator.
+ * Same operation, arguments and numerics as nq_lrb_matvec, minus the workspace: the
+ * scratch (stage-1 tickets, t and the per-slice partials) lives in one statically sized
+ * array of NQ_NOALLOC_SCRATCH_BYTES inside libnq.so, which every GPU that loads the library
+ * holds until the process exits.  A call whose scratch need (nq_workspace_bytes for the same
+ * layer and M <= 8) exceeds that size returns NQ_ERR_SCRATCH_LIMIT without launching.
+ * The first call on a device looks up the array's device address (set-up, once per
+ * device, on the calling thread with that device current); make that first call before
+ * any stream capture.  Every call clears the ticket header on `stream` before launching.
+ * All calls on a device share the one array: calls that can overlap on the GPU (different
+ * streams, or the same stream without ordering) race and must be serialised by the caller.
+ * Never calls cudaMalloc, cudaFree or any allocating routine.
+ */
+#define NQ_NOALLOC_SCRATCH_BYTES (2u * 1024u * 1024u)
+NQ_API nq_status nq_lrb_matvec_noalloc(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y, int64_t M,
+                                       void* stream);
 
 /* Human-readable name of a status code (static storage). */
 NQ_API const char* nq_status_string(nq_status s);

@@ -118,6 +118,8 @@ const char* nq_status_string(nq_status s) {
         case NQ_ERR_DEVICE: return "NQ_ERR_DEVICE: current device is not sm_100 (B200)";
         case NQ_ERR_LAUNCH: return "NQ_ERR_LAUNCH: kernel launch or asynchronous CUDA error";
         case NQ_ERR_TIMEOUT: return "NQ_ERR_TIMEOUT: a bounded device-side wait gave up";
+        case NQ_ERR_SCRATCH_LIMIT:
+            return "NQ_ERR_SCRATCH_LIMIT: the call needs more scratch than nq_lrb_matvec_noalloc's static array";
     }
     return "unknown nq_status";
 }

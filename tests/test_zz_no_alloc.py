@@ -1,0 +1,79 @@
+"""nq_lrb_matvec_noalloc: the decode entry point for callers that cannot allocate device
+memory (engine plug-ins handed only their tensors, code issued during graph capture,
+allocator-free C callers).  Its scratch is a static array inside libnq.so.
+
+Called here through the C ABI with ctypes, twice in a row per layer (the second call runs
+on the scratch the first one left behind), and checked against nq_lrb_matvec -- the entry
+point that takes a caller workspace -- within the parity tolerance of the other tests.
+This file is collected last so that a run stopping at the first failure has already run
+every other test; it also passes on its own in a fresh process (the first call does the
+per-device set-up).
+"""
+import ctypes
+
+import numpy as np
+import pytest
+
+import oracle
+from rank_binary_factorized_b200 import synth
+from tests.gpu_util import (REL, ABS, bf16_bits_to_f64, download_bf16_bits, half_ulp_bf16, need_gpu, nq,
+                            upload_bf16, upload_projection)
+
+pytestmark = pytest.mark.gpu
+
+NQ_ERR_SCRATCH_LIMIT = 8
+
+
+def noalloc_fn():
+    mod = nq()
+    fn = mod.raw_lib().nq_lrb_matvec_noalloc
+    fn.restype = ctypes.c_int
+    fn.argtypes = [ctypes.POINTER(mod.nq_lrb_layer), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                   ctypes.c_void_p]
+    return fn
+
+
+@pytest.mark.parametrize("workload,M", [("tiny", 1), ("attn7b", 1), ("attn7b", 8), ("layer70b", 1)])
+def test_noalloc_matches_workspace_entry_point_on_two_calls(workload, M):
+    need_gpu()
+    import torch
+    mod = nq()
+    fn = noalloc_fn()
+    projs = synth.make_workload(workload)
+    p = projs[-1]  # layer70b: the down projection (d_in = 28672, the largest stage 1)
+    L = upload_projection(p)
+    stream = torch.cuda.current_stream()
+    for call in range(2):
+        xb = synth.make_input(workload, p.d_in, M, key=500 + call)
+        x = upload_bf16(xb)
+        y_ws = mod.lrb_matvec(L, x)  # existing entry point, caller workspace
+        y_na = torch.empty_like(y_ws)
+        st = fn(ctypes.byref(L.struct), x.data_ptr(), y_na.data_ptr(), M, ctypes.c_void_p(stream.cuda_stream))
+        assert st == 0, mod.status_string(st)
+        mod.sync_status()
+        got = bf16_bits_to_f64(download_bf16_bits(y_na))
+        want = bf16_bits_to_f64(download_bf16_bits(y_ws))
+        rows = np.linspace(0, p.d_out - 1, 64).astype(np.int64)
+        _, S = oracle.dense_packed(p.U, p.V, p.s1, p.s2, p.r, xb, rows=rows)
+        tol = REL * S + ABS + half_ulp_bf16(want[:, rows])
+        assert np.all(np.abs(got[:, rows] - want[:, rows]) <= tol), "call %d" % call
+        # the scale of S is the same across rows; hold every row to the sampled bound
+        assert np.all(np.abs(got - want) <= REL * np.median(S, axis=1, keepdims=True) + ABS
+                      + half_ulp_bf16(want)), "call %d, all rows" % call
+
+
+def test_noalloc_rejects_sizes_beyond_its_scratch():
+    need_gpu()
+    mod = nq()
+    fn = noalloc_fn()
+    # M = 2 at r = 24576 over d_in = 32768: t plus the stage-1 partials need several MB,
+    # more than NQ_NOALLOC_SCRATCH_BYTES (2 MiB); the call must refuse before launching
+    M = 2
+    p = synth.make_projection("big", 64, 32768, 24576, seed=501)
+    L = upload_projection(p)
+    x = upload_bf16(synth.acts_bf16(synth.rng_for(502), (M, p.d_in)))
+    y = upload_bf16(np.zeros((M, p.d_out), dtype=np.uint16))
+    assert L.workspace_bytes(M) > 2 * 1024 * 1024
+    st = fn(ctypes.byref(L.struct), x.data_ptr(), y.data_ptr(), M, None)
+    assert st == NQ_ERR_SCRATCH_LIMIT
+    assert "scratch" in mod.status_string(st)
