@@ -46,6 +46,9 @@ def parse_args():
     ap.add_argument("--impl", choices=["nq", "reference"], default="nq")
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--headline-only", action="store_true", help="skip the other workloads")
+    ap.add_argument("--only", default=None,
+                    help="run just these extra sections (comma list of attn7b_b8, mlp7b, layer70b, prefill, pack) "
+                         "after the headline; implies no CPU baseline")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU oracle sample budget")
     return ap.parse_args()
 
@@ -302,7 +305,9 @@ def gpu_arm(args, rank, world, local):
     if not args.headline_only:
         result["extra"] = extras(torch, nq, stream, args, hbm_gbs, bf16_tf, bf16_tf_sus, peak_src)
 
-    if rank == 0 and world == 1:
+    if args.only is not None:
+        pass
+    elif rank == 0 and world == 1:
         result["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     elif rank == 0:
         result["cpu_baseline"] = None
@@ -338,63 +343,84 @@ def extras(torch, nq, stream, args, hbm_gbs, bf16_tf, bf16_tf_sus, peak_src):
     out = {}
     steps = max(5, args.steps // 5)
     warm = max(3, args.warmup)
+    want = None if args.only is None else set(args.only.split(","))
+
+    def on(name):
+        return want is None or name in want
 
     # decode batch 8 of the headline shape
     (_, d_out, d_in, r), = synth.WORKLOADS[HEADLINE]
+    if on("attn7b_b8"):
+        out.update(_extra_b8(torch, nq, stream, steps, warm, hbm_gbs, d_out, d_in, r))
+    for wl in ("mlp7b", "layer70b"):
+        if on(wl):
+            out[wl] = _extra_block(torch, nq, stream, steps, warm, hbm_gbs, wl)
+    if on("prefill"):
+        out["prefill70b_gate"] = _extra_prefill(torch, nq, stream, steps, bf16_tf)
+    if on("pack"):
+        out["pack_70b_gate_U"] = _extra_pack(torch, nq, stream, steps, warm, hbm_gbs)
+    nq.sync_status(stream)
+    return out
+
+
+def _extra_b8(torch, nq, stream, steps, warm, hbm_gbs, d_out, d_in, r):
     lb = decode_bytes(d_out, d_in, r, 8)
     ch = Chain(torch, nq, d_out, d_in, r, 8, n_instances(lb), seed=synth.workload_seed(HEADLINE) + 50)
     g = graph_of(torch, lambda: ch.run(nq, stream), stream)
     ms = timed_replays(torch, g, stream, steps, warm)
     us = ms * 1e3 / (steps * ch.n)
-    out["attn7b_b8"] = {"us_per_layer": round(us, 3), "GB_s": round(lb / us / 1e3, 1),
-                        "frac_hbm": round(lb / us / 1e3 / hbm_gbs, 4)}
     del g, ch
+    return {"attn7b_b8": {"us_per_layer": round(us, 3), "GB_s": round(lb / us / 1e3, 1),
+                          "frac_hbm": round(lb / us / 1e3 / hbm_gbs, 4)}}
 
-    # MLP block (7B) and 70B decoder layer: one block = all its projections (+ SiLU.mul)
-    for wl in ("mlp7b", "layer70b"):
-        shapes = synth.WORKLOADS[wl]
-        block_bytes = sum(decode_bytes(do, di, r, 1) for (_, do, di, r) in shapes)
-        reps = max(2, int(np.ceil(3 * L2_BYTES / block_bytes)))
-        blocks = []
-        for b in range(reps):
-            projs = {}
-            for idx, (name, do, di, rr) in enumerate(shapes):
-                p = synth.make_projection(name, do, di, rr, seed=synth.workload_seed(wl), key=1000 * b + idx)
-                projs[name] = nq.Layer.from_host(p.U, p.V, p.s1, p.s2, rr)
-            blocks.append(projs)
-        need = max(L.workspace_bytes(1) for bl in blocks for L in bl.values())
-        ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
-        dmodel = shapes[0][2]
-        x = torch.zeros((1, dmodel), dtype=torch.bfloat16, device="cuda").normal_()
-        bufs = {name: torch.empty((1, do), dtype=torch.bfloat16, device="cuda") for (name, do, di, rr) in shapes}
-        h = torch.empty((1, blocks[0]["gate"].d_out), dtype=torch.bfloat16, device="cuda")
-        attn_in = torch.zeros((1, shapes[0][1]), dtype=torch.bfloat16, device="cuda").normal_()
 
-        def run_blocks():
-            xx = x
-            for bl in blocks:
-                if "q" in bl:
-                    for name in ("q", "k", "v"):
-                        nq.layer_forward(bl[name], xx, bufs[name], ws=ws, stream=stream)
-                    nq.layer_forward(bl["o"], attn_in, bufs["o"], ws=ws, stream=stream)
-                    xin = bufs["o"]
-                else:
-                    xin = xx
-                nq.layer_forward(bl["gate"], xin, bufs["gate"], ws=ws, stream=stream)
-                nq.layer_forward(bl["up"], xin, bufs["up"], ws=ws, stream=stream)
-                nq.silu_mul(bufs["gate"], bufs["up"], h, stream=stream)
-                nq.layer_forward(bl["down"], h, bufs["down"], ws=ws, stream=stream)
-                xx = bufs["down"]
+def _extra_block(torch, nq, stream, steps, warm, hbm_gbs, wl):
+    """A 7B MLP block or a 70B decoder layer's projections (+ SiLU.mul), decode batch 1."""
+    shapes = synth.WORKLOADS[wl]
+    block_bytes = sum(decode_bytes(do, di, r, 1) for (_, do, di, r) in shapes)
+    reps = max(2, int(np.ceil(3 * L2_BYTES / block_bytes)))
+    blocks = []
+    for b in range(reps):
+        projs = {}
+        for idx, (name, do, di, rr) in enumerate(shapes):
+            p = synth.make_projection(name, do, di, rr, seed=synth.workload_seed(wl), key=1000 * b + idx)
+            projs[name] = nq.Layer.from_host(p.U, p.V, p.s1, p.s2, rr)
+        blocks.append(projs)
+    need = max(L.workspace_bytes(1) for bl in blocks for L in bl.values())
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    dmodel = shapes[0][2]
+    x = torch.zeros((1, dmodel), dtype=torch.bfloat16, device="cuda").normal_()
+    bufs = {name: torch.empty((1, do), dtype=torch.bfloat16, device="cuda") for (name, do, di, rr) in shapes}
+    h = torch.empty((1, blocks[0]["gate"].d_out), dtype=torch.bfloat16, device="cuda")
+    attn_in = torch.zeros((1, shapes[0][1]), dtype=torch.bfloat16, device="cuda").normal_()
 
-        g = graph_of(torch, run_blocks, stream)
-        ms = timed_replays(torch, g, stream, steps, warm)
-        us = ms * 1e3 / (steps * reps)
-        out[wl] = {"us_per_block": round(us, 3), "block_bytes": block_bytes, "GB_s": round(block_bytes / us / 1e3, 1),
-                   "frac_hbm": round(block_bytes / us / 1e3 / hbm_gbs, 4), "blocks_per_step": reps,
-                   "block": "+".join(n for (n, *_r) in shapes) + " + silu_mul"}
-        del g, blocks
+    def run_blocks():
+        xx = x
+        for bl in blocks:
+            if "q" in bl:
+                for name in ("q", "k", "v"):
+                    nq.layer_forward(bl[name], xx, bufs[name], ws=ws, stream=stream)
+                nq.layer_forward(bl["o"], attn_in, bufs["o"], ws=ws, stream=stream)
+                xin = bufs["o"]
+            else:
+                xin = xx
+            nq.layer_forward(bl["gate"], xin, bufs["gate"], ws=ws, stream=stream)
+            nq.layer_forward(bl["up"], xin, bufs["up"], ws=ws, stream=stream)
+            nq.silu_mul(bufs["gate"], bufs["up"], h, stream=stream)
+            nq.layer_forward(bl["down"], h, bufs["down"], ws=ws, stream=stream)
+            xx = bufs["down"]
 
-    # prefill, 70B gate projection
+    g = graph_of(torch, run_blocks, stream)
+    ms = timed_replays(torch, g, stream, steps, warm)
+    us = ms * 1e3 / (steps * reps)
+    del g, blocks
+    return {"us_per_block": round(us, 3), "block_bytes": block_bytes, "GB_s": round(block_bytes / us / 1e3, 1),
+            "frac_hbm": round(block_bytes / us / 1e3 / hbm_gbs, 4), "blocks_per_step": reps,
+            "block": "+".join(n for (n, *_r) in shapes) + " + silu_mul"}
+
+
+def _extra_prefill(torch, nq, stream, steps, bf16_tf):
+    """The 70B gate projection (28672 x 8192, r = 3520) on the tensor-core path."""
     (_, do, di, r), = synth.WORKLOADS["prefill70b"]
     p = synth.make_projection("gate", do, di, r, seed=synth.workload_seed("prefill70b"))
     L = nq.Layer.from_host(p.U, p.V, p.s1, p.s2, r)
@@ -411,9 +437,11 @@ def extras(torch, nq, stream, args, hbm_gbs, bf16_tf, bf16_tf_sus, peak_src):
         pre["M%d" % M] = {"us": round(us, 2), "TFLOP_s": round(flops / us / 1e6, 2),
                           "frac_bf16": round(flops / us / 1e6 / bf16_tf, 4)}
         del g
-    out["prefill70b_gate"] = pre
+    return pre
 
-    # pack: the 70B gate U, 28672 x 3520 fp32 -> packed words
+
+def _extra_pack(torch, nq, stream, steps, warm, hbm_gbs):
+    """Pack of the 70B gate U: 28672 x 3520 fp32 latent -> packed words."""
     rows, rr = 28672, 3520
     lat = torch.randn((rows, rr), dtype=torch.float32, device="cuda")
     pk = torch.empty((rows, rr // 32), dtype=torch.int32, device="cuda")
@@ -421,10 +449,8 @@ def extras(torch, nq, stream, args, hbm_gbs, bf16_tf, bf16_tf_sus, peak_src):
     ms = timed_replays(torch, g, stream, steps, warm)
     us = ms * 1e3 / steps
     pbytes = 4 * rows * rr + rows * rr // 8
-    out["pack_70b_gate_U"] = {"us": round(us, 2), "GB_s": round(pbytes / us / 1e3, 1),
-                              "frac_hbm": round(pbytes / us / 1e3 / hbm_gbs, 4)}
-    nq.sync_status(stream)
-    return out
+    del g
+    return {"us": round(us, 2), "GB_s": round(pbytes / us / 1e3, 1), "frac_hbm": round(pbytes / us / 1e3 / hbm_gbs, 4)}
 
 
 # --------------------------------------------------------------------------- CPU oracle

@@ -16,187 +16,492 @@
 //
 // Stage 2 stages t in shared memory transposed so that lanes reading consecutive words hit
 // consecutive banks; each warp sweeps one row of U with 128-byte coalesced loads.
+#include <cooperative_groups.h>
+
 #include "nq_common.cuh"
 
 namespace nq {
 
-constexpr int kS1Threads = 256;
-constexpr int kS1WordsPerChunk = 8;  // 32-byte row segments: one full DRAM sector per row
-
-template <int MB>
-struct S1Cfg {
-    static constexpr int KB = (MB <= 2) ? 32 : (MB <= 4 ? 16 : 8);  // bits per thread
-    static constexpr int NBG = 32 / KB;                                // bit groups per word
-    static constexpr int JG = kS1Threads / (kS1WordsPerChunk * NBG);   // row subsets per block
-    static constexpr int OUT = kS1WordsPerChunk * 32 * MB;             // outputs per block
-};
-
-__host__ __device__ __forceinline__ constexpr int pad32(int o) { return o + (o >> 5); }
-
-template <int MB>
-__global__ void __launch_bounds__(kS1Threads) decode_stage1_kernel(
-    const uint32_t* __restrict__ V, int64_t ldv, const uint16_t* __restrict__ s2, const uint16_t* __restrict__ x,
-    int M, int64_t d_in, int64_t r, int rows_per_slice, float* __restrict__ part, float* __restrict__ t,
-    unsigned int* __restrict__ tickets) {
-    using C = S1Cfg<MB>;
-    extern __shared__ float smem[];
-    float* z_s = smem;                             // [MB][rows_per_slice]
-    float* red = smem + MB * rows_per_slice;       // [JG][pad32(OUT)]
-    __shared__ unsigned int s_is_last;
-
-    const int tid = threadIdx.x;
-    const int wl = tid % kS1WordsPerChunk;
-    const int bg = (tid / kS1WordsPerChunk) % C::NBG;
-    const int jg = tid / (kS1WordsPerChunk * C::NBG);
-    const int64_t nw = r / 32;
-    const int64_t w = static_cast<int64_t>(blockIdx.x) * kS1WordsPerChunk + wl;
-    const bool wvalid = w < nw;
-    const int S = gridDim.y;
-    const int s = blockIdx.y;
-    const int64_t j0 = static_cast<int64_t>(s) * rows_per_slice;
-    const int64_t j1 = min(d_in, j0 + rows_per_slice);
-    const int rows = static_cast<int>(j1 - j0);
-
-    pdl_wait();  // x (and the workspace) may be written by the previous grid
-
-    // z[m][j] = s2_j * x[m][j] in fp32 (exact: 11 x 8 significant bits)
-    for (int e = tid; e < MB * rows; e += kS1Threads) {
-        const int m = e / rows;
-        const int jj = e - m * rows;
-        float z = 0.0f;
-        if (m < M) z = f16_bits_to_float(s2[j0 + jj]) * bf16_bits_to_float(x[static_cast<int64_t>(m) * d_in + j0 + jj]);
-        z_s[m * rows_per_slice + jj] = z;
-    }
-    __syncthreads();
-
-    float acc[C::KB][MB];
-#pragma unroll
-    for (int c = 0; c < C::KB; ++c)
-#pragma unroll
-        for (int m = 0; m < MB; ++m) acc[c][m] = 0.0f;
-
-    if (wvalid) {
-        const uint32_t* vp = V + w;
-        for (int jj = jg; jj < rows; jj += C::JG) {
-            const uint32_t word = __ldg(vp + (j0 + jj) * ldv) >> (bg * C::KB);
-            float z[MB];
-#pragma unroll
-            for (int m = 0; m < MB; ++m) z[m] = z_s[m * rows_per_slice + jj];
-#pragma unroll
-            for (int c = 0; c < C::KB; ++c) {
-                // bit 1 -> +z, bit 0 -> -z: flip the sign bit of z when the bit is clear
-                const uint32_t flip = ((~word) << (31 - c)) & 0x80000000u;
-#pragma unroll
-                for (int m = 0; m < MB; ++m) acc[c][m] += __uint_as_float(__float_as_uint(z[m]) ^ flip);
-            }
-        }
-    }
-
-    // fold the JG row subsets of this block
-    {
-        float* dst = red + jg * pad32(C::OUT);
-#pragma unroll
-        for (int c = 0; c < C::KB; ++c)
-#pragma unroll
-            for (int m = 0; m < MB; ++m) dst[pad32((wl * 32 + bg * C::KB + c) * MB + m)] = acc[c][m];
-    }
-    __syncthreads();
-
-    const int64_t kbase = static_cast<int64_t>(blockIdx.x) * kS1WordsPerChunk * 32;
-    for (int o = tid; o < C::OUT; o += kS1Threads) {
-        float v = 0.0f;
-        for (int g = 0; g < C::JG; ++g) v += red[g * pad32(C::OUT) + pad32(o)];
-        const int m = o % MB;
-        const int64_t k = kbase + o / MB;
-        if (m < M && k < r) part[(static_cast<int64_t>(s) * M + m) * r + k] = v;
-    }
-
-    // last block of this chunk sums the S partials in slice order
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) {
-        const unsigned int prev = atomicAdd(&tickets[blockIdx.x], 1u);
-        s_is_last = (prev == static_cast<unsigned int>(S - 1)) ? 1u : 0u;
-    }
-    __syncthreads();
-    if (s_is_last) {
-        __threadfence();
-        for (int o = tid; o < C::OUT; o += kS1Threads) {
-            const int m = o % MB;
-            const int64_t k = kbase + o / MB;
-            if (m < M && k < r) {
-                // fixed slice order; the loads of a group of 8 are independent and in flight together
-                const float* pp = part + static_cast<int64_t>(m) * r + k;
-                const int64_t step = static_cast<int64_t>(M) * r;
-                float v = 0.0f;
-                int q = 0;
-                for (; q + 8 <= S; q += 8) {
-                    float a[8];
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) a[u] = __ldcg(pp + (q + u) * step);
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) v += a[u];
-                }
-                for (; q < S; ++q) v += __ldcg(pp + q * step);
-                t[static_cast<int64_t>(m) * r + k] = v;
-            }
-        }
-        if (tid == 0) tickets[blockIdx.x] = 0u;  // restore for the next call
-    }
+// ------------------------------------------------------------------ shared helpers
+__device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-constexpr int kS2Threads = 256;
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-template <int MB>
-__global__ void __launch_bounds__(kS2Threads) decode_stage2_kernel(
-    const uint32_t* __restrict__ U, int64_t ldu, const uint16_t* __restrict__ s1, const float* __restrict__ t,
-    uint16_t* __restrict__ y, int M, int64_t d_out, int64_t r) {
-    extern __shared__ float ts[];  // [MB][32][nw]: ts[(m*32 + c)*nw + w] = t[m][32w + c]
-    const int nw = static_cast<int>(r / 32);
-    const int tid = threadIdx.x;
-    const int lane = tid & 31;
+// Balanced base-256 digit q (0, 1, 2) of a 23-bit signed integer, as an s8 byte.
+__device__ __forceinline__ uint32_t digit_byte(int v, int q) {
+    int d0 = ((v + 128) & 255) - 128;
+    if (q == 0) return static_cast<uint32_t>(d0) & 255u;
+    int v1 = (v - d0) >> 8;
+    int d1 = ((v1 + 128) & 255) - 128;
+    if (q == 1) return static_cast<uint32_t>(d1) & 255u;
+    return static_cast<uint32_t>((v1 - d1) >> 8) & 255u;
+}
 
-    pdl_wait();
 
-    // consecutive threads fill consecutive words w of one (m, c) row: conflict-free stores
-    for (int e = tid; e < MB * static_cast<int>(r); e += kS2Threads) {
-        const int mc = e / nw;  // m * 32 + c
-        const int w = e - mc * nw;
-        const int m = mc >> 5;
-        ts[e] = (m < M) ? t[static_cast<int64_t>(m) * r + 32 * w + (mc & 31)] : 0.0f;
+// Sum of one 64-bit value per thread over the block; every thread gets the total.
+__device__ __forceinline__ long long block_sum_i64(long long v, long long* scratch /* [warps] */) {
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __syncthreads();
+    if (lane == 0) scratch[warp] = v;
+    __syncthreads();
+    long long tot = 0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) tot += scratch[w];
+    return tot;
+}
+
+// ------------------------------------------------------------------ stage 1 (integer MMA)
+//
+// t[m][k] = sum_j (2 v_jk - 1) z[m][j],  z = s2 (.) x,  v in {0, 1} the packed bits of V.
+// V's bits run along k, the reduction runs along j, so four rows j..j+3 of one word column
+// are first byte-transposed (8 PRMTs): word b of the result holds byte b of each of the four
+// words.  For an output k with bit position g = k mod 8 in byte b = (k mod 32) / 8, the
+// register  word_b & (0x01010101 << g)  holds the four bits v_{j..j+3,k} as the values
+// {0, 2^g}: the A operand of mma.sync m16n8k32 (u8) for one row k and four K elements j.  z is
+// quantised per CTA to 23-bit integers (three signed base-256 digits, the s8 B operand), so
+// the products accumulate exactly in int32; each row's 2^g weight is shifted back exactly.
+//
+// Blocks form a thread-block cluster along d_in: block (c, q) owns word chunk c (8 words =
+// 256 outputs k) and row slice q of V.  Each block turns its exact integer partial into an
+// fp64 value with its own scale; after a cluster barrier, block q sums a 1/CS share of the
+// chunk's outputs over the CS blocks' shared memory (distributed shared memory) in rank
+// order and writes t.  No atomics, no global partials: deterministic.
+
+constexpr int kS1Threads = 256;
+constexpr int kS1Words = 8;            // words (of 32 outputs) per cluster chunk
+constexpr int kS1Outs = kS1Words * 32;  // outputs k per chunk
+
+struct S1Params {
+    const uint32_t* V;
+    int64_t ldv;
+    const uint16_t* s2;
+    const uint16_t* x;
+    float* t;
+    int M;
+    int64_t d_in;
+    int r, nw;
+    int rows_per_slice;  // rows of V per block (multiple of 32)
+    int jc_rows;         // rows staged per pass (multiple of 32)
+};
+
+template <int NT>
+struct S1Layout {
+    static constexpr int SWZ = (NT == 1) ? 8 : 24;  // words per quad row of the z table
+};
+
+// 4x4 byte transpose: out[b] = (byte b of w0, byte b of w1, byte b of w2, byte b of w3)
+__device__ __forceinline__ void byte_transpose4(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, uint32_t (&o)[4]) {
+    const uint32_t t0 = __byte_perm(w0, w1, 0x5140);  // w0.b0 w1.b0 w0.b1 w1.b1
+    const uint32_t t1 = __byte_perm(w0, w1, 0x7362);  // w0.b2 w1.b2 w0.b3 w1.b3
+    const uint32_t t2 = __byte_perm(w2, w3, 0x5140);
+    const uint32_t t3 = __byte_perm(w2, w3, 0x7362);
+    o[0] = __byte_perm(t0, t2, 0x5410);
+    o[1] = __byte_perm(t0, t2, 0x7632);
+    o[2] = __byte_perm(t1, t3, 0x5410);
+    o[3] = __byte_perm(t1, t3, 0x7632);
+}
+
+template <int NT>
+__global__ void __launch_bounds__(kS1Threads, 1) decode_stage1_kernel(const S1Params p) {
+    namespace cg = cooperative_groups;
+    constexpr int SWZ = S1Layout<NT>::SWZ;
+    extern __shared__ __align__(16) uint32_t smem1[];
+    const int nq_rows = p.jc_rows / 4;  // quads per pass
+    const int nkb = p.jc_rows / 32;     // K steps per pass
+    uint32_t* aws = smem1;                          // [8 words][nkb][2][4][4]
+    uint32_t* zq = aws + kS1Words * nkb * 32;       // [nq_rows][SWZ]
+    int* red = reinterpret_cast<int*>(zq + nq_rows * SWZ);               // [256][NT*8]
+    double* part = reinterpret_cast<double*>(red + kS1Outs * NT * 8);   // [M][256]
+    __shared__ int s_shift[NQ_MATVEC_MAX_M];
+    __shared__ float s_mul[NQ_MATVEC_MAX_M];
+    __shared__ unsigned long long s_zsum[NQ_MATVEC_MAX_M];
+    __shared__ float s_wmax[kS1Threads / 32][NQ_MATVEC_MAX_M];
+    __shared__ long long s_red64[kS1Threads / 32];
+
+    cg::cluster_group cluster = cg::this_cluster();
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int gid = lane >> 2, tig = lane & 3;
+    const int chunk = blockIdx.x;
+    const int q = blockIdx.y;  // slice index == rank in the cluster
+    const int CS = gridDim.y;
+    const int64_t j0 = static_cast<int64_t>(q) * p.rows_per_slice;
+    const int64_t j1 = min(p.d_in, j0 + p.rows_per_slice);
+    const int wglob0 = chunk * kS1Words;
+
+    // byte-transposed V quads of rows [jb, jb + jc_rows) into aws
+    auto build_aws = [&](int64_t jb) {
+        for (int e = tid; e < kS1Words * nq_rows; e += kS1Threads) {
+            const int w = e % kS1Words, jq = e / kS1Words;
+            const int wg = wglob0 + w;
+            uint32_t v[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int64_t j = jb + 4 * jq + i;
+                v[i] = (wg < p.nw && j < j1) ? __ldg(p.V + j * p.ldv + wg) : 0u;
+            }
+            uint32_t o[4];
+            byte_transpose4(v[0], v[1], v[2], v[3], o);
+            const int kb = jq >> 3, jl = jq & 7, t4 = jl & 3, half = jl >> 2;
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int h = b >> 1, slot = (b & 1) + 2 * half;
+                aws[(((w * nkb + kb) * 2 + h) * 4 + t4) * 4 + slot] = o[b];
+            }
+        }
+    };
+
+    build_aws(j0);  // weights only: may overlap the previous grid
+    pdl_launch_dependents();
+    pdl_wait();     // x may be written by the previous grid
+
+    // ---- slice scale: |z_q| < 2^22, z_q = rint(z * 2^shift)
+    {
+        for (int m = 0; m < p.M; ++m) {
+            const uint16_t* xm = p.x + static_cast<int64_t>(m) * p.d_in;
+            float v = 0.0f;
+#pragma unroll 4
+            for (int64_t j = j0 + tid; j < j1; j += kS1Threads)
+                v = fmaxf(v, fabsf(f16_bits_to_float(p.s2[j]) * bf16_bits_to_float(xm[j])));
+            for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+            if (lane == 0) s_wmax[warp][m] = v;
+        }
+        for (int e = tid; e < kS1Outs * NT * 8; e += kS1Threads) red[e] = 0;
+        __syncthreads();
+        if (tid < p.M) {
+            float v = 0.0f;
+            for (int w = 0; w < kS1Threads / 32; ++w) v = fmaxf(v, s_wmax[w][tid]);
+            int e = 0;
+            frexpf(v, &e);
+            const int sh = (v > 0.0f) ? min(max(22 - e, -126), 126) : 0;
+            s_shift[tid] = sh;
+            s_mul[tid] = ldexpf(1.0f, sh);
+        }
+        __syncthreads();
+    }
+    long long zsum[NQ_MATVEC_MAX_M];
+#pragma unroll
+    for (int m = 0; m < NQ_MATVEC_MAX_M; ++m) zsum[m] = 0;
+
+    // ---- passes over the slice: z table, then MMAs; integer accumulators live in registers
+    int acc[2][NT][4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[h][nt][e] = 0;
+    const bool warp_active = (wglob0 + warp) < p.nw;
+    const uint32_t msk = 0x01010101u << gid;
+
+    for (int64_t jb = j0; jb < j1; jb += p.jc_rows) {
+        if (jb != j0) {
+            __syncthreads();  // previous pass done with aws / zq
+            build_aws(jb);
+        }
+        // z digits: byte i of zq[jq][3m + q] = digit q of z_q(m, row jb + 4jq + i)
+        for (int i = tid; i < nq_rows * SWZ / 4; i += kS1Threads)
+            reinterpret_cast<uint4*>(zq)[i] = make_uint4(0u, 0u, 0u, 0u);
+        __syncthreads();
+        {
+            uint8_t* zb = reinterpret_cast<uint8_t*>(zq);
+            const int64_t jend = min(j1, jb + p.jc_rows);
+            for (int m = 0; m < p.M; ++m) {
+                const uint16_t* xm = p.x + static_cast<int64_t>(m) * p.d_in;
+                const float mul = s_mul[m];
+                long long zs = 0;
+#pragma unroll 4
+                for (int64_t j = jb + tid; j < jend; j += kS1Threads) {
+                    const int v = __float2int_rn(f16_bits_to_float(p.s2[j]) * bf16_bits_to_float(xm[j]) * mul);
+                    zs += v;
+                    const int jl = static_cast<int>(j - jb);
+                    const int base = ((jl >> 2) * SWZ + 3 * m) * 4 + (jl & 3);
+                    zb[base] = static_cast<uint8_t>(digit_byte(v, 0));
+                    zb[base + 4] = static_cast<uint8_t>(digit_byte(v, 1));
+                    zb[base + 8] = static_cast<uint8_t>(digit_byte(v, 2));
+                }
+                zsum[m] += zs;
+            }
+        }
+        __syncthreads();
+
+        if (warp_active) {
+            const int w = warp;
+            for (int kb = 0; kb < nkb; ++kb) {
+                uint32_t bf[NT][2];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    bf[nt][0] = zq[(8 * kb + tig) * SWZ + nt * 8 + gid];
+                    bf[nt][1] = zq[(8 * kb + 4 + tig) * SWZ + nt * 8 + gid];
+                }
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const uint4 a = *reinterpret_cast<const uint4*>(aws + (((w * nkb + kb) * 2 + h) * 4 + tig) * 4);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+                        mma_u8s8(acc[h][nt], a.x & msk, a.y & msk, a.z & msk, a.w & msk, bf[nt][0], bf[nt][1]);
+                }
+            }
+        }
+    }
+
+    for (int m = 0; m < p.M; ++m) {
+        const long long tot = block_sum_i64(zsum[m], s_red64);
+        if (tid == 0) s_zsum[m] = static_cast<unsigned long long>(tot);
     }
     __syncthreads();
 
-    const int64_t warp = static_cast<int64_t>(blockIdx.x) * (kS2Threads / 32) + (tid >> 5);
-    const int64_t n_warps = static_cast<int64_t>(gridDim.x) * (kS2Threads / 32);
-    for (int64_t i = warp; i < d_out; i += n_warps) {
-        float acc[MB];
+    // ---- exact per-output integers: row gid of M-tile (w, h) is k = 32w + 8(2h) + gid,
+    // row gid+8 is k = 32w + 8(2h+1) + gid; both carry the weight 2^gid
+    if (warp_active) {
 #pragma unroll
-        for (int m = 0; m < MB; ++m) acc[m] = 0.0f;
-        const uint32_t* urow = U + i * ldu;
-        for (int w = lane; w < nw; w += 32) {
-            const uint32_t nword = ~__ldg(urow + w);
+        for (int h = 0; h < 2; ++h)
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                const uint32_t flip = (nword << (31 - c)) & 0x80000000u;
+            for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                for (int m = 0; m < MB; ++m)
-                    acc[m] += __uint_as_float(__float_as_uint(ts[(m * 32 + c) * nw + w]) ^ flip);
+                for (int e = 0; e < 4; ++e) {
+                    const int kl = 32 * warp + 8 * (2 * h + (e >> 1)) + gid;
+                    const int col = nt * 8 + 2 * tig + (e & 1);
+                    red[kl * (NT * 8) + col] = acc[h][nt][e] >> gid;
+                }
+    }
+    __syncthreads();
+    for (int e = tid; e < p.M * kS1Outs; e += kS1Threads) {
+        const int m = e / kS1Outs, kl = e - m * kS1Outs;
+        const int* rr = red + kl * (NT * 8) + 3 * m;
+        const long long P = static_cast<long long>(rr[0]) + (static_cast<long long>(rr[1]) << 8) +
+                            (static_cast<long long>(rr[2]) << 16);
+        const long long val = 2 * P - static_cast<long long>(s_zsum[m]);
+        part[m * kS1Outs + kl] = ldexp(static_cast<double>(val), -s_shift[m]);
+    }
+
+    // ---- cluster reduction over the CS row slices, rank order
+    cluster.sync();
+    {
+        const int per = (kS1Outs + CS - 1) / CS;
+        const int k_lo = q * per, k_hi = min(kS1Outs, k_lo + per);
+        for (int e = tid; e < p.M * (k_hi - k_lo); e += kS1Threads) {
+            const int m = e / (k_hi - k_lo), kl = k_lo + (e - m * (k_hi - k_lo));
+            const int64_t k = static_cast<int64_t>(wglob0) * 32 + kl;
+            if (k < p.r) {
+                double sum = 0.0;
+                for (int rank = 0; rank < CS; ++rank) {
+                    const double* rp = cluster.map_shared_rank(part, rank);
+                    sum += rp[m * kS1Outs + kl];
+                }
+                p.t[static_cast<int64_t>(m) * p.r + k] = static_cast<float>(sum);
             }
         }
-#pragma unroll
-        for (int m = 0; m < MB; ++m) {
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], off);
-        }
-        if (lane < M) {
-            float v = acc[0];
-#pragma unroll
-            for (int m = 1; m < MB; ++m)
-                if (lane == m) v = acc[m];
-            y[static_cast<int64_t>(lane) * d_out + i] = float_to_bf16_bits(f16_bits_to_float(s1[i]) * v);
-        }
     }
+    cluster.sync();  // keep this block's shared memory alive until every peer has read it
+}
+
+// ------------------------------------------------------------------ stage 2 (integer MMA)
+//
+// y[m][i] = s1_i * sum_k (2 u_ik - 1) t[m][k] with u in {0, 1} the packed bits of U.
+// t is quantised per batch row to a 23-bit fixed-point integer t_q = rint(t * 2^sh) (|t_q| <
+// 2^22) and split into three signed base-256 digits (planes) t_q = d0 + 2^8 d1 + 2^16 d2.
+// The packed words feed mma.sync m16n8k32 (A u8, B s8, D s32) directly: for a bit offset
+// s in 0..7 the register  word & (0x01010101 << s)  holds, in its four bytes, the bits
+// s, s+8, s+16, s+24 of the word as the values {0, 2^s} -- four K elements for one AND.
+// The B operand supplies the t digits for those same four k, so the MMA for offset s
+// accumulates 2^s * sum u_ik d_q(k) over k = s (mod 8); separate accumulators per s are
+// shifted back (exactly: each is a multiple of 2^s) and summed.  Everything up to the final
+// scale is integer arithmetic, so the result is exact for the quantised t and independent of
+// summation order.
+constexpr int kS2Threads = 256;
+constexpr int kS2Warps = kS2Threads / 32;
+
+struct S2Params {
+    const uint32_t* U;
+    int64_t ldu;
+    const uint16_t* s1;
+    const float* t;
+    uint16_t* y;
+    int M;
+    int64_t d_out;
+    int r, nw, nwp;      // rank, words per row, words padded to a multiple of 8
+    int su;              // shared-memory row stride of U (words), = 4 (mod 32)
+    int mt_total;        // 16-row M-tiles of U
+    int chunk_mt;        // M-tiles staged in shared memory at a time
+};
+
+template <int NT>
+struct S2Layout {
+    static constexpr int SW = (NT == 1) ? 8 : 24;  // words per (s, w) entry row of the B table
+};
+
+template <int NT>
+__global__ void __launch_bounds__(kS2Threads, 1) decode_stage2_kernel(const S2Params p) {
+    extern __shared__ __align__(16) uint32_t smem2[];
+    constexpr int SW = S2Layout<NT>::SW;
+    uint32_t* bt = smem2;                                  // [8][nwp][SW]
+    uint32_t* ublk = bt + 8 * p.nwp * SW;                  // [chunk_mt*16][su]
+    int* red = reinterpret_cast<int*>(ublk + p.chunk_mt * 16 * p.su);  // [chunk_mt*16][NT*8]
+    __shared__ int s_shift[NQ_MATVEC_MAX_M];
+    __shared__ float s_mul[NQ_MATVEC_MAX_M];
+    __shared__ unsigned long long s_tsum[NQ_MATVEC_MAX_M];
+    __shared__ float s_wmax[kS2Warps][NQ_MATVEC_MAX_M];
+    __shared__ long long s_red64[kS2Warps];
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int G = gridDim.x;
+    const int mt0 = static_cast<int>((static_cast<int64_t>(blockIdx.x) * p.mt_total) / G);
+    const int mt1 = static_cast<int>((static_cast<int64_t>(blockIdx.x + 1) * p.mt_total) / G);
+
+    // stage the rows of U of M-tiles [a, b) into ublk (row stride su); weights only, so this
+    // may run before the previous grid has finished
+    auto load_u = [&](int a, int b) {
+        const int64_t row0 = static_cast<int64_t>(a) * 16;
+        const int64_t row1 = min(static_cast<int64_t>(b) * 16, p.d_out);
+        const int rows = static_cast<int>(row1 - row0);
+        const bool even = ((p.ldu & 1) == 0) && ((p.nw & 1) == 0);
+        if (even) {
+            const int per_row = p.nw / 2;
+            for (int e = tid; e < rows * per_row; e += kS2Threads) {
+                const int rr = e / per_row, c = e - rr * per_row;
+                cp_async8(static_cast<uint32_t>(__cvta_generic_to_shared(ublk + rr * p.su + 2 * c)),
+                          p.U + (row0 + rr) * p.ldu + 2 * c);
+            }
+        } else {
+            for (int e = tid; e < rows * p.nw; e += kS2Threads) {
+                const int rr = e / p.nw, c = e - rr * p.nw;
+                cp_async4(static_cast<uint32_t>(__cvta_generic_to_shared(ublk + rr * p.su + c)),
+                          p.U + (row0 + rr) * p.ldu + c);
+            }
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+
+    if (mt0 < mt1) load_u(mt0, min(mt1, mt0 + p.chunk_mt));
+    pdl_launch_dependents();
+    pdl_wait();  // t comes from stage 1 of this call
+
+    // ---- per-batch-row scale: |t_q| < 2^22 with t_q = rint(t * 2^shift)
+    {
+        for (int i = tid; i < 2 * p.nwp * SW; i += kS2Threads)  // 8 * nwp * SW words, 16 B at a time
+            reinterpret_cast<uint4*>(bt)[i] = make_uint4(0u, 0u, 0u, 0u);
+        for (int m = 0; m < p.M; ++m) {
+            const float* tm = p.t + static_cast<int64_t>(m) * p.r;
+            float v = 0.0f;
+#pragma unroll 8
+            for (int k = tid; k < p.r; k += kS2Threads) v = fmaxf(v, fabsf(tm[k]));
+            for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+            if (lane == 0) s_wmax[warp][m] = v;
+        }
+        __syncthreads();
+        if (tid < p.M) {
+            float v = 0.0f;
+            for (int w = 0; w < kS2Warps; ++w) v = fmaxf(v, s_wmax[w][tid]);
+            int e = 0;
+            frexpf(v, &e);  // v < 2^e
+            const int sh = (v > 0.0f) ? min(max(22 - e, -126), 126) : 0;
+            s_shift[tid] = sh;
+            s_mul[tid] = ldexpf(1.0f, sh);
+        }
+        __syncthreads();
+        // quantise, scatter the three digits of t_q(m, k) into the B table, sum t_q:
+        // digit q of t_q(m, k) is byte (k mod 32) / 8 of word bt[((k mod 8) * nwp + k / 32) * SW + 3m + q]
+        uint8_t* btb = reinterpret_cast<uint8_t*>(bt);
+        for (int m = 0; m < p.M; ++m) {
+            const float* tm = p.t + static_cast<int64_t>(m) * p.r;
+            const float mul = s_mul[m];
+            long long ts = 0;
+#pragma unroll 4
+            for (int k = tid; k < p.r; k += kS2Threads) {
+                const int v = __float2int_rn(tm[k] * mul);
+                ts += v;
+                const int base = (((k & 7) * p.nwp + (k >> 5)) * SW + 3 * m) * 4 + ((k >> 3) & 3);
+                btb[base] = static_cast<uint8_t>(digit_byte(v, 0));
+                btb[base + 4] = static_cast<uint8_t>(digit_byte(v, 1));
+                btb[base + 8] = static_cast<uint8_t>(digit_byte(v, 2));
+            }
+            ts = block_sum_i64(ts, s_red64);
+            if (tid == 0) s_tsum[m] = static_cast<unsigned long long>(ts);
+        }
+        __syncthreads();
+    }
+
+    const int gid = lane >> 2, tig = lane & 3;
+    const int ng = p.nwp / 8;
+    for (int c0 = mt0; c0 < mt1; c0 += p.chunk_mt) {
+        const int c1 = min(mt1, c0 + p.chunk_mt);
+        const int nmt = c1 - c0;
+        for (int e = tid; e < nmt * 16 * NT * 8; e += kS2Threads) red[e] = 0;
+        cp_async_wait_all();
+        __syncthreads();
+
+        const int kp_count = max(1, min(ng, kS2Warps / nmt));
+        const int jobs = nmt * kp_count;
+        for (int job = warp; job < jobs; job += kS2Warps) {
+            const int mtl = job / kp_count, kp = job - mtl * kp_count;
+            const int g_lo = (kp * ng) / kp_count, g_hi = ((kp + 1) * ng) / kp_count;
+            int acc[8][NT][4];
+#pragma unroll
+            for (int s = 0; s < 8; ++s)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) acc[s][nt][e] = 0;
+            const uint32_t* u0 = ublk + (mtl * 16 + gid) * p.su;
+            const uint32_t* u1 = u0 + 8 * p.su;
+            for (int g = g_lo; g < g_hi; ++g) {
+                const int wb = 8 * g;
+                const uint32_t w00 = u0[wb + tig], w01 = u0[wb + 4 + tig];
+                const uint32_t w10 = u1[wb + tig], w11 = u1[wb + 4 + tig];
+#pragma unroll
+                for (int s = 0; s < 8; ++s) {
+                    const uint32_t msk = 0x01010101u << s;
+                    const uint32_t a0 = w00 & msk, a1 = w10 & msk, a2 = w01 & msk, a3 = w11 & msk;
+                    const uint32_t* b = bt + (s * p.nwp + wb) * SW;
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+                        mma_u8s8(acc[s][nt], a0, a1, a2, a3, b[tig * SW + nt * 8 + gid], b[(4 + tig) * SW + nt * 8 + gid]);
+                }
+            }
+            // D[row][col]: e = 0,1 -> row gid, cols 2tig, 2tig+1; e = 2,3 -> row gid+8
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    int v = 0;
+#pragma unroll
+                    for (int s = 0; s < 8; ++s) v += acc[s][nt][e] >> s;
+                    const int row = mtl * 16 + gid + ((e >> 1) << 3);
+                    const int col = nt * 8 + 2 * tig + (e & 1);
+                    atomicAdd(&red[row * (NT * 8) + col], v);
+                }
+        }
+        __syncthreads();
+
+        // epilogue: y = s1 * 2^-shift * (2 P - Tsum), P = d0 + 2^8 d1 + 2^16 d2
+        for (int e = tid; e < nmt * 16 * p.M; e += kS2Threads) {
+            const int row = e / p.M, m = e - row * p.M;
+            const int64_t i = static_cast<int64_t>(c0) * 16 + row;
+            if (i < p.d_out) {
+                const int* rr = red + row * (NT * 8) + 3 * m;
+                const long long P = static_cast<long long>(rr[0]) + (static_cast<long long>(rr[1]) << 8) +
+                                    (static_cast<long long>(rr[2]) << 16);
+                const long long val = 2 * P - static_cast<long long>(s_tsum[m]);
+                const double yv = static_cast<double>(f16_bits_to_float(p.s1[i])) * ldexp(static_cast<double>(val), -s_shift[m]);
+                p.y[static_cast<int64_t>(m) * p.d_out + i] = __bfloat16_as_ushort(__double2bfloat16(yv));
+            }
+        }
+        __syncthreads();
+        if (c1 < mt1) load_u(c1, min(mt1, c1 + p.chunk_mt));
+    }
+    cp_async_wait_all();
 }
 
 }  // namespace nq
@@ -204,81 +509,105 @@ __global__ void __launch_bounds__(kS2Threads) decode_stage2_kernel(
 // ------------------------------------------------------------------------------ host side
 namespace {
 
-struct DecodePlan {
-    int64_t n_chunks;
-    int S;
-    int rows_per_slice;
-    size_t off_t, off_part, off_tickets, total;
-};
-
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 constexpr size_t kWsHeader = NQ_WS_HEADER_BYTES;
+constexpr size_t kStage1SmemBudget = 200 * 1024;
+constexpr size_t kStage2SmemBudget = 200 * 1024;
 
-DecodePlan plan_decode(int64_t d_in, int64_t r, int64_t M) {
-    DecodePlan p{};
+int ntiles_for(int64_t M) { return static_cast<int>((3 * M + 7) / 8); }
+
+struct S1Plan {
+    int n_chunks, CS, rows_per_slice, jc_rows;
+    size_t smem;
+};
+
+S1Plan plan_stage1(int64_t d_in, int64_t r, int64_t M) {
+    S1Plan p{};
     const int64_t nw = r / 32;
-    p.n_chunks = (nw + nq::kS1WordsPerChunk - 1) / nq::kS1WordsPerChunk;
-    const int64_t target = nq_host::sm_count();
-    int64_t S = (target + p.n_chunks - 1) / p.n_chunks;
-    if (S > 16) S = 16;                          // few partials: the last block sums them
-    const int64_t min_s = (d_in + 2047) / 2048;  // at most 2048 rows per slice (z staging)
-    if (S < min_s) S = min_s;
-    if (S > d_in) S = d_in;
-    if (S < 1) S = 1;
-    p.rows_per_slice = static_cast<int>((d_in + S - 1) / S);
-    p.S = static_cast<int>((d_in + p.rows_per_slice - 1) / p.rows_per_slice);
-    // The tickets live at a fixed place, the first kWsHeader bytes of every workspace, so that
-    // calls with different shapes (and the prefill path, which starts after the header too)
-    // can share one workspace without landing data on a counter that must read zero.
-    p.off_tickets = 0;
-    p.off_t = kWsHeader;
-    p.off_part = p.off_t + align256(static_cast<size_t>(M * r) * sizeof(float));
-    p.total = p.off_part + align256(static_cast<size_t>(p.S) * M * r * sizeof(float));
+    p.n_chunks = static_cast<int>((nw + nq::kS1Words - 1) / nq::kS1Words);
+    int cs = p.n_chunks <= 8 ? 16 : (p.n_chunks <= 18 ? 8 : (p.n_chunks <= 37 ? 4 : 2));
+    while (cs > 1 && static_cast<int64_t>(cs) * 32 > d_in) cs >>= 1;
+    p.CS = cs;
+    p.rows_per_slice = static_cast<int>(((d_in + cs - 1) / cs + 31) / 32 * 32);
+    const int nt = ntiles_for(M);
+    const int swz = nt == 1 ? 8 : 24;
+    const size_t fixed = static_cast<size_t>(nq::kS1Outs) * nt * 8 * 4 + static_cast<size_t>(M) * nq::kS1Outs * 8;
+    int64_t jc = static_cast<int64_t>((kStage1SmemBudget - fixed) / (32 + swz)) / 32 * 32;
+    if (jc > p.rows_per_slice) jc = p.rows_per_slice;
+    if (jc < 32) jc = 32;
+    p.jc_rows = static_cast<int>(jc);
+    p.smem = static_cast<size_t>(jc) * (32 + swz) + fixed;
     return p;
 }
 
-template <int MB>
-nq_status launch_decode_mb(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y, int M, void* ws,
-                           cudaStream_t stream, bool pdl) {
-    const DecodePlan p = plan_decode(L->d_in, L->r, M);
-    char* base = static_cast<char*>(ws);
-    float* t = reinterpret_cast<float*>(base + p.off_t);
-    float* part = reinterpret_cast<float*>(base + p.off_part);
-    unsigned int* tickets = reinterpret_cast<unsigned int*>(base + p.off_tickets);
+size_t decode_ws_bytes(int64_t r, int64_t M) { return kWsHeader + align256(static_cast<size_t>(M * r) * sizeof(float)); }
 
-    using C = nq::S1Cfg<MB>;
-    const size_t smem1 = (static_cast<size_t>(MB) * p.rows_per_slice + static_cast<size_t>(C::JG) * nq::pad32(C::OUT)) *
-                         sizeof(float);
-    static bool attr1 = false;
-    if (!attr1) {
-        cudaFuncSetAttribute(nq::decode_stage1_kernel<MB>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-        cudaFuncSetAttribute(nq::decode_stage2_kernel<MB>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-        attr1 = true;
-    }
+template <int NT>
+void set_attrs_once() {
+    static bool done[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || done[dev]) return;
+    cudaFuncSetAttribute(nq::decode_stage1_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(kStage1SmemBudget));
+    cudaFuncSetAttribute(nq::decode_stage1_kernel<NT>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    cudaFuncSetAttribute(nq::decode_stage2_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(kStage2SmemBudget));
+    done[dev] = true;
+}
+
+template <int NT>
+nq_status launch_decode_nt(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y, int M, void* ws,
+                           cudaStream_t stream, bool pdl) {
+    set_attrs_once<NT>();
+    float* t = reinterpret_cast<float*>(static_cast<char*>(ws) + kWsHeader);
     {
-        const uint32_t* V = L->V;
-        int64_t ldv = L->ldv, d_in = L->d_in, r = L->r;
-        const uint16_t* s2 = L->s2;
-        int rps = p.rows_per_slice;
-        void* args[] = {&V, &ldv, &s2, &x, &M, &d_in, &r, &rps, &part, &t, &tickets};
-        dim3 grid(static_cast<unsigned>(p.n_chunks), static_cast<unsigned>(p.S));
-        if (nq_host::launch_pdl(reinterpret_cast<const void*>(nq::decode_stage1_kernel<MB>), grid,
-                                dim3(nq::kS1Threads), smem1, stream, args, pdl) != cudaSuccess)
+        const S1Plan sp = plan_stage1(L->d_in, L->r, M);
+        nq::S1Params q{};
+        q.V = L->V;
+        q.ldv = L->ldv;
+        q.s2 = L->s2;
+        q.x = x;
+        q.t = t;
+        q.M = M;
+        q.d_in = L->d_in;
+        q.r = static_cast<int>(L->r);
+        q.nw = static_cast<int>(L->r / 32);
+        q.rows_per_slice = sp.rows_per_slice;
+        q.jc_rows = sp.jc_rows;
+        void* args[] = {&q};
+        if (nq_host::launch_ex(reinterpret_cast<const void*>(nq::decode_stage1_kernel<NT>),
+                               dim3(sp.n_chunks, sp.CS), dim3(nq::kS1Threads), sp.smem, stream, args, pdl,
+                               sp.CS) != cudaSuccess)
             return NQ_ERR_LAUNCH;
     }
     {
-        const uint32_t* U = L->U;
-        int64_t ldu = L->ldu, d_out = L->d_out, r = L->r;
-        const uint16_t* s1 = L->s1;
-        const float* tc = t;
-        void* args[] = {&U, &ldu, &s1, &tc, &y, &M, &d_out, &r};
-        const size_t smem2 = static_cast<size_t>(MB) * L->r * sizeof(float);
-        int64_t blocks = (L->d_out + 7) / 8;
-        const int64_t cap = 2LL * nq_host::sm_count();
-        if (blocks > cap) blocks = cap;
-        if (nq_host::launch_pdl(reinterpret_cast<const void*>(nq::decode_stage2_kernel<MB>),
-                                dim3(static_cast<unsigned>(blocks)), dim3(nq::kS2Threads), smem2, stream, args,
-                                pdl) != cudaSuccess)
+        nq::S2Params q{};
+        q.U = L->U;
+        q.ldu = L->ldu;
+        q.s1 = L->s1;
+        q.t = t;
+        q.y = y;
+        q.M = M;
+        q.d_out = L->d_out;
+        q.r = static_cast<int>(L->r);
+        q.nw = static_cast<int>(L->r / 32);
+        q.nwp = (q.nw + 7) / 8 * 8;
+        q.su = q.nwp + ((4 - q.nwp % 32) + 32) % 32;
+        q.mt_total = static_cast<int>((L->d_out + 15) / 16);
+        int grid = nq_host::sm_count();
+        if (grid > q.mt_total) grid = q.mt_total;
+        const int per_cta = (q.mt_total + grid - 1) / grid;
+        const size_t bt_bytes = static_cast<size_t>(8) * q.nwp * nq::S2Layout<NT>::SW * 4;
+        const size_t per_mt = static_cast<size_t>(16) * q.su * 4 + static_cast<size_t>(16) * NT * 8 * 4;
+        int chunk = per_cta;
+        if (bt_bytes + chunk * per_mt > kStage2SmemBudget) chunk = static_cast<int>((kStage2SmemBudget - bt_bytes) / per_mt);
+        if (chunk < 1) return NQ_ERR_SHAPE;
+        q.chunk_mt = chunk;
+        const size_t smem2 = bt_bytes + chunk * per_mt;
+        void* args[] = {&q};
+        if (nq_host::launch_ex(reinterpret_cast<const void*>(nq::decode_stage2_kernel<NT>), dim3(grid),
+                               dim3(nq::kS2Threads), smem2, stream, args, pdl, 1) != cudaSuccess)
             return NQ_ERR_LAUNCH;
     }
     return NQ_OK;
@@ -286,20 +615,28 @@ nq_status launch_decode_mb(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y
 
 }  // namespace
 
-size_t nq_decode_workspace_bytes(int64_t d_in, int64_t r, int64_t M) { return plan_decode(d_in, r, M).total; }
+size_t nq_decode_workspace_bytes(int64_t d_in, int64_t r, int64_t M) {
+    (void)d_in;
+    return decode_ws_bytes(r, M);
+}
 
-// Shared-memory need of stage 2 (t staged per batch row): the caller rejects layers whose
-// rank does not fit.
+// Shared memory stage 2 needs at the least (its B table plus one staged M-tile of U); the
+// caller rejects layers for which this exceeds the budget.
 size_t nq_decode_stage2_smem(int64_t r, int64_t M) {
-    const int64_t mb = M <= 1 ? 1 : (M <= 2 ? 2 : (M <= 4 ? 4 : 8));
-    return static_cast<size_t>(mb * r) * sizeof(float);
+    const int64_t nt = ntiles_for(M);
+    const int64_t nwp = (r / 32 + 7) / 8 * 8;
+    const int64_t sw = nt == 1 ? 8 : 24;
+    const int64_t su = nwp + ((4 - nwp % 32) + 32) % 32;
+    const size_t need = static_cast<size_t>(8 * nwp * sw * 4 + 16 * su * 4 + 16 * nt * 8 * 4);
+    return need <= kStage2SmemBudget ? need : kStage2SmemBudget + 1;
 }
 
 nq_status nq_launch_decode(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y, int64_t M, void* ws,
                            cudaStream_t stream, bool pdl) {
     const int m = static_cast<int>(M);
-    if (M <= 1) return launch_decode_mb<1>(L, x, y, m, ws, stream, pdl);
-    if (M <= 2) return launch_decode_mb<2>(L, x, y, m, ws, stream, pdl);
-    if (M <= 4) return launch_decode_mb<4>(L, x, y, m, ws, stream, pdl);
-    return launch_decode_mb<8>(L, x, y, m, ws, stream, pdl);
+    switch (ntiles_for(M)) {
+        case 1: return launch_decode_nt<1>(L, x, y, m, ws, stream, pdl);
+        case 2: return launch_decode_nt<2>(L, x, y, m, ws, stream, pdl);
+        default: return launch_decode_nt<3>(L, x, y, m, ws, stream, pdl);
+    }
 }

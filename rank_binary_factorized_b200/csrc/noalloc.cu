@@ -52,11 +52,11 @@ extern "C" NQ_API nq_status nq_lrb_matvec_noalloc(const nq_lrb_layer* L, const u
     if (L->d_out <= 0 || L->d_in <= 0 || L->r <= 0 || (L->r % 32) != 0 || L->r > NQ_MAX_RANK_LIMIT) return NQ_ERR_SHAPE;
     if (L->ldu < L->r / 32 || L->ldv < L->r / 32) return NQ_ERR_SHAPE;
     if (M < 1 || M > NQ_MATVEC_MAX_M) return NQ_ERR_SHAPE;
-    if (nq_decode_stage2_smem(L->r, M) > 200 * 1024) return NQ_ERR_SHAPE;
     if (!aligned16(L->U) || !aligned16(L->V) || !aligned16(L->s1) || !aligned16(L->s2) || !aligned16(x) ||
         !aligned16(y))
         return NQ_ERR_ALIGN;
     if (nq_decode_workspace_bytes(L->d_in, L->r, M) > NQ_NOALLOC_SCRATCH_BYTES) return NQ_ERR_SCRATCH_LIMIT;
+    if (nq_decode_stage2_smem(L->r, M) > 200 * 1024) return NQ_ERR_SHAPE;
     int dev = -1, major = 0, minor = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return NQ_ERR_DEVICE;
     cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);

@@ -60,4 +60,7 @@ int sm_count();                                   // multiprocessors of the curr
 unsigned int* error_word();                       // device address of the error word
 cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem, cudaStream_t s, void** args,
                        bool pdl);
+// as launch_pdl, with thread-block clusters of (1, cluster_y, 1) when cluster_y > 1
+cudaError_t launch_ex(const void* fn, dim3 grid, dim3 block, size_t smem, cudaStream_t s, void** args, bool pdl,
+                      int cluster_y);
 }  // namespace nq_host
