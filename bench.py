@@ -302,7 +302,7 @@ def gpu_arm(args, rank, world, local):
     # the chain of layer_forward calls (captured once as a graph), D2H of the result
     result["e2e"] = e2e_measure(torch, nq, chain, stream, args, dist, world)
 
-    if not args.headline_only:
+    if not args.headline_only or args.only is not None:
         result["extra"] = extras(torch, nq, stream, args, hbm_gbs, bf16_tf, bf16_tf_sus, peak_src)
 
     if args.only is not None:

@@ -39,6 +39,18 @@ __device__ __forceinline__ void cp_async8(uint32_t dst, const void* src) {
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
+// The three balanced base-256 digits of a 23-bit signed integer v = a0 + 2^8 a1 + 2^16 a2,
+// each in [-128, 127], returned as s8 bytes.
+__device__ __forceinline__ void digits3(int v, uint32_t& d0, uint32_t& d1, uint32_t& d2) {
+    const int a0 = (v << 24) >> 24;  // the low byte, sign-extended
+    const int v1 = (v - a0) >> 8;    // exact: v - a0 is a multiple of 256
+    const int a1 = (v1 << 24) >> 24;
+    const int a2 = (v1 - a1) >> 8;
+    d0 = static_cast<uint32_t>(a0) & 255u;
+    d1 = static_cast<uint32_t>(a1) & 255u;
+    d2 = static_cast<uint32_t>(a2) & 255u;
+}
+
 // Balanced base-256 digit q (0, 1, 2) of a 23-bit signed integer, as an s8 byte.
 __device__ __forceinline__ uint32_t digit_byte(int v, int q) {
     int d0 = ((v + 128) & 255) - 128;
@@ -94,6 +106,7 @@ struct S1Params {
     int r, nw;
     int rows_per_slice;  // rows of V per block (multiple of 32)
     int jc_rows;         // rows staged per pass (multiple of 32)
+    int zstage;          // z of the slice (M x rows_per_slice fp32) is kept in shared memory
 };
 
 template <int NT>
@@ -121,9 +134,11 @@ __global__ void __launch_bounds__(kS1Threads, 1) decode_stage1_kernel(const S1Pa
     const int nq_rows = p.jc_rows / 4;  // quads per pass
     const int nkb = p.jc_rows / 32;     // K steps per pass
     uint32_t* aws = smem1;                          // [8 words][nkb][2][4][4]
-    uint32_t* zq = aws + kS1Words * nkb * 32;       // [nq_rows][SWZ]
+    uint32_t* zq = aws + kS1Words * (nkb * 32 + 4);  // [nq_rows][SWZ]
     int* red = reinterpret_cast<int*>(zq + nq_rows * SWZ);               // [256][NT*8]
     double* part = reinterpret_cast<double*>(red + kS1Outs * NT * 8);   // [M][256]
+    float* zs_s = reinterpret_cast<float*>(part + p.M * kS1Outs);         // [M][zld] when p.zstage
+    const int zld = p.rows_per_slice + p.rows_per_slice / 32;             // one pad word per 32
     __shared__ int s_shift[NQ_MATVEC_MAX_M];
     __shared__ float s_mul[NQ_MATVEC_MAX_M];
     __shared__ unsigned long long s_zsum[NQ_MATVEC_MAX_M];
@@ -142,22 +157,34 @@ __global__ void __launch_bounds__(kS1Threads, 1) decode_stage1_kernel(const S1Pa
 
     // byte-transposed V quads of rows [jb, jb + jc_rows) into aws
     auto build_aws = [&](int64_t jb) {
-        for (int e = tid; e < kS1Words * nq_rows; e += kS1Threads) {
-            const int w = e % kS1Words, jq = e / kS1Words;
-            const int wg = wglob0 + w;
-            uint32_t v[4];
+        constexpr int U = 4;  // quads per thread in flight at once
+        const int tasks = kS1Words * nq_rows;
+        for (int e0 = tid; e0 < tasks; e0 += U * kS1Threads) {
+            uint32_t v[U][4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int64_t j = jb + 4 * jq + i;
-                v[i] = (wg < p.nw && j < j1) ? __ldg(p.V + j * p.ldv + wg) : 0u;
+            for (int u = 0; u < U; ++u) {
+                const int e = e0 + u * kS1Threads;
+                const int w = e % kS1Words, jq = e / kS1Words;
+                const int wg = wglob0 + w;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int64_t j = jb + 4 * jq + i;
+                    v[u][i] = (e < tasks && wg < p.nw && j < j1) ? __ldg(p.V + j * p.ldv + wg) : 0u;
+                }
             }
-            uint32_t o[4];
-            byte_transpose4(v[0], v[1], v[2], v[3], o);
-            const int kb = jq >> 3, jl = jq & 7, t4 = jl & 3, half = jl >> 2;
 #pragma unroll
-            for (int b = 0; b < 4; ++b) {
-                const int h = b >> 1, slot = (b & 1) + 2 * half;
-                aws[(((w * nkb + kb) * 2 + h) * 4 + t4) * 4 + slot] = o[b];
+            for (int u = 0; u < U; ++u) {
+                const int e = e0 + u * kS1Threads;
+                if (e >= tasks) break;
+                const int w = e % kS1Words, jq = e / kS1Words;
+                uint32_t o[4];
+                byte_transpose4(v[u][0], v[u][1], v[u][2], v[u][3], o);
+                const int kb = jq >> 3, jl = jq & 7, t4 = jl & 3, half = jl >> 2;
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    const int h = b >> 1, slot = (b & 1) + 2 * half;
+                    aws[w * (nkb * 32 + 4) + ((kb * 2 + h) * 4 + t4) * 4 + slot] = o[b];
+                }
             }
         }
     };
@@ -172,8 +199,14 @@ __global__ void __launch_bounds__(kS1Threads, 1) decode_stage1_kernel(const S1Pa
             const uint16_t* xm = p.x + static_cast<int64_t>(m) * p.d_in;
             float v = 0.0f;
 #pragma unroll 4
-            for (int64_t j = j0 + tid; j < j1; j += kS1Threads)
-                v = fmaxf(v, fabsf(f16_bits_to_float(p.s2[j]) * bf16_bits_to_float(xm[j])));
+            for (int64_t j = j0 + tid; j < j1; j += kS1Threads) {
+                const float z = f16_bits_to_float(p.s2[j]) * bf16_bits_to_float(xm[j]);
+                if (p.zstage) {
+                    const int jl = static_cast<int>(j - j0);
+                    zs_s[m * zld + jl + (jl >> 5)] = z;
+                }
+                v = fmaxf(v, fabsf(z));
+            }
             for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
             if (lane == 0) s_wmax[warp][m] = v;
         }
@@ -195,13 +228,16 @@ __global__ void __launch_bounds__(kS1Threads, 1) decode_stage1_kernel(const S1Pa
     for (int m = 0; m < NQ_MATVEC_MAX_M; ++m) zsum[m] = 0;
 
     // ---- passes over the slice: z table, then MMAs; integer accumulators live in registers
-    int acc[2][NT][4];
+    // two accumulator sets, even and odd K steps, for two independent MMA chains per tile
+    int acc[2][2][NT][4];
 #pragma unroll
-    for (int h = 0; h < 2; ++h)
+    for (int par = 0; par < 2; ++par)
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
+        for (int h = 0; h < 2; ++h)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) acc[h][nt][e] = 0;
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[par][h][nt][e] = 0;
     const bool warp_active = (wglob0 + warp) < p.nw;
     const uint32_t msk = 0x01010101u << gid;
 
@@ -210,26 +246,52 @@ __global__ void __launch_bounds__(kS1Threads, 1) decode_stage1_kernel(const S1Pa
             __syncthreads();  // previous pass done with aws / zq
             build_aws(jb);
         }
-        // z digits: byte i of zq[jq][3m + q] = digit q of z_q(m, row jb + 4jq + i)
-        for (int i = tid; i < nq_rows * SWZ / 4; i += kS1Threads)
-            reinterpret_cast<uint4*>(zq)[i] = make_uint4(0u, 0u, 0u, 0u);
-        __syncthreads();
+        // z table: word zq[jq * SWZ + 3m + q] holds digit q of z_q(m, row jb + 4jq + i) in byte i;
+        // one thread builds the three digit words of one (jq, m) from four z values
         {
-            uint8_t* zb = reinterpret_cast<uint8_t*>(zq);
+            constexpr int MG = (NT * 8 + 2) / 3;
             const int64_t jend = min(j1, jb + p.jc_rows);
+            for (int e = tid; e < nq_rows * MG; e += kS1Threads) {
+                const int m = e % MG, jq = e / MG;  // MG is a compile-time constant
+                uint32_t d0 = 0u, d1 = 0u, d2 = 0u;
+                if (m < p.M) {
+                    const float mul = s_mul[m];
+                    const uint16_t* xm = p.x + static_cast<int64_t>(m) * p.d_in;
+                    float zv[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int64_t j = jb + 4 * jq + i;
+                        zv[i] = 0.0f;
+                        if (j < jend) {
+                            const int jl = static_cast<int>(j - j0);
+                            zv[i] = p.zstage ? zs_s[m * zld + jl + (jl >> 5)]
+                                             : f16_bits_to_float(p.s2[j]) * bf16_bits_to_float(xm[j]);
+                        }
+                    }
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        uint32_t a0, a1, a2;
+                        digits3(__float2int_rn(zv[i] * mul), a0, a1, a2);
+                        d0 |= a0 << (8 * i);
+                        d1 |= a1 << (8 * i);
+                        d2 |= a2 << (8 * i);
+                    }
+                }
+                uint32_t* dst = zq + jq * SWZ + 3 * m;
+                if (3 * m < NT * 8) dst[0] = d0;
+                if (3 * m + 1 < NT * 8) dst[1] = d1;
+                if (3 * m + 2 < NT * 8) dst[2] = d2;
+            }
             for (int m = 0; m < p.M; ++m) {
                 const uint16_t* xm = p.x + static_cast<int64_t>(m) * p.d_in;
                 const float mul = s_mul[m];
                 long long zs = 0;
 #pragma unroll 4
                 for (int64_t j = jb + tid; j < jend; j += kS1Threads) {
-                    const int v = __float2int_rn(f16_bits_to_float(p.s2[j]) * bf16_bits_to_float(xm[j]) * mul);
-                    zs += v;
-                    const int jl = static_cast<int>(j - jb);
-                    const int base = ((jl >> 2) * SWZ + 3 * m) * 4 + (jl & 3);
-                    zb[base] = static_cast<uint8_t>(digit_byte(v, 0));
-                    zb[base + 4] = static_cast<uint8_t>(digit_byte(v, 1));
-                    zb[base + 8] = static_cast<uint8_t>(digit_byte(v, 2));
+                    const int jl = static_cast<int>(j - j0);
+                    const float z = p.zstage ? zs_s[m * zld + jl + (jl >> 5)]
+                                             : f16_bits_to_float(p.s2[j]) * bf16_bits_to_float(xm[j]);
+                    zs += __float2int_rn(z * mul);
                 }
                 zsum[m] += zs;
             }
@@ -238,19 +300,25 @@ __global__ void __launch_bounds__(kS1Threads, 1) decode_stage1_kernel(const S1Pa
 
         if (warp_active) {
             const int w = warp;
-            for (int kb = 0; kb < nkb; ++kb) {
-                uint32_t bf[NT][2];
+            for (int kb2 = 0; kb2 < nkb; kb2 += 2) {
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    bf[nt][0] = zq[(8 * kb + tig) * SWZ + nt * 8 + gid];
-                    bf[nt][1] = zq[(8 * kb + 4 + tig) * SWZ + nt * 8 + gid];
-                }
+                for (int par = 0; par < 2; ++par) {
+                    const int kb = kb2 + par;
+                    if (kb < nkb) {
+                        uint32_t bf[NT][2];
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const uint4 a = *reinterpret_cast<const uint4*>(aws + (((w * nkb + kb) * 2 + h) * 4 + tig) * 4);
+                        for (int nt = 0; nt < NT; ++nt) {
+                            bf[nt][0] = zq[(8 * kb + tig) * SWZ + nt * 8 + gid];
+                            bf[nt][1] = zq[(8 * kb + 4 + tig) * SWZ + nt * 8 + gid];
+                        }
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt)
-                        mma_u8s8(acc[h][nt], a.x & msk, a.y & msk, a.z & msk, a.w & msk, bf[nt][0], bf[nt][1]);
+                        for (int h = 0; h < 2; ++h) {
+                            const uint4 a = *reinterpret_cast<const uint4*>(aws + w * (nkb * 32 + 4) + ((kb * 2 + h) * 4 + tig) * 4);
+#pragma unroll
+                            for (int nt = 0; nt < NT; ++nt)
+                                mma_u8s8(acc[par][h][nt], a.x & msk, a.y & msk, a.z & msk, a.w & msk, bf[nt][0], bf[nt][1]);
+                        }
+                    }
                 }
             }
         }
@@ -273,7 +341,7 @@ __global__ void __launch_bounds__(kS1Threads, 1) decode_stage1_kernel(const S1Pa
                 for (int e = 0; e < 4; ++e) {
                     const int kl = 32 * warp + 8 * (2 * h + (e >> 1)) + gid;
                     const int col = nt * 8 + 2 * tig + (e & 1);
-                    red[kl * (NT * 8) + col] = acc[h][nt][e] >> gid;
+                    red[kl * (NT * 8) + col] = (acc[0][h][nt][e] >> gid) + (acc[1][h][nt][e] >> gid);
                 }
     }
     __syncthreads();
@@ -295,11 +363,14 @@ __global__ void __launch_bounds__(kS1Threads, 1) decode_stage1_kernel(const S1Pa
             const int m = e / (k_hi - k_lo), kl = k_lo + (e - m * (k_hi - k_lo));
             const int64_t k = static_cast<int64_t>(wglob0) * 32 + kl;
             if (k < p.r) {
+                // all remote loads in flight together, then summed in rank order
+                double v[16];
+#pragma unroll
+                for (int rank = 0; rank < 16; ++rank)
+                    v[rank] = (rank < CS) ? cluster.map_shared_rank(part, rank)[m * kS1Outs + kl] : 0.0;
                 double sum = 0.0;
-                for (int rank = 0; rank < CS; ++rank) {
-                    const double* rp = cluster.map_shared_rank(part, rank);
-                    sum += rp[m * kS1Outs + kl];
-                }
+#pragma unroll
+                for (int rank = 0; rank < 16; ++rank) sum += v[rank];
                 p.t[static_cast<int64_t>(m) * p.r + k] = static_cast<float>(sum);
             }
         }
@@ -335,6 +406,7 @@ struct S2Params {
     int su;              // shared-memory row stride of U (words), = 4 (mod 32)
     int mt_total;        // 16-row M-tiles of U
     int chunk_mt;        // M-tiles staged in shared memory at a time
+    int tstage;          // t (M x r fp32) is copied into shared memory for the table build
 };
 
 template <int NT>
@@ -349,6 +421,7 @@ __global__ void __launch_bounds__(kS2Threads, 1) decode_stage2_kernel(const S2Pa
     uint32_t* bt = smem2;                                  // [8][nwp][SW]
     uint32_t* ublk = bt + 8 * p.nwp * SW;                  // [chunk_mt*16][su]
     int* red = reinterpret_cast<int*>(ublk + p.chunk_mt * 16 * p.su);  // [chunk_mt*16][NT*8]
+    float* ts_s = reinterpret_cast<float*>(red + p.chunk_mt * 16 * NT * 8);  // [M][r] when p.tstage
     __shared__ int s_shift[NQ_MATVEC_MAX_M];
     __shared__ float s_mul[NQ_MATVEC_MAX_M];
     __shared__ unsigned long long s_tsum[NQ_MATVEC_MAX_M];
@@ -390,13 +463,15 @@ __global__ void __launch_bounds__(kS2Threads, 1) decode_stage2_kernel(const S2Pa
 
     // ---- per-batch-row scale: |t_q| < 2^22 with t_q = rint(t * 2^shift)
     {
-        for (int i = tid; i < 2 * p.nwp * SW; i += kS2Threads)  // 8 * nwp * SW words, 16 B at a time
-            reinterpret_cast<uint4*>(bt)[i] = make_uint4(0u, 0u, 0u, 0u);
         for (int m = 0; m < p.M; ++m) {
             const float* tm = p.t + static_cast<int64_t>(m) * p.r;
             float v = 0.0f;
 #pragma unroll 8
-            for (int k = tid; k < p.r; k += kS2Threads) v = fmaxf(v, fabsf(tm[k]));
+            for (int k = tid; k < p.r; k += kS2Threads) {
+                const float tv = tm[k];
+                if (p.tstage) ts_s[m * (p.r + p.r / 32) + k + (k >> 5)] = tv;
+                v = fmaxf(v, fabsf(tv));
+            }
             for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
             if (lane == 0) s_wmax[warp][m] = v;
         }
@@ -411,22 +486,45 @@ __global__ void __launch_bounds__(kS2Threads, 1) decode_stage2_kernel(const S2Pa
             s_mul[tid] = ldexpf(1.0f, sh);
         }
         __syncthreads();
-        // quantise, scatter the three digits of t_q(m, k) into the B table, sum t_q:
-        // digit q of t_q(m, k) is byte (k mod 32) / 8 of word bt[((k mod 8) * nwp + k / 32) * SW + 3m + q]
-        uint8_t* btb = reinterpret_cast<uint8_t*>(bt);
+        // t staged with one pad word after every 32 values, so that the table build's
+        // stride-32 reads fall in different banks
+        const int tld = p.tstage ? p.r + p.r / 32 : p.r;
+        auto t_at = [&](int m, int k) -> float {
+            return p.tstage ? ts_s[m * tld + k + (k >> 5)] : p.t[static_cast<int64_t>(m) * p.r + k];
+        };
+        // B table: word bt[(s * nwp + w) * SW + 3m + q] holds digit q of t_q(m, 32w + s + 8b) in
+        // byte b; one thread builds the digit words of one (s, w) for every batch row
+        constexpr int MG = (NT * 8 + 2) / 3;  // column groups of three
+        for (int sw = tid; sw < 8 * p.nwp; sw += kS2Threads) {
+            const int s_ = sw / p.nwp, w = sw - s_ * p.nwp;
+            uint32_t* row = bt + sw * SW;
+#pragma unroll
+            for (int m = 0; m < MG; ++m) {
+                uint32_t d0 = 0u, d1 = 0u, d2 = 0u;
+                if (m < p.M && w < p.nw) {
+                    const float mul = s_mul[m];
+                    float tv[4];
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) tv[b] = t_at(m, 32 * w + s_ + 8 * b);
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) {
+                        uint32_t a0, a1, a2;
+                        digits3(__float2int_rn(tv[b] * mul), a0, a1, a2);
+                        d0 |= a0 << (8 * b);
+                        d1 |= a1 << (8 * b);
+                        d2 |= a2 << (8 * b);
+                    }
+                }
+                if (3 * m < NT * 8) row[3 * m] = d0;
+                if (3 * m + 1 < NT * 8) row[3 * m + 1] = d1;
+                if (3 * m + 2 < NT * 8) row[3 * m + 2] = d2;
+            }
+        }
         for (int m = 0; m < p.M; ++m) {
-            const float* tm = p.t + static_cast<int64_t>(m) * p.r;
             const float mul = s_mul[m];
             long long ts = 0;
 #pragma unroll 4
-            for (int k = tid; k < p.r; k += kS2Threads) {
-                const int v = __float2int_rn(tm[k] * mul);
-                ts += v;
-                const int base = (((k & 7) * p.nwp + (k >> 5)) * SW + 3 * m) * 4 + ((k >> 3) & 3);
-                btb[base] = static_cast<uint8_t>(digit_byte(v, 0));
-                btb[base + 4] = static_cast<uint8_t>(digit_byte(v, 1));
-                btb[base + 8] = static_cast<uint8_t>(digit_byte(v, 2));
-            }
+            for (int k = tid; k < p.r; k += kS2Threads) ts += __float2int_rn(t_at(m, k) * mul);
             ts = block_sum_i64(ts, s_red64);
             if (tid == 0) s_tsum[m] = static_cast<unsigned long long>(ts);
         }
@@ -442,33 +540,43 @@ __global__ void __launch_bounds__(kS2Threads, 1) decode_stage2_kernel(const S2Pa
         cp_async_wait_all();
         __syncthreads();
 
-        const int kp_count = max(1, min(ng, kS2Warps / nmt));
-        const int jobs = nmt * kp_count;
-        for (int job = warp; job < jobs; job += kS2Warps) {
-            const int mtl = job / kp_count, kp = job - mtl * kp_count;
-            const int g_lo = (kp * ng) / kp_count, g_hi = ((kp + 1) * ng) / kp_count;
+        // each warp takes an equal, contiguous share of the (M-tile, word-group) pairs in
+        // M-tile-major order and flushes its accumulators whenever its run leaves an M-tile
+        const int pairs = nmt * ng;
+        const int p_lo = (warp * pairs) / kS2Warps, p_hi = ((warp + 1) * pairs) / kS2Warps;
+        int pp = p_lo;
+        while (pp < p_hi) {
+            const int mtl = pp / ng;
+            const int g_lo = pp - mtl * ng;
+            const int g_hi = min(ng, g_lo + (p_hi - pp));
+            pp += g_hi - g_lo;
             int acc[8][NT][4];
 #pragma unroll
-            for (int s = 0; s < 8; ++s)
+            for (int s_ = 0; s_ < 8; ++s_)
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) acc[s][nt][e] = 0;
+                    for (int e = 0; e < 4; ++e) acc[s_][nt][e] = 0;
             const uint32_t* u0 = ublk + (mtl * 16 + gid) * p.su;
             const uint32_t* u1 = u0 + 8 * p.su;
+            uint32_t w00 = u0[8 * g_lo + tig], w01 = u0[8 * g_lo + 4 + tig];
+            uint32_t w10 = u1[8 * g_lo + tig], w11 = u1[8 * g_lo + 4 + tig];
             for (int g = g_lo; g < g_hi; ++g) {
                 const int wb = 8 * g;
-                const uint32_t w00 = u0[wb + tig], w01 = u0[wb + 4 + tig];
-                const uint32_t w10 = u1[wb + tig], w11 = u1[wb + 4 + tig];
+                // next group's words, loaded while this group's MMAs issue
+                const int wn = (g + 1 < g_hi) ? wb + 8 : wb;
+                const uint32_t n00 = u0[wn + tig], n01 = u0[wn + 4 + tig];
+                const uint32_t n10 = u1[wn + tig], n11 = u1[wn + 4 + tig];
 #pragma unroll
-                for (int s = 0; s < 8; ++s) {
-                    const uint32_t msk = 0x01010101u << s;
+                for (int s_ = 0; s_ < 8; ++s_) {
+                    const uint32_t msk = 0x01010101u << s_;
                     const uint32_t a0 = w00 & msk, a1 = w10 & msk, a2 = w01 & msk, a3 = w11 & msk;
-                    const uint32_t* b = bt + (s * p.nwp + wb) * SW;
+                    const uint32_t* b = bt + (s_ * p.nwp + wb) * SW;
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt)
-                        mma_u8s8(acc[s][nt], a0, a1, a2, a3, b[tig * SW + nt * 8 + gid], b[(4 + tig) * SW + nt * 8 + gid]);
+                        mma_u8s8(acc[s_][nt], a0, a1, a2, a3, b[tig * SW + nt * 8 + gid], b[(4 + tig) * SW + nt * 8 + gid]);
                 }
+                w00 = n00; w01 = n01; w10 = n10; w11 = n11;
             }
             // D[row][col]: e = 0,1 -> row gid, cols 2tig, 2tig+1; e = 2,3 -> row gid+8
 #pragma unroll
@@ -477,7 +585,7 @@ __global__ void __launch_bounds__(kS2Threads, 1) decode_stage2_kernel(const S2Pa
                 for (int e = 0; e < 4; ++e) {
                     int v = 0;
 #pragma unroll
-                    for (int s = 0; s < 8; ++s) v += acc[s][nt][e] >> s;
+                    for (int s_ = 0; s_ < 8; ++s_) v += acc[s_][nt][e] >> s_;
                     const int row = mtl * 16 + gid + ((e >> 1) << 3);
                     const int col = nt * 8 + 2 * tig + (e & 1);
                     atomicAdd(&red[row * (NT * 8) + col], v);
@@ -517,7 +625,7 @@ constexpr size_t kStage2SmemBudget = 200 * 1024;
 int ntiles_for(int64_t M) { return static_cast<int>((3 * M + 7) / 8); }
 
 struct S1Plan {
-    int n_chunks, CS, rows_per_slice, jc_rows;
+    int n_chunks, CS, rows_per_slice, jc_rows, zstage;
     size_t smem;
 };
 
@@ -531,12 +639,16 @@ S1Plan plan_stage1(int64_t d_in, int64_t r, int64_t M) {
     p.rows_per_slice = static_cast<int>(((d_in + cs - 1) / cs + 31) / 32 * 32);
     const int nt = ntiles_for(M);
     const int swz = nt == 1 ? 8 : 24;
-    const size_t fixed = static_cast<size_t>(nq::kS1Outs) * nt * 8 * 4 + static_cast<size_t>(M) * nq::kS1Outs * 8;
+    const size_t fixed = static_cast<size_t>(nq::kS1Outs) * nt * 8 * 4 + static_cast<size_t>(M) * nq::kS1Outs * 8 +
+                         nq::kS1Words * 16;
     int64_t jc = static_cast<int64_t>((kStage1SmemBudget - fixed) / (32 + swz)) / 32 * 32;
     if (jc > p.rows_per_slice) jc = p.rows_per_slice;
     if (jc < 32) jc = 32;
     p.jc_rows = static_cast<int>(jc);
-    p.smem = static_cast<size_t>(jc) * (32 + swz) + fixed;
+    p.smem = static_cast<size_t>(jc) * (32 + swz) + fixed + nq::kS1Words * 16;
+    const size_t z_bytes = static_cast<size_t>(M) * (p.rows_per_slice + p.rows_per_slice / 32) * sizeof(float);
+    p.zstage = (p.smem + z_bytes <= kStage1SmemBudget && z_bytes <= 48 * 1024) ? 1 : 0;
+    if (p.zstage) p.smem += z_bytes;
     return p;
 }
 
@@ -575,6 +687,7 @@ nq_status launch_decode_nt(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y
         q.nw = static_cast<int>(L->r / 32);
         q.rows_per_slice = sp.rows_per_slice;
         q.jc_rows = sp.jc_rows;
+        q.zstage = sp.zstage;
         void* args[] = {&q};
         if (nq_host::launch_ex(reinterpret_cast<const void*>(nq::decode_stage1_kernel<NT>),
                                dim3(sp.n_chunks, sp.CS), dim3(nq::kS1Threads), sp.smem, stream, args, pdl,
@@ -604,7 +717,10 @@ nq_status launch_decode_nt(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y
         if (bt_bytes + chunk * per_mt > kStage2SmemBudget) chunk = static_cast<int>((kStage2SmemBudget - bt_bytes) / per_mt);
         if (chunk < 1) return NQ_ERR_SHAPE;
         q.chunk_mt = chunk;
-        const size_t smem2 = bt_bytes + chunk * per_mt;
+        size_t smem2 = bt_bytes + chunk * per_mt;
+        const size_t t_bytes = static_cast<size_t>(M) * (L->r + L->r / 32) * sizeof(float);
+        q.tstage = (smem2 + t_bytes <= kStage2SmemBudget && t_bytes <= 48 * 1024) ? 1 : 0;
+        if (q.tstage) smem2 += t_bytes;
         void* args[] = {&q};
         if (nq_host::launch_ex(reinterpret_cast<const void*>(nq::decode_stage2_kernel<NT>), dim3(grid),
                                dim3(nq::kS2Threads), smem2, stream, args, pdl, 1) != cudaSuccess)

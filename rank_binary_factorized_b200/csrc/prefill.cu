@@ -183,57 +183,73 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     } else if (warp < 6) {
         // ---------------------------------------------------------------- A expansion (weights)
         const int t = threadIdx.x - 64;  // 0..127
-        uint32_t it = 0;
-        bool ok = true;
-        for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+        // The two packed words of iteration `j` (tile, k block) of this CTA.  Loads run
+        // kPrefetch iterations ahead of their use in a register ring, so the L2/DRAM latency
+        // of the words overlaps the expansion and the waits of the iterations before.
+        auto load_words = [&](uint32_t j, uint32_t& w0, uint32_t& w1) {
+            w0 = 0u;
+            w1 = 0u;
+            const int tile = blockIdx.x + static_cast<int>(j / nkb) * gridDim.x;
+            if (tile >= n_tiles) return;
+            const int kb = static_cast<int>(j % nkb);
             const int tw = tile % args.n_tiles_w;
-            for (int kb = 0; kb < nkb; ++kb, ++it) {
-                const int s = it % kStages;
-                const uint32_t ph = (it / kStages) & 1u;
-                // load this thread's two words before waiting for the stage
-                uint32_t w0 = 0u, w1 = 0u;
-                int64_t row, wcol;
-                if (MODE == kModeU) {
-                    row = static_cast<int64_t>(tw) * kTileW + t;  // output row i
-                    wcol = static_cast<int64_t>(kb) * 2;          // words of k = 64 kb .. 64 kb + 63
-                    if (row < args.rows_w) {
-                        const uint32_t* p = args.bits + row * args.ld + wcol;
-                        if (wcol < args.nwords) w0 = __ldg(p);
-                        if (wcol + 1 < args.nwords) w1 = __ldg(p + 1);
-                    }
-                } else {
-                    row = static_cast<int64_t>(kb) * kTileK + (t >> 1);             // input feature j
-                    wcol = static_cast<int64_t>(tw) * (kTileW / 32) + (t & 1) * 2;  // words of k
-                    if (row < args.K) {
-                        const uint32_t* p = args.bits + row * args.ld + wcol;
-                        if (wcol < args.nwords) w0 = __ldg(p);
-                        if (wcol + 1 < args.nwords) w1 = __ldg(p + 1);
-                    }
-                }
-                if (!(ok = tc::mbar_wait(empty(s), ph ^ 1u, err))) break;
-                const uint32_t a = a_tile(s);
-                if (MODE == kModeU) {
-                    // row t of a K-major SW128 tile: 8 chunks of 16 B, chunk c holds K = 8c .. 8c+7
-                    const uint32_t row_base = a + (t >> 3) * 1024u + (t & 7) * 128u;
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const uint32_t byte = ((c < 4 ? w0 : w1) >> (8 * (c & 3))) & 0xFFu;
-                        sts128(row_base + ((c ^ (t & 7)) << 4), expand_byte_pm1(byte));
-                    }
-                } else {
-                    // K-row j_local = t/2 of an MN-major SW128 tile; this thread's 64 M-elements
-                    // (k) are words q = 2(t&1), 2(t&1)+1 of the tile's four, i.e. M-group t&1
-                    const int jl = t >> 1;
-                    const uint32_t atom = a + ((jl >> 3) * 2 + (t & 1)) * 1024u + (jl & 7) * 128u;
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const uint32_t byte = ((c < 4 ? w0 : w1) >> (8 * (c & 3))) & 0xFFu;
-                        sts128(atom + ((c ^ (jl & 7)) << 4), expand_byte_pm1(byte));
-                    }
-                }
-                tc::fence_proxy_async_smem();
-                tc::mbar_arrive(full_a(s));
+            int64_t row, wcol;
+            bool row_ok;
+            if (MODE == kModeU) {
+                row = static_cast<int64_t>(tw) * kTileW + t;  // output row i
+                wcol = static_cast<int64_t>(kb) * 2;          // words of k = 64 kb .. 64 kb + 63
+                row_ok = row < args.rows_w;
+            } else {
+                row = static_cast<int64_t>(kb) * kTileK + (t >> 1);             // input feature j
+                wcol = static_cast<int64_t>(tw) * (kTileW / 32) + (t & 1) * 2;  // words of k
+                row_ok = row < args.K;
             }
+            if (row_ok) {
+                const uint32_t* p = args.bits + row * args.ld + wcol;
+                if (wcol < args.nwords) w0 = __ldg(p);
+                if (wcol + 1 < args.nwords) w1 = __ldg(p + 1);
+            }
+        };
+        constexpr int kPrefetch = 4;
+        uint32_t ring0[kPrefetch], ring1[kPrefetch];
+#pragma unroll
+        for (int i = 0; i < kPrefetch; ++i) load_words(static_cast<uint32_t>(i), ring0[i], ring1[i]);
+        const int my_tiles = (n_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x);
+        const uint32_t total_it = static_cast<uint32_t>(my_tiles > 0 ? my_tiles : 0) * static_cast<uint32_t>(nkb);
+        bool ok = true;
+        for (uint32_t it = 0; it < total_it && ok; ++it) {
+            const int s = it % kStages;
+            const uint32_t ph = (it / kStages) & 1u;
+            const uint32_t w0 = ring0[0], w1 = ring1[0];
+#pragma unroll
+            for (int i = 0; i + 1 < kPrefetch; ++i) {
+                ring0[i] = ring0[i + 1];
+                ring1[i] = ring1[i + 1];
+            }
+            load_words(it + kPrefetch, ring0[kPrefetch - 1], ring1[kPrefetch - 1]);
+            if (!(ok = tc::mbar_wait(empty(s), ph ^ 1u, err))) break;
+            const uint32_t a = a_tile(s);
+            if (MODE == kModeU) {
+                // row t of a K-major SW128 tile: 8 chunks of 16 B, chunk c holds K = 8c .. 8c+7
+                const uint32_t row_base = a + (t >> 3) * 1024u + (t & 7) * 128u;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint32_t byte = ((c < 4 ? w0 : w1) >> (8 * (c & 3))) & 0xFFu;
+                    sts128(row_base + ((c ^ (t & 7)) << 4), expand_byte_pm1(byte));
+                }
+            } else {
+                // K-row j_local = t/2 of an MN-major SW128 tile; this thread's 64 M-elements
+                // (k) are words q = 2(t&1), 2(t&1)+1 of the tile's four, i.e. M-group t&1
+                const int jl = t >> 1;
+                const uint32_t atom = a + ((jl >> 3) * 2 + (t & 1)) * 1024u + (jl & 7) * 128u;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint32_t byte = ((c < 4 ? w0 : w1) >> (8 * (c & 3))) & 0xFFu;
+                    sts128(atom + ((c ^ (jl & 7)) << 4), expand_byte_pm1(byte));
+                }
+            }
+            tc::fence_proxy_async_smem();
+            tc::mbar_arrive(full_a(s));
         }
     } else {
         // ---------------------------------------------------------------- epilogue
