@@ -91,7 +91,10 @@ __device__ __forceinline__ long long block_sum_i64(long long v, long long* scrat
 // chunk's outputs over the CS blocks' shared memory (distributed shared memory) in rank
 // order and writes t.  No atomics, no global partials: deterministic.
 
-constexpr int kS1Threads = 256;
+// Threads per stage-1 block: 256 (one warp per word column) or 512 (two warps per word column,
+// each half of the K range).  512 hides more latency on long row slices but fills the
+// register file, so the block can no longer share an SM with the previous kernel's blocks
+// under programmatic dependent launch; the host picks 512 only for long slices and NT <= 2.
 constexpr int kS1Words = 8;            // words (of 32 outputs) per cluster chunk
 constexpr int kS1Outs = kS1Words * 32;  // outputs k per chunk
 
@@ -126,8 +129,10 @@ __device__ __forceinline__ void byte_transpose4(uint32_t w0, uint32_t w1, uint32
     o[3] = __byte_perm(t1, t3, 0x7632);
 }
 
-template <int NT>
-__global__ void __launch_bounds__(kS1Threads, 1) decode_stage1_kernel(const S1Params p) {
+template <int NT, int TH>
+__global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const S1Params p) {
+    constexpr int kS1Threads = TH;
+    constexpr int kKSplit = kS1Threads / (32 * kS1Words);  // warps per word column
     namespace cg = cooperative_groups;
     constexpr int SWZ = S1Layout<NT>::SWZ;
     extern __shared__ __align__(16) uint32_t smem1[];
@@ -136,8 +141,8 @@ __global__ void __launch_bounds__(kS1Threads, 1) decode_stage1_kernel(const S1Pa
     uint32_t* aws = smem1;                          // [8 words][nkb][2][4][4]
     uint32_t* zq = aws + kS1Words * (nkb * 32 + 4);  // [nq_rows][SWZ]
     int* red = reinterpret_cast<int*>(zq + nq_rows * SWZ);               // [256][NT*8]
-    double* part = reinterpret_cast<double*>(red + kS1Outs * NT * 8);   // [M][256]
-    float* zs_s = reinterpret_cast<float*>(part + p.M * kS1Outs);         // [M][zld] when p.zstage
+    double* part = reinterpret_cast<double*>(red + kS1Outs * NT * 8);   // inbox [M][per][CS]
+    float* zs_s = reinterpret_cast<float*>(part + p.M * (kS1Outs + 16));  // [M][zld] when p.zstage
     const int zld = p.rows_per_slice + p.rows_per_slice / 32;             // one pad word per 32
     __shared__ int s_shift[NQ_MATVEC_MAX_M];
     __shared__ float s_mul[NQ_MATVEC_MAX_M];
@@ -198,7 +203,7 @@ __global__ void __launch_bounds__(kS1Threads, 1) decode_stage1_kernel(const S1Pa
         for (int m = 0; m < p.M; ++m) {
             const uint16_t* xm = p.x + static_cast<int64_t>(m) * p.d_in;
             float v = 0.0f;
-#pragma unroll 4
+#pragma unroll 8
             for (int64_t j = j0 + tid; j < j1; j += kS1Threads) {
                 const float z = f16_bits_to_float(p.s2[j]) * bf16_bits_to_float(xm[j]);
                 if (p.zstage) {
@@ -238,7 +243,9 @@ __global__ void __launch_bounds__(kS1Threads, 1) decode_stage1_kernel(const S1Pa
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) acc[par][h][nt][e] = 0;
-    const bool warp_active = (wglob0 + warp) < p.nw;
+    const int wcol = warp % kS1Words;          // word column of this warp
+    const int khalf = warp / kS1Words;         // which share of the K steps
+    const bool warp_active = (wglob0 + wcol) < p.nw;
     const uint32_t msk = 0x01010101u << gid;
 
     for (int64_t jb = j0; jb < j1; jb += p.jc_rows) {
@@ -299,12 +306,13 @@ __global__ void __launch_bounds__(kS1Threads, 1) decode_stage1_kernel(const S1Pa
         __syncthreads();
 
         if (warp_active) {
-            const int w = warp;
-            for (int kb2 = 0; kb2 < nkb; kb2 += 2) {
+            const int w = wcol;
+            const int kb_lo = (khalf * nkb) / kKSplit, kb_hi = ((khalf + 1) * nkb) / kKSplit;
+            for (int kb2 = kb_lo; kb2 < kb_hi; kb2 += 2) {
 #pragma unroll
                 for (int par = 0; par < 2; ++par) {
                     const int kb = kb2 + par;
-                    if (kb < nkb) {
+                    if (kb < kb_hi) {
                         uint32_t bf[NT][2];
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt) {
@@ -339,43 +347,41 @@ __global__ void __launch_bounds__(kS1Threads, 1) decode_stage1_kernel(const S1Pa
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const int kl = 32 * warp + 8 * (2 * h + (e >> 1)) + gid;
+                    const int kl = 32 * wcol + 8 * (2 * h + (e >> 1)) + gid;
                     const int col = nt * 8 + 2 * tig + (e & 1);
-                    red[kl * (NT * 8) + col] = (acc[0][h][nt][e] >> gid) + (acc[1][h][nt][e] >> gid);
+                    atomicAdd(&red[kl * (NT * 8) + col], (acc[0][h][nt][e] >> gid) + (acc[1][h][nt][e] >> gid));
                 }
     }
     __syncthreads();
+    // ---- cluster reduction over the CS row slices.  Output k of the chunk belongs to the
+    // block of rank k / per; every block stores its fp64 partial for k into slot [rank of
+    // the sender] of the owner's inbox (distributed shared memory), one cluster barrier
+    // publishes the stores, and each owner sums its slots in rank order.
+    const int per = (kS1Outs + CS - 1) / CS;
     for (int e = tid; e < p.M * kS1Outs; e += kS1Threads) {
         const int m = e / kS1Outs, kl = e - m * kS1Outs;
         const int* rr = red + kl * (NT * 8) + 3 * m;
         const long long P = static_cast<long long>(rr[0]) + (static_cast<long long>(rr[1]) << 8) +
                             (static_cast<long long>(rr[2]) << 16);
         const long long val = 2 * P - static_cast<long long>(s_zsum[m]);
-        part[m * kS1Outs + kl] = ldexp(static_cast<double>(val), -s_shift[m]);
+        const int owner = kl / per, ko = kl - owner * per;
+        double* dst = cluster.map_shared_rank(part, owner);
+        dst[(m * per + ko) * CS + q] = ldexp(static_cast<double>(val), -s_shift[m]);
     }
-
-    // ---- cluster reduction over the CS row slices, rank order
     cluster.sync();
     {
-        const int per = (kS1Outs + CS - 1) / CS;
         const int k_lo = q * per, k_hi = min(kS1Outs, k_lo + per);
         for (int e = tid; e < p.M * (k_hi - k_lo); e += kS1Threads) {
-            const int m = e / (k_hi - k_lo), kl = k_lo + (e - m * (k_hi - k_lo));
-            const int64_t k = static_cast<int64_t>(wglob0) * 32 + kl;
+            const int m = e / (k_hi - k_lo), ko = e - m * (k_hi - k_lo);
+            const int64_t k = static_cast<int64_t>(wglob0) * 32 + k_lo + ko;
             if (k < p.r) {
-                // all remote loads in flight together, then summed in rank order
-                double v[16];
-#pragma unroll
-                for (int rank = 0; rank < 16; ++rank)
-                    v[rank] = (rank < CS) ? cluster.map_shared_rank(part, rank)[m * kS1Outs + kl] : 0.0;
+                const double* src = part + (m * per + ko) * CS;
                 double sum = 0.0;
-#pragma unroll
-                for (int rank = 0; rank < 16; ++rank) sum += v[rank];
+                for (int rank = 0; rank < CS; ++rank) sum += src[rank];
                 p.t[static_cast<int64_t>(m) * p.r + k] = static_cast<float>(sum);
             }
         }
     }
-    cluster.sync();  // keep this block's shared memory alive until every peer has read it
 }
 
 // ------------------------------------------------------------------ stage 2 (integer MMA)
@@ -391,8 +397,7 @@ __global__ void __launch_bounds__(kS1Threads, 1) decode_stage1_kernel(const S1Pa
 // shifted back (exactly: each is a multiple of 2^s) and summed.  Everything up to the final
 // scale is integer arithmetic, so the result is exact for the quantised t and independent of
 // summation order.
-constexpr int kS2Threads = 256;
-constexpr int kS2Warps = kS2Threads / 32;
+// Threads per stage-2 block: 256, or 512 for many M-tiles per block at NT = 1 (see stage 1).
 
 struct S2Params {
     const uint32_t* U;
@@ -414,8 +419,10 @@ struct S2Layout {
     static constexpr int SW = (NT == 1) ? 8 : 24;  // words per (s, w) entry row of the B table
 };
 
-template <int NT>
-__global__ void __launch_bounds__(kS2Threads, 1) decode_stage2_kernel(const S2Params p) {
+template <int NT, int TH>
+__global__ void __launch_bounds__(TH, 1) decode_stage2_kernel(const S2Params p) {
+    constexpr int kS2Threads = TH;
+    constexpr int kS2Warps = kS2Threads / 32;
     extern __shared__ __align__(16) uint32_t smem2[];
     constexpr int SW = S2Layout<NT>::SW;
     uint32_t* bt = smem2;                                  // [8][nwp][SW]
@@ -639,7 +646,7 @@ S1Plan plan_stage1(int64_t d_in, int64_t r, int64_t M) {
     p.rows_per_slice = static_cast<int>(((d_in + cs - 1) / cs + 31) / 32 * 32);
     const int nt = ntiles_for(M);
     const int swz = nt == 1 ? 8 : 24;
-    const size_t fixed = static_cast<size_t>(nq::kS1Outs) * nt * 8 * 4 + static_cast<size_t>(M) * nq::kS1Outs * 8 +
+    const size_t fixed = static_cast<size_t>(nq::kS1Outs) * nt * 8 * 4 + static_cast<size_t>(M) * (nq::kS1Outs + 16) * 8 +
                          nq::kS1Words * 16;
     int64_t jc = static_cast<int64_t>((kStage1SmemBudget - fixed) / (32 + swz)) / 32 * 32;
     if (jc > p.rows_per_slice) jc = p.rows_per_slice;
@@ -654,16 +661,16 @@ S1Plan plan_stage1(int64_t d_in, int64_t r, int64_t M) {
 
 size_t decode_ws_bytes(int64_t r, int64_t M) { return kWsHeader + align256(static_cast<size_t>(M * r) * sizeof(float)); }
 
-template <int NT>
+template <int NT, int TH1, int TH2>
 void set_attrs_once() {
     static bool done[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || done[dev]) return;
-    cudaFuncSetAttribute(nq::decode_stage1_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(nq::decode_stage1_kernel<NT, TH1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(kStage1SmemBudget));
-    cudaFuncSetAttribute(nq::decode_stage1_kernel<NT>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    cudaFuncSetAttribute(nq::decode_stage2_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(nq::decode_stage1_kernel<NT, TH1>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    cudaFuncSetAttribute(nq::decode_stage2_kernel<NT, TH2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(kStage2SmemBudget));
     done[dev] = true;
 }
@@ -671,7 +678,6 @@ void set_attrs_once() {
 template <int NT>
 nq_status launch_decode_nt(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y, int M, void* ws,
                            cudaStream_t stream, bool pdl) {
-    set_attrs_once<NT>();
     float* t = reinterpret_cast<float*>(static_cast<char*>(ws) + kWsHeader);
     {
         const S1Plan sp = plan_stage1(L->d_in, L->r, M);
@@ -689,8 +695,12 @@ nq_status launch_decode_nt(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y
         q.jc_rows = sp.jc_rows;
         q.zstage = sp.zstage;
         void* args[] = {&q};
-        if (nq_host::launch_ex(reinterpret_cast<const void*>(nq::decode_stage1_kernel<NT>),
-                               dim3(sp.n_chunks, sp.CS), dim3(nq::kS1Threads), sp.smem, stream, args, pdl,
+        const bool wide = (NT <= 2) && sp.rows_per_slice >= 1024;
+        const void* fn = wide ? reinterpret_cast<const void*>(nq::decode_stage1_kernel<NT, (NT <= 2 ? 512 : 256)>)
+                              : reinterpret_cast<const void*>(nq::decode_stage1_kernel<NT, 256>);
+        if (wide) set_attrs_once<NT, (NT <= 2 ? 512 : 256), 256>();
+        else set_attrs_once<NT, 256, 256>();
+        if (nq_host::launch_ex(fn, dim3(sp.n_chunks, sp.CS), dim3(wide ? 512 : 256), sp.smem, stream, args, pdl,
                                sp.CS) != cudaSuccess)
             return NQ_ERR_LAUNCH;
     }
@@ -722,8 +732,12 @@ nq_status launch_decode_nt(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y
         q.tstage = (smem2 + t_bytes <= kStage2SmemBudget && t_bytes <= 48 * 1024) ? 1 : 0;
         if (q.tstage) smem2 += t_bytes;
         void* args[] = {&q};
-        if (nq_host::launch_ex(reinterpret_cast<const void*>(nq::decode_stage2_kernel<NT>), dim3(grid),
-                               dim3(nq::kS2Threads), smem2, stream, args, pdl, 1) != cudaSuccess)
+        const bool wide = (NT == 1) && per_cta >= 6;
+        const void* fn = wide ? reinterpret_cast<const void*>(nq::decode_stage2_kernel<NT, (NT == 1 ? 512 : 256)>)
+                              : reinterpret_cast<const void*>(nq::decode_stage2_kernel<NT, 256>);
+        if (wide) set_attrs_once<NT, 256, (NT == 1 ? 512 : 256)>();
+        else set_attrs_once<NT, 256, 256>();
+        if (nq_host::launch_ex(fn, dim3(grid), dim3(wide ? 512 : 256), smem2, stream, args, pdl, 1) != cudaSuccess)
             return NQ_ERR_LAUNCH;
     }
     return NQ_OK;

@@ -52,14 +52,14 @@ struct PrefillArgs {
 
 // fp16 +1 = 0x3C00, -1 = 0xBC00; two elements per 32-bit word, element 2i in the low half.
 // Expands the 8 bits of `byte` (element e = bit e) into 8 fp16 values (16 bytes).
-__device__ __forceinline__ uint4 expand_byte_pm1(uint32_t byte) {
-    const uint32_t nb = ~byte;
+// `nbyte` holds the complemented bits (1 = negative) in its low 8 bits and zeros above.
+// For pair q, (nbyte >> 2q) * 0x40008000 puts bit 2q at bit 15 and bit 2q+1 at bit 31: the
+// product's two shifted copies occupy bits 15..22 and 30..31 (higher bits fall off), so they
+// never overlap and no carry disturbs the two sign positions.
+__device__ __forceinline__ uint4 expand_nbyte_pm1(uint32_t nbyte) {
     uint32_t r[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const uint32_t two = (nb >> (2 * q)) & 3u;  // bit0 -> element 2q, bit1 -> element 2q+1 (1 = negative)
-        r[q] = 0x3C003C00u | ((two * 0x40008000u) & 0x80008000u);
-    }
+    for (int q = 0; q < 4; ++q) r[q] = 0x3C003C00u | (((nbyte >> (2 * q)) * 0x40008000u) & 0x80008000u);
     return make_uint4(r[0], r[1], r[2], r[3]);
 }
 
@@ -200,8 +200,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 wcol = static_cast<int64_t>(kb) * 2;          // words of k = 64 kb .. 64 kb + 63
                 row_ok = row < args.rows_w;
             } else {
-                row = static_cast<int64_t>(kb) * kTileK + (t >> 1);             // input feature j
-                wcol = static_cast<int64_t>(tw) * (kTileW / 32) + (t & 1) * 2;  // words of k
+                const int jl = (t & 7) | ((t >> 4) << 3), h = (t >> 3) & 1;
+                row = static_cast<int64_t>(kb) * kTileK + jl;                  // input feature j
+                wcol = static_cast<int64_t>(tw) * (kTileW / 32) + h * 2;       // words of k
                 row_ok = row < args.K;
             }
             if (row_ok) {
@@ -229,23 +230,26 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             load_words(it + kPrefetch, ring0[kPrefetch - 1], ring1[kPrefetch - 1]);
             if (!(ok = tc::mbar_wait(empty(s), ph ^ 1u, err))) break;
             const uint32_t a = a_tile(s);
+            const uint32_t n0 = ~w0, n1 = ~w1;
             if (MODE == kModeU) {
                 // row t of a K-major SW128 tile: 8 chunks of 16 B, chunk c holds K = 8c .. 8c+7
                 const uint32_t row_base = a + (t >> 3) * 1024u + (t & 7) * 128u;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
-                    const uint32_t byte = ((c < 4 ? w0 : w1) >> (8 * (c & 3))) & 0xFFu;
-                    sts128(row_base + ((c ^ (t & 7)) << 4), expand_byte_pm1(byte));
+                    const uint32_t nbyte = ((c < 4 ? n0 : n1) >> (8 * (c & 3))) & 0xFFu;
+                    sts128(row_base + ((c ^ (t & 7)) << 4), expand_nbyte_pm1(nbyte));
                 }
             } else {
-                // K-row j_local = t/2 of an MN-major SW128 tile; this thread's 64 M-elements
-                // (k) are words q = 2(t&1), 2(t&1)+1 of the tile's four, i.e. M-group t&1
-                const int jl = t >> 1;
-                const uint32_t atom = a + ((jl >> 3) * 2 + (t & 1)) * 1024u + (jl & 7) * 128u;
+                // K-row jl of an MN-major SW128 tile; this thread's 64 M-elements (k) are words
+                // 2h, 2h+1 of the tile's four, i.e. M-group h.  Lanes 0..7 of each 8-lane group
+                // take eight different K-rows (distinct swizzle phases, conflict-free stores).
+                const int jl = (t & 7) | ((t >> 4) << 3);
+                const int h = (t >> 3) & 1;
+                const uint32_t atom = a + ((jl >> 3) * 2 + h) * 1024u + (jl & 7) * 128u;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
-                    const uint32_t byte = ((c < 4 ? w0 : w1) >> (8 * (c & 3))) & 0xFFu;
-                    sts128(atom + ((c ^ (jl & 7)) << 4), expand_byte_pm1(byte));
+                    const uint32_t nbyte = ((c < 4 ? n0 : n1) >> (8 * (c & 3))) & 0xFFu;
+                    sts128(atom + ((c ^ (jl & 7)) << 4), expand_nbyte_pm1(nbyte));
                 }
             }
             tc::fence_proxy_async_smem();
