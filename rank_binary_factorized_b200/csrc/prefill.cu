@@ -30,7 +30,9 @@ constexpr int kTileW = 128;       // MMA M: weight rows per tile
 constexpr int kTileK = 64;        // K per pipeline stage (one 128-byte swizzle row of fp16)
 constexpr int kStages = 4;
 constexpr int kTmemCols = 512;
-constexpr int kPrefillThreads = 320;  // warp 0 TMA, warp 1 MMA + TMEM, warps 2-5 expand, 6-9 epilogue
+constexpr int kExpandWarps = 8;     // warps 2..9 expand the packed weights
+constexpr int kEpiWarp0 = 2 + kExpandWarps;  // warps 10..13: epilogue
+constexpr int kPrefillThreads = 32 * (kEpiWarp0 + 4);
 constexpr int kABytes = kTileW * kTileK * 2;  // 16 KB
 
 enum PrefillMode : int { kModeV = 0, kModeU = 1 };
@@ -94,13 +96,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            tc::mbar_init(full_a(s), 128);
+            tc::mbar_init(full_a(s), kExpandWarps);
             tc::mbar_init(full_b(s), 1);
             tc::mbar_init(empty(s), 1);
         }
         for (int a = 0; a < 2; ++a) {
             tc::mbar_init(acc_full(a), 1);
-            tc::mbar_init(acc_empty(a), 128);
+            tc::mbar_init(acc_empty(a), 4);
         }
         tc::mbar_init(drain_bar, 1);
         tc::mbar_fence_init();
@@ -180,80 +182,87 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             tc::mma_commit(drain_bar);
             tc::mbar_wait(drain_bar, 0u, err);
         }
-    } else if (warp < 6) {
+    } else if (warp < kEpiWarp0) {
         // ---------------------------------------------------------------- A expansion (weights)
-        const int t = threadIdx.x - 64;  // 0..127
+        // 256 threads, one packed word (32 weights) per thread per k block:
+        //  U (K-major): row = t / 2, word 2 kb + (t & 1) -> chunks 4 (t & 1) .. +3 of the row
+        //  V (MN-major): K-row jl, M-group h, word `half` of that group; lanes 0..7 of every
+        //  8-lane group take eight different K-rows so their 16-byte stores hit distinct banks
+        const int t = threadIdx.x - 64;  // 0..255
         // The two packed words of iteration `j` (tile, k block) of this CTA.  Loads run
         // kPrefetch iterations ahead of their use in a register ring, so the L2/DRAM latency
         // of the words overlaps the expansion and the waits of the iterations before.
-        auto load_words = [&](uint32_t j, uint32_t& w0, uint32_t& w1) {
-            w0 = 0u;
-            w1 = 0u;
-            const int tile = blockIdx.x + static_cast<int>(j / nkb) * gridDim.x;
-            if (tile >= n_tiles) return;
-            const int kb = static_cast<int>(j % nkb);
-            const int tw = tile % args.n_tiles_w;
-            int64_t row, wcol;
-            bool row_ok;
-            if (MODE == kModeU) {
-                row = static_cast<int64_t>(tw) * kTileW + t;  // output row i
-                wcol = static_cast<int64_t>(kb) * 2;          // words of k = 64 kb .. 64 kb + 63
-                row_ok = row < args.rows_w;
-            } else {
-                const int jl = (t & 7) | ((t >> 4) << 3), h = (t >> 3) & 1;
-                row = static_cast<int64_t>(kb) * kTileK + jl;                  // input feature j
-                wcol = static_cast<int64_t>(tw) * (kTileW / 32) + h * 2;       // words of k
-                row_ok = row < args.K;
-            }
-            if (row_ok) {
-                const uint32_t* p = args.bits + row * args.ld + wcol;
-                if (wcol < args.nwords) w0 = __ldg(p);
-                if (wcol + 1 < args.nwords) w1 = __ldg(p + 1);
+        // Per-thread constants of the word this thread expands, and a cursor (tile, k block)
+        // for the prefetch that runs kPrefetch iterations ahead; advanced by increments only.
+        int64_t row_off;  // row index within a tile (U) or within a k block (V)
+        int word_off;     // word offset within the k block (U) or within the tile's 4 words (V)
+        if (MODE == kModeU) {
+            row_off = t >> 1;
+            word_off = t & 1;
+        } else {
+            row_off = (t & 7) | ((t >> 5) << 3);
+            word_off = ((t >> 4) & 1) * 2 + ((t >> 3) & 1);
+        }
+        int pf_tile = blockIdx.x, pf_kb = 0, pf_tw = blockIdx.x % args.n_tiles_w;
+        auto load_next = [&](uint32_t& w) {
+            w = 0u;
+            if (pf_tile < n_tiles) {
+                int64_t row, wcol;
+                bool row_ok;
+                if (MODE == kModeU) {
+                    row = static_cast<int64_t>(pf_tw) * kTileW + row_off;
+                    wcol = static_cast<int64_t>(pf_kb) * 2 + word_off;
+                    row_ok = row < args.rows_w;
+                } else {
+                    row = static_cast<int64_t>(pf_kb) * kTileK + row_off;
+                    wcol = static_cast<int64_t>(pf_tw) * (kTileW / 32) + word_off;
+                    row_ok = row < args.K;
+                }
+                if (row_ok && wcol < args.nwords) w = __ldg(args.bits + row * args.ld + wcol);
+                if (++pf_kb == nkb) {
+                    pf_kb = 0;
+                    pf_tile += gridDim.x;
+                    pf_tw += gridDim.x;
+                    while (pf_tw >= args.n_tiles_w) pf_tw -= args.n_tiles_w;
+                }
             }
         };
         constexpr int kPrefetch = 4;
-        uint32_t ring0[kPrefetch], ring1[kPrefetch];
+        uint32_t ring[kPrefetch];
 #pragma unroll
-        for (int i = 0; i < kPrefetch; ++i) load_words(static_cast<uint32_t>(i), ring0[i], ring1[i]);
+        for (int i = 0; i < kPrefetch; ++i) load_next(ring[i]);
         const int my_tiles = (n_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x);
         const uint32_t total_it = static_cast<uint32_t>(my_tiles > 0 ? my_tiles : 0) * static_cast<uint32_t>(nkb);
         bool ok = true;
         for (uint32_t it = 0; it < total_it && ok; ++it) {
             const int s = it % kStages;
             const uint32_t ph = (it / kStages) & 1u;
-            const uint32_t w0 = ring0[0], w1 = ring1[0];
+            const uint32_t wcur = ring[0];
 #pragma unroll
-            for (int i = 0; i + 1 < kPrefetch; ++i) {
-                ring0[i] = ring0[i + 1];
-                ring1[i] = ring1[i + 1];
-            }
-            load_words(it + kPrefetch, ring0[kPrefetch - 1], ring1[kPrefetch - 1]);
+            for (int i = 0; i + 1 < kPrefetch; ++i) ring[i] = ring[i + 1];
+            load_next(ring[kPrefetch - 1]);
             if (!(ok = tc::mbar_wait(empty(s), ph ^ 1u, err))) break;
             const uint32_t a = a_tile(s);
-            const uint32_t n0 = ~w0, n1 = ~w1;
+            const uint32_t nw = ~wcur;
             if (MODE == kModeU) {
-                // row t of a K-major SW128 tile: 8 chunks of 16 B, chunk c holds K = 8c .. 8c+7
-                const uint32_t row_base = a + (t >> 3) * 1024u + (t & 7) * 128u;
+                // half (t & 1) of row t/2 of a K-major SW128 tile: chunks 4 (t & 1) .. +3
+                const int row = t >> 1, c0 = 4 * (t & 1);
+                const uint32_t row_base = a + (row >> 3) * 1024u + (row & 7) * 128u;
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint32_t nbyte = ((c < 4 ? n0 : n1) >> (8 * (c & 3))) & 0xFFu;
-                    sts128(row_base + ((c ^ (t & 7)) << 4), expand_nbyte_pm1(nbyte));
-                }
+                for (int c = 0; c < 4; ++c)
+                    sts128(row_base + (((c0 + c) ^ (row & 7)) << 4), expand_nbyte_pm1((nw >> (8 * c)) & 0xFFu));
             } else {
-                // K-row jl of an MN-major SW128 tile; this thread's 64 M-elements (k) are words
-                // 2h, 2h+1 of the tile's four, i.e. M-group h.  Lanes 0..7 of each 8-lane group
-                // take eight different K-rows (distinct swizzle phases, conflict-free stores).
-                const int jl = (t & 7) | ((t >> 4) << 3);
-                const int h = (t >> 3) & 1;
+                const int jl = (t & 7) | ((t >> 5) << 3), half = (t >> 3) & 1, h = (t >> 4) & 1;
                 const uint32_t atom = a + ((jl >> 3) * 2 + h) * 1024u + (jl & 7) * 128u;
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint32_t nbyte = ((c < 4 ? n0 : n1) >> (8 * (c & 3))) & 0xFFu;
-                    sts128(atom + ((c ^ (jl & 7)) << 4), expand_nbyte_pm1(nbyte));
-                }
+                for (int c = 0; c < 4; ++c)
+                    sts128(atom + (((4 * half + c) ^ (jl & 7)) << 4), expand_nbyte_pm1((nw >> (8 * c)) & 0xFFu));
             }
+            // each lane makes its own stores visible to the tensor core's (async) proxy; one
+            // arrive per warp after the warp has converged
             tc::fence_proxy_async_smem();
-            tc::mbar_arrive(full_a(s));
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(full_a(s));
         }
     } else {
         // ---------------------------------------------------------------- epilogue
@@ -294,7 +303,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 }
             }
             tc::tc_fence_before();
-            tc::mbar_arrive(acc_empty(acc));
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(acc_empty(acc));
         }
     }
 
