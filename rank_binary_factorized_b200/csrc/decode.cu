@@ -38,6 +38,11 @@ __device__ __forceinline__ void cp_async8(uint32_t dst, const void* src) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// Asks the memory system to bring [src, src + bytes) into L2 (no data returns to the SM);
+// src and bytes are multiples of 16.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 
 // The three balanced base-256 digits of a 23-bit signed integer v = a0 + 2^8 a1 + 2^16 a2,
 // each in [-128, 127], returned as s8 bytes.
@@ -61,18 +66,6 @@ __device__ __forceinline__ uint32_t digit_byte(int v, int q) {
     return static_cast<uint32_t>((v1 - d1) >> 8) & 255u;
 }
 
-
-// Sum of one 64-bit value per thread over the block; every thread gets the total.
-__device__ __forceinline__ long long block_sum_i64(long long v, long long* scratch /* [warps] */) {
-    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    __syncthreads();
-    if (lane == 0) scratch[warp] = v;
-    __syncthreads();
-    long long tot = 0;
-    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) tot += scratch[w];
-    return tot;
-}
 
 // ------------------------------------------------------------------ stage 1 (integer MMA)
 //
@@ -110,6 +103,8 @@ struct S1Params {
     int rows_per_slice;  // rows of V per block (multiple of 32)
     int jc_rows;         // rows staged per pass (multiple of 32)
     int zstage;          // z of the slice (M x rows_per_slice fp32) is kept in shared memory
+    const uint32_t* upf;  // U of the same layer: its first upf_bytes (a multiple of 16) are
+    int64_t upf_bytes;    // prefetched into L2 for stage 2, 1/grid of them per block
 };
 
 template <int NT>
@@ -148,7 +143,6 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const S1Params p) 
     __shared__ float s_mul[NQ_MATVEC_MAX_M];
     __shared__ unsigned long long s_zsum[NQ_MATVEC_MAX_M];
     __shared__ float s_wmax[kS1Threads / 32][NQ_MATVEC_MAX_M];
-    __shared__ long long s_red64[kS1Threads / 32];
 
     cg::cluster_group cluster = cg::this_cluster();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -194,6 +188,25 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const S1Params p) 
         }
     };
 
+    // stage 2's weights: start their way from HBM into L2 now, so that stage 2 reads them there
+    if (tid == 0 && p.upf_bytes > 0) {
+        const int G = gridDim.x * gridDim.y, b = blockIdx.y * gridDim.x + blockIdx.x;
+        const int64_t share = ((p.upf_bytes + G - 1) / G + 15) & ~static_cast<int64_t>(15);
+        const int64_t beg = static_cast<int64_t>(b) * share, end = min(beg + share, p.upf_bytes);
+        for (int64_t off = beg; off < end; off += 32768)
+            prefetch_l2_bulk(reinterpret_cast<const char*>(p.upf) + off,
+                             static_cast<uint32_t>(min(static_cast<int64_t>(32768), end - off)));
+    }
+    // s2 of the slice (a weight) is read before the wait, into registers when the slice has
+    // at most kS2Reg rows per thread
+    constexpr int kS2Reg = 8;
+    const bool s2reg = (j1 - j0) <= static_cast<int64_t>(kS2Reg) * kS1Threads;
+    float s2r[kS2Reg];
+#pragma unroll
+    for (int i = 0; i < kS2Reg; ++i) {
+        const int64_t j = j0 + tid + static_cast<int64_t>(i) * kS1Threads;
+        s2r[i] = (s2reg && j < j1) ? f16_bits_to_float(__ldg(p.s2 + j)) : 0.0f;
+    }
     build_aws(j0);  // weights only: may overlap the previous grid
     pdl_launch_dependents();
     pdl_wait();     // x may be written by the previous grid
@@ -203,19 +216,35 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const S1Params p) 
         for (int m = 0; m < p.M; ++m) {
             const uint16_t* xm = p.x + static_cast<int64_t>(m) * p.d_in;
             float v = 0.0f;
-#pragma unroll 8
-            for (int64_t j = j0 + tid; j < j1; j += kS1Threads) {
-                const float z = f16_bits_to_float(p.s2[j]) * bf16_bits_to_float(xm[j]);
-                if (p.zstage) {
-                    const int jl = static_cast<int>(j - j0);
-                    zs_s[m * zld + jl + (jl >> 5)] = z;
+            if (s2reg) {
+#pragma unroll
+                for (int i = 0; i < kS2Reg; ++i) {
+                    const int64_t j = j0 + tid + static_cast<int64_t>(i) * kS1Threads;
+                    if (j < j1) {
+                        const float z = s2r[i] * bf16_bits_to_float(xm[j]);
+                        if (p.zstage) {
+                            const int jl = static_cast<int>(j - j0);
+                            zs_s[m * zld + jl + (jl >> 5)] = z;
+                        }
+                        v = fmaxf(v, fabsf(z));
+                    }
                 }
-                v = fmaxf(v, fabsf(z));
+            } else {
+#pragma unroll 8
+                for (int64_t j = j0 + tid; j < j1; j += kS1Threads) {
+                    const float z = f16_bits_to_float(p.s2[j]) * bf16_bits_to_float(xm[j]);
+                    if (p.zstage) {
+                        const int jl = static_cast<int>(j - j0);
+                        zs_s[m * zld + jl + (jl >> 5)] = z;
+                    }
+                    v = fmaxf(v, fabsf(z));
+                }
             }
             for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
             if (lane == 0) s_wmax[warp][m] = v;
         }
         for (int e = tid; e < kS1Outs * NT * 8; e += kS1Threads) red[e] = 0;
+        if (tid < NQ_MATVEC_MAX_M) s_zsum[tid] = 0ull;
         __syncthreads();
         if (tid < p.M) {
             float v = 0.0f;
@@ -228,9 +257,11 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const S1Params p) 
         }
         __syncthreads();
     }
-    long long zsum[NQ_MATVEC_MAX_M];
+    // per-thread partial sums of the quantised z, per batch row (column group of the z table)
+    constexpr int MG = (NT * 8 + 2) / 3;
+    long long zacc[MG];
 #pragma unroll
-    for (int m = 0; m < NQ_MATVEC_MAX_M; ++m) zsum[m] = 0;
+    for (int m = 0; m < MG; ++m) zacc[m] = 0;
 
     // ---- passes over the slice: z table, then MMAs; integer accumulators live in registers
     // two accumulator sets, even and odd K steps, for two independent MMA chains per tile
@@ -254,9 +285,9 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const S1Params p) 
             build_aws(jb);
         }
         // z table: word zq[jq * SWZ + 3m + q] holds digit q of z_q(m, row jb + 4jq + i) in byte i;
-        // one thread builds the three digit words of one (jq, m) from four z values
+        // one thread builds the three digit words of one (jq, m) from four z values.  Every row
+        // of the pass lies in exactly one quad, so the quads' integers also give sum_j z_q(m, j).
         {
-            constexpr int MG = (NT * 8 + 2) / 3;
             const int64_t jend = min(j1, jb + p.jc_rows);
             for (int e = tid; e < nq_rows * MG; e += kS1Threads) {
                 const int m = e % MG, jq = e / MG;  // MG is a compile-time constant
@@ -275,32 +306,25 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const S1Params p) 
                                              : f16_bits_to_float(p.s2[j]) * bf16_bits_to_float(xm[j]);
                         }
                     }
+                    int qsum = 0;
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         uint32_t a0, a1, a2;
-                        digits3(__float2int_rn(zv[i] * mul), a0, a1, a2);
+                        const int qv = __float2int_rn(zv[i] * mul);
+                        qsum += qv;
+                        digits3(qv, a0, a1, a2);
                         d0 |= a0 << (8 * i);
                         d1 |= a1 << (8 * i);
                         d2 |= a2 << (8 * i);
                     }
+#pragma unroll
+                    for (int mm = 0; mm < MG; ++mm)
+                        if (mm == m) zacc[mm] += qsum;
                 }
                 uint32_t* dst = zq + jq * SWZ + 3 * m;
                 if (3 * m < NT * 8) dst[0] = d0;
                 if (3 * m + 1 < NT * 8) dst[1] = d1;
                 if (3 * m + 2 < NT * 8) dst[2] = d2;
-            }
-            for (int m = 0; m < p.M; ++m) {
-                const uint16_t* xm = p.x + static_cast<int64_t>(m) * p.d_in;
-                const float mul = s_mul[m];
-                long long zs = 0;
-#pragma unroll 4
-                for (int64_t j = jb + tid; j < jend; j += kS1Threads) {
-                    const int jl = static_cast<int>(j - j0);
-                    const float z = p.zstage ? zs_s[m * zld + jl + (jl >> 5)]
-                                             : f16_bits_to_float(p.s2[j]) * bf16_bits_to_float(xm[j]);
-                    zs += __float2int_rn(z * mul);
-                }
-                zsum[m] += zs;
             }
         }
         __syncthreads();
@@ -332,11 +356,15 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const S1Params p) 
         }
     }
 
-    for (int m = 0; m < p.M; ++m) {
-        const long long tot = block_sum_i64(zsum[m], s_red64);
-        if (tid == 0) s_zsum[m] = static_cast<unsigned long long>(tot);
+    // per-warp partial sums into s_zsum; read after the barriers of the reduction below
+#pragma unroll
+    for (int m = 0; m < MG; ++m) {
+        if (m < p.M) {
+            long long v = zacc[m];
+            for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+            if (lane == 0) atomicAdd(&s_zsum[m], static_cast<unsigned long long>(v));
+        }
     }
-    __syncthreads();
 
     // ---- exact per-output integers: row gid of M-tile (w, h) is k = 32w + 8(2h) + gid,
     // row gid+8 is k = 32w + 8(2h+1) + gid; both carry the weight 2^gid
@@ -414,26 +442,31 @@ struct S2Params {
     int tstage;          // t (M x r fp32) is copied into shared memory for the table build
 };
 
+// B table layout: the two B-fragment words of lane (gid, tig) for bit offset s, word group g
+// (8 words) and column tile nt sit next to each other, lanes in order, so one 64-bit load per
+// lane and MMA reads 256 contiguous bytes:
+//   word ((((s * ng + g) * NT + nt) * 32 + 4 * gid + tig) * 2 + half)
+// holds the digits of column 8 nt + gid for word 8 g + tig + 4 half.
 template <int NT>
-struct S2Layout {
-    static constexpr int SW = (NT == 1) ? 8 : 24;  // words per (s, w) entry row of the B table
-};
+__device__ __forceinline__ int s2_bidx(int s_, int w, int col, int ng) {
+    const int g = w >> 3, tg = w & 3, half = (w >> 2) & 1;
+    return ((((s_ * ng + g) * NT + (col >> 3)) * 32 + 4 * (col & 7) + tg) * 2 + half);
+}
 
 template <int NT, int TH>
 __global__ void __launch_bounds__(TH, 1) decode_stage2_kernel(const S2Params p) {
     constexpr int kS2Threads = TH;
     constexpr int kS2Warps = kS2Threads / 32;
     extern __shared__ __align__(16) uint32_t smem2[];
-    constexpr int SW = S2Layout<NT>::SW;
-    uint32_t* bt = smem2;                                  // [8][nwp][SW]
-    uint32_t* ublk = bt + 8 * p.nwp * SW;                  // [chunk_mt*16][su]
+    uint32_t* bt = smem2;                                  // 8 * nwp * NT*8 words (s2_bidx)
+    uint32_t* ublk = bt + 8 * p.nwp * NT * 8;              // [chunk_mt*16][su]
     int* red = reinterpret_cast<int*>(ublk + p.chunk_mt * 16 * p.su);  // [chunk_mt*16][NT*8]
-    float* ts_s = reinterpret_cast<float*>(red + p.chunk_mt * 16 * NT * 8);  // [M][r] when p.tstage
+    float* s1_s = reinterpret_cast<float*>(red + p.chunk_mt * 16 * NT * 8);  // [chunk_mt*16]
+    float* ts_s = s1_s + p.chunk_mt * 16;                                   // [M][r] when p.tstage
     __shared__ int s_shift[NQ_MATVEC_MAX_M];
     __shared__ float s_mul[NQ_MATVEC_MAX_M];
     __shared__ unsigned long long s_tsum[NQ_MATVEC_MAX_M];
     __shared__ float s_wmax[kS2Warps][NQ_MATVEC_MAX_M];
-    __shared__ long long s_red64[kS2Warps];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int G = gridDim.x;
@@ -447,24 +480,30 @@ __global__ void __launch_bounds__(TH, 1) decode_stage2_kernel(const S2Params p) 
         const int64_t row1 = min(static_cast<int64_t>(b) * 16, p.d_out);
         const int rows = static_cast<int>(row1 - row0);
         const bool even = ((p.ldu & 1) == 0) && ((p.nw & 1) == 0);
-        if (even) {
-            const int per_row = p.nw / 2;
-            for (int e = tid; e < rows * per_row; e += kS2Threads) {
-                const int rr = e / per_row, c = e - rr * per_row;
-                cp_async8(static_cast<uint32_t>(__cvta_generic_to_shared(ublk + rr * p.su + 2 * c)),
-                          p.U + (row0 + rr) * p.ldu + 2 * c);
-            }
-        } else {
-            for (int e = tid; e < rows * p.nw; e += kS2Threads) {
-                const int rr = e / p.nw, c = e - rr * p.nw;
-                cp_async4(static_cast<uint32_t>(__cvta_generic_to_shared(ublk + rr * p.su + c)),
-                          p.U + (row0 + rr) * p.ldu + c);
+        // one warp per row, lanes along the row
+        for (int rr = warp; rr < rows; rr += kS2Warps) {
+            const uint32_t* src = p.U + (row0 + rr) * p.ldu;
+            const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(ublk + rr * p.su));
+            if (even) {
+                for (int c = lane; c < p.nw / 2; c += 32) cp_async8(dst + 8u * c, src + 2 * c);
+            } else {
+                for (int c = lane; c < p.nw; c += 32) cp_async4(dst + 4u * c, src + c);
             }
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
 
-    if (mt0 < mt1) load_u(mt0, min(mt1, mt0 + p.chunk_mt));
+    // s1 of the same rows (a weight), as fp32, for the epilogue
+    auto load_s1 = [&](int a, int b) {
+        const int64_t row0 = static_cast<int64_t>(a) * 16;
+        const int rows = static_cast<int>(min(static_cast<int64_t>(b) * 16, p.d_out) - row0);
+        for (int i = tid; i < rows; i += kS2Threads) s1_s[i] = f16_bits_to_float(__ldg(p.s1 + row0 + i));
+    };
+
+    if (mt0 < mt1) {
+        load_u(mt0, min(mt1, mt0 + p.chunk_mt));
+        load_s1(mt0, min(mt1, mt0 + p.chunk_mt));
+    }
     pdl_launch_dependents();
     pdl_wait();  // t comes from stage 1 of this call
 
@@ -482,6 +521,7 @@ __global__ void __launch_bounds__(TH, 1) decode_stage2_kernel(const S2Params p) 
             for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
             if (lane == 0) s_wmax[warp][m] = v;
         }
+        if (tid < NQ_MATVEC_MAX_M) s_tsum[tid] = 0ull;
         __syncthreads();
         if (tid < p.M) {
             float v = 0.0f;
@@ -499,12 +539,16 @@ __global__ void __launch_bounds__(TH, 1) decode_stage2_kernel(const S2Params p) 
         auto t_at = [&](int m, int k) -> float {
             return p.tstage ? ts_s[m * tld + k + (k >> 5)] : p.t[static_cast<int64_t>(m) * p.r + k];
         };
-        // B table: word bt[(s * nwp + w) * SW + 3m + q] holds digit q of t_q(m, 32w + s + 8b) in
-        // byte b; one thread builds the digit words of one (s, w) for every batch row
+        // B table: the word for (s, w, column 3m + q) holds digit q of t_q(m, 32w + s + 8b) in
+        // byte b; one thread builds the digit words of one (s, w) for every batch row.  Every k
+        // < r lies in exactly one entry, so the entries' integers also give sum_k t_q(m, k).
+        const int ngp = p.nwp / 8;
         constexpr int MG = (NT * 8 + 2) / 3;  // column groups of three
+        long long tacc[MG];
+#pragma unroll
+        for (int m = 0; m < MG; ++m) tacc[m] = 0;
         for (int sw = tid; sw < 8 * p.nwp; sw += kS2Threads) {
             const int s_ = sw / p.nwp, w = sw - s_ * p.nwp;
-            uint32_t* row = bt + sw * SW;
 #pragma unroll
             for (int m = 0; m < MG; ++m) {
                 uint32_t d0 = 0u, d1 = 0u, d2 = 0u;
@@ -513,29 +557,34 @@ __global__ void __launch_bounds__(TH, 1) decode_stage2_kernel(const S2Params p) 
                     float tv[4];
 #pragma unroll
                     for (int b = 0; b < 4; ++b) tv[b] = t_at(m, 32 * w + s_ + 8 * b);
+                    int qsum = 0;
 #pragma unroll
                     for (int b = 0; b < 4; ++b) {
                         uint32_t a0, a1, a2;
-                        digits3(__float2int_rn(tv[b] * mul), a0, a1, a2);
+                        const int qv = __float2int_rn(tv[b] * mul);
+                        qsum += qv;
+                        digits3(qv, a0, a1, a2);
                         d0 |= a0 << (8 * b);
                         d1 |= a1 << (8 * b);
                         d2 |= a2 << (8 * b);
                     }
+                    tacc[m] += qsum;
                 }
-                if (3 * m < NT * 8) row[3 * m] = d0;
-                if (3 * m + 1 < NT * 8) row[3 * m + 1] = d1;
-                if (3 * m + 2 < NT * 8) row[3 * m + 2] = d2;
+                if (3 * m < NT * 8) bt[s2_bidx<NT>(s_, w, 3 * m, ngp)] = d0;
+                if (3 * m + 1 < NT * 8) bt[s2_bidx<NT>(s_, w, 3 * m + 1, ngp)] = d1;
+                if (3 * m + 2 < NT * 8) bt[s2_bidx<NT>(s_, w, 3 * m + 2, ngp)] = d2;
             }
         }
-        for (int m = 0; m < p.M; ++m) {
-            const float mul = s_mul[m];
-            long long ts = 0;
-#pragma unroll 4
-            for (int k = tid; k < p.r; k += kS2Threads) ts += __float2int_rn(t_at(m, k) * mul);
-            ts = block_sum_i64(ts, s_red64);
-            if (tid == 0) s_tsum[m] = static_cast<unsigned long long>(ts);
+        // per-warp partial sums into s_tsum; read by the epilogue, after the barriers below
+#pragma unroll
+        for (int m = 0; m < MG; ++m) {
+            if (m < p.M) {
+                long long v = tacc[m];
+                for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+                if (lane == 0) atomicAdd(&s_tsum[m], static_cast<unsigned long long>(v));
+            }
         }
-        __syncthreads();
+        // (the barrier before the MMAs publishes the table)
     }
 
     const int gid = lane >> 2, tig = lane & 3;
@@ -578,10 +627,12 @@ __global__ void __launch_bounds__(TH, 1) decode_stage2_kernel(const S2Params p) 
                 for (int s_ = 0; s_ < 8; ++s_) {
                     const uint32_t msk = 0x01010101u << s_;
                     const uint32_t a0 = w00 & msk, a1 = w10 & msk, a2 = w01 & msk, a3 = w11 & msk;
-                    const uint32_t* b = bt + (s_ * p.nwp + wb) * SW;
+                    const uint2* b = reinterpret_cast<const uint2*>(bt) + ((s_ * ng + g) * NT) * 32 + lane;
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt)
-                        mma_u8s8(acc[s_][nt], a0, a1, a2, a3, b[tig * SW + nt * 8 + gid], b[(4 + tig) * SW + nt * 8 + gid]);
+                    for (int nt = 0; nt < NT; ++nt) {
+                        const uint2 bb = b[nt * 32];
+                        mma_u8s8(acc[s_][nt], a0, a1, a2, a3, bb.x, bb.y);
+                    }
                 }
                 w00 = n00; w01 = n01; w10 = n10; w11 = n11;
             }
@@ -609,12 +660,15 @@ __global__ void __launch_bounds__(TH, 1) decode_stage2_kernel(const S2Params p) 
                 const long long P = static_cast<long long>(rr[0]) + (static_cast<long long>(rr[1]) << 8) +
                                     (static_cast<long long>(rr[2]) << 16);
                 const long long val = 2 * P - static_cast<long long>(s_tsum[m]);
-                const double yv = static_cast<double>(f16_bits_to_float(p.s1[i])) * ldexp(static_cast<double>(val), -s_shift[m]);
+                const double yv = static_cast<double>(s1_s[row]) * ldexp(static_cast<double>(val), -s_shift[m]);
                 p.y[static_cast<int64_t>(m) * p.d_out + i] = __bfloat16_as_ushort(__double2bfloat16(yv));
             }
         }
         __syncthreads();
-        if (c1 < mt1) load_u(c1, min(mt1, c1 + p.chunk_mt));
+        if (c1 < mt1) {
+            load_u(c1, min(mt1, c1 + p.chunk_mt));
+            load_s1(c1, min(mt1, c1 + p.chunk_mt));
+        }
     }
     cp_async_wait_all();
 }
@@ -694,6 +748,9 @@ nq_status launch_decode_nt(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y
         q.rows_per_slice = sp.rows_per_slice;
         q.jc_rows = sp.jc_rows;
         q.zstage = sp.zstage;
+        q.upf = L->U;
+        // U up to the last valid word of its last row, rounded down to 16 bytes
+        q.upf_bytes = (((L->d_out - 1) * L->ldu + L->r / 32) * 4) & ~static_cast<int64_t>(15);
         void* args[] = {&q};
         const bool wide = (NT <= 2) && sp.rows_per_slice >= 1024;
         const void* fn = wide ? reinterpret_cast<const void*>(nq::decode_stage1_kernel<NT, (NT <= 2 ? 512 : 256)>)
@@ -721,8 +778,8 @@ nq_status launch_decode_nt(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y
         int grid = nq_host::sm_count();
         if (grid > q.mt_total) grid = q.mt_total;
         const int per_cta = (q.mt_total + grid - 1) / grid;
-        const size_t bt_bytes = static_cast<size_t>(8) * q.nwp * nq::S2Layout<NT>::SW * 4;
-        const size_t per_mt = static_cast<size_t>(16) * q.su * 4 + static_cast<size_t>(16) * NT * 8 * 4;
+        const size_t bt_bytes = static_cast<size_t>(8) * q.nwp * NT * 8 * 4;
+        const size_t per_mt = static_cast<size_t>(16) * q.su * 4 + static_cast<size_t>(16) * NT * 8 * 4 + 16 * 4;
         int chunk = per_cta;
         if (bt_bytes + chunk * per_mt > kStage2SmemBudget) chunk = static_cast<int>((kStage2SmemBudget - bt_bytes) / per_mt);
         if (chunk < 1) return NQ_ERR_SHAPE;
@@ -755,9 +812,9 @@ size_t nq_decode_workspace_bytes(int64_t d_in, int64_t r, int64_t M) {
 size_t nq_decode_stage2_smem(int64_t r, int64_t M) {
     const int64_t nt = ntiles_for(M);
     const int64_t nwp = (r / 32 + 7) / 8 * 8;
-    const int64_t sw = nt == 1 ? 8 : 24;
+    const int64_t sw = nt * 8;  // B-table columns
     const int64_t su = nwp + ((4 - nwp % 32) + 32) % 32;
-    const size_t need = static_cast<size_t>(8 * nwp * sw * 4 + 16 * su * 4 + 16 * nt * 8 * 4);
+    const size_t need = static_cast<size_t>(8 * nwp * sw * 4 + 16 * su * 4 + 16 * nt * 8 * 4 + 16 * 4);
     return need <= kStage2SmemBudget ? need : kStage2SmemBudget + 1;
 }
 

@@ -11,7 +11,7 @@
 //
 // Both products run in one persistent warp-specialised kernel, D[w][n] = sum_K A[w][K] B[n][K]:
 //   * A (the weights, MMA M = 128 rows of U, or of V^T) is expanded on chip from the packed
-//     words to fp16 +-1 by four producer warps that write the UMMA 128-byte-swizzled
+//     words to fp16 +-1 by eight producer warps that write the UMMA 128-byte-swizzled
 //     layout straight into shared memory (K-major for U, whose bits run along K = r;
 //     MN-major for V^T, whose bits run along M = r);
 //   * B (the activations Z or T, MMA N = up to 256 tokens) arrives by TMA tile loads;
@@ -189,11 +189,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         //  V (MN-major): K-row jl, M-group h, word `half` of that group; lanes 0..7 of every
         //  8-lane group take eight different K-rows so their 16-byte stores hit distinct banks
         const int t = threadIdx.x - 64;  // 0..255
-        // The two packed words of iteration `j` (tile, k block) of this CTA.  Loads run
-        // kPrefetch iterations ahead of their use in a register ring, so the L2/DRAM latency
-        // of the words overlaps the expansion and the waits of the iterations before.
-        // Per-thread constants of the word this thread expands, and a cursor (tile, k block)
-        // for the prefetch that runs kPrefetch iterations ahead; advanced by increments only.
+        // Each thread's packed word is loaded kPrefetch iterations ahead of its use into a
+        // register ring, so the L2/DRAM latency of the words overlaps the expansion and the
+        // waits of the iterations before.  The load address comes from per-thread constants
+        // and a (tile, k block) cursor that only ever increments (no integer division).
         int64_t row_off;  // row index within a tile (U) or within a k block (V)
         int word_off;     // word offset within the k block (U) or within the tile's 4 words (V)
         if (MODE == kModeU) {
