@@ -8,14 +8,14 @@
 //   stage 1:  t[m][k] = sum_j V_jk * (s2_j * x[m][j])          (reduction over d_in)
 //   stage 2:  y[m][i] = bf16( s1_i * sum_k U_ik * t[m][k] )      (reduction over r)
 //
-// Stage 1 is a split-d_in reduction: block (c, s) owns word chunk c (WC words = WC*32
-// columns of t) and row slice s of V.  Threads own (word, bit group, row subset) and keep
-// fp32 accumulators; the block folds its row subsets through shared memory, writes one
-// partial per slice, and the last block of each chunk to finish (an atomic ticket) sums the
-// partials in slice order.  No atomics touch the values, so t is run-to-run identical.
-//
-// Stage 2 stages t in shared memory transposed so that lanes reading consecutive words hit
-// consecutive banks; each warp sweeps one row of U with 128-byte coalesced loads.
+// Both stages run on the integer tensor path (mma.sync m16n8k32, u8 x s8 -> s32): the
+// packed bits, masked per bit offset, are the A operand as they are; the activations,
+// quantised to 23-bit fixed point and split into three base-256 digits, are the B operand.
+// Stage 1 is a split-d_in reduction over thread-block clusters (one cluster per chunk of 256
+// outputs, one block per row slice of V) that sum their exact partials in distributed
+// shared memory; stage 2 gives every block a run of 16-row tiles of U with t's digit table in
+// shared memory.  The two kernels chain by programmatic dependent launch: each reads its
+// weights before it waits for the previous grid.
 #include <cooperative_groups.h>
 
 #include "nq_common.cuh"

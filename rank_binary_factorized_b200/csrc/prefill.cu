@@ -22,18 +22,27 @@
 // error word, drains its own copies and MMAs, frees TMEM and returns.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+#include <cstring>
+
 #include "tc_common.cuh"
 
 namespace nq {
 
 constexpr int kTileW = 128;       // MMA M: weight rows per tile
 constexpr int kTileK = 64;        // K per pipeline stage (one 128-byte swizzle row of fp16)
-constexpr int kStages = 4;
+constexpr int kMaxStages = 12;   // pipeline depth: as many stages as fit (fewer for wide tiles)
 constexpr int kTmemCols = 512;
 constexpr int kExpandWarps = 8;     // warps 2..9 expand the packed weights
+constexpr int kExpandGroups = 2;    // in groups that fill alternate stages
+constexpr int kGroupWarps = kExpandWarps / kExpandGroups;
+static_assert(2 * 32 * kGroupWarps == 256, "a stage is 256 packed words, two per producer thread");
 constexpr int kEpiWarp0 = 2 + kExpandWarps;  // warps 10..13: epilogue
 constexpr int kPrefillThreads = 32 * (kEpiWarp0 + 4);
 constexpr int kABytes = kTileW * kTileK * 2;  // 16 KB
+// Packed-sign box a stage receives by TMA (4 words x 128 rows of U, or 4 words x 64 rows of V)
+constexpr int kBitsWords = 4;
+constexpr int kBitsBytes = kBitsWords * 4 * kTileW;  // slot size (2 KB)
 
 enum PrefillMode : int { kModeV = 0, kModeU = 1 };
 
@@ -45,23 +54,25 @@ struct PrefillArgs {
     int64_t nwords;        // valid words per row of `bits` (r / 32)
     int64_t M;             // tokens
     int tile_n;            // tokens per tile (multiple of 16, <= 256)
+    int stages;            // pipeline stages in shared memory (2 .. kMaxStages)
     int n_tiles_w, n_tiles_n, n_kblocks;
     void* out;             // mode V: T fp16 [M][ldo]; mode U: Y bf16 [M][ldo]
     int64_t ldo;
     const uint16_t* s1;    // mode U
     unsigned int* err;
+    int bits_tma;          // packed signs arrive by TMA (row stride a multiple of 16 bytes)
 };
 
 // fp16 +1 = 0x3C00, -1 = 0xBC00; two elements per 32-bit word, element 2i in the low half.
-// Expands the 8 bits of `byte` (element e = bit e) into 8 fp16 values (16 bytes).
-// `nbyte` holds the complemented bits (1 = negative) in its low 8 bits and zeros above.
-// For pair q, (nbyte >> 2q) * 0x40008000 puts bit 2q at bit 15 and bit 2q+1 at bit 31: the
-// product's two shifted copies occupy bits 15..22 and 30..31 (higher bits fall off), so they
-// never overlap and no carry disturbs the two sign positions.
-__device__ __forceinline__ uint4 expand_nbyte_pm1(uint32_t nbyte) {
+// Expands the 8 bits of `byte` (element e = bit e, 1 = +1) into 8 fp16 values (16 bytes).
+// For pair q, byte * (2^(15 - 2q) + 2^(30 - 2q)) puts bit 2q at bit 15 and bit 2q+1 at bit 31;
+// the product's two shifted copies of the byte (bits 15-2q .. 22-2q and 30-2q .. 37-2q)
+// never overlap, so no carry disturbs the two sign positions.  Masked, they are the signs of
+// the two elements with 1 = +1; XOR with the pattern of (-1, -1) flips them into fp16 signs.
+__device__ __forceinline__ uint4 expand_byte_pm1(uint32_t byte) {
     uint32_t r[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) r[q] = 0x3C003C00u | (((nbyte >> (2 * q)) * 0x40008000u) & 0x80008000u);
+    for (int q = 0; q < 4; ++q) r[q] = ((byte * (0x40008000u >> (2 * q))) & 0x80008000u) ^ 0xBC00BC00u;
     return make_uint4(r[0], r[1], r[2], r[3]);
 }
 
@@ -72,31 +83,38 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
 
 template <int MODE>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
-    lrb_umma_kernel(const __grid_constant__ CUtensorMap tmap_b, const PrefillArgs args) {
+    lrb_umma_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant__ CUtensorMap tmap_bits,
+                    const PrefillArgs args) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base (the 128-byte swizzle pattern is a function of address bits 4-9)
     const uint32_t smem_base = (tc::smem_u32(smem_raw) + 1023u) & ~1023u;
     const int tile_n = args.tile_n;
     const uint32_t b_bytes = static_cast<uint32_t>(tile_n) * kTileK * 2;
-    const uint32_t stage_bytes = kABytes + ((b_bytes + 1023u) & ~1023u);
-    const uint32_t bar_base = smem_base + kStages * stage_bytes;
+    const uint32_t stage_bytes = kABytes + ((b_bytes + 1023u) & ~1023u) + kBitsBytes;
+    const int stages = args.stages;
+    const uint32_t bar_base = smem_base + stages * stage_bytes;
     // barriers: full_a[S], full_b[S], empty[S], acc_full[2], acc_empty[2], drain
     auto full_a = [&](int s) { return bar_base + 8u * s; };
-    auto full_b = [&](int s) { return bar_base + 8u * (kStages + s); };
-    auto empty = [&](int s) { return bar_base + 8u * (2 * kStages + s); };
-    auto acc_full = [&](int a) { return bar_base + 8u * (3 * kStages + a); };
-    auto acc_empty = [&](int a) { return bar_base + 8u * (3 * kStages + 2 + a); };
-    const uint32_t drain_bar = bar_base + 8u * (3 * kStages + 4);
-    const uint32_t tmem_slot = bar_base + 8u * (3 * kStages + 5);
+    auto full_b = [&](int s) { return bar_base + 8u * (kMaxStages + s); };
+    auto empty = [&](int s) { return bar_base + 8u * (2 * kMaxStages + s); };
+    auto acc_full = [&](int a) { return bar_base + 8u * (3 * kMaxStages + a); };
+    auto acc_empty = [&](int a) { return bar_base + 8u * (3 * kMaxStages + 2 + a); };
+    const uint32_t drain_bar = bar_base + 8u * (3 * kMaxStages + 4);
+    const uint32_t tmem_slot = bar_base + 8u * (3 * kMaxStages + 5);
     auto a_tile = [&](int s) { return smem_base + s * stage_bytes; };
     auto b_tile = [&](int s) { return smem_base + s * stage_bytes + kABytes; };
+    auto bits_tile = [&](int s) { return smem_base + (s + 1) * stage_bytes - kBitsBytes; };
+    // bytes of packed signs per stage and their box origin for k block kb of weight tile tw
+    const uint32_t bits_bytes = (MODE == kModeU) ? kBitsWords * 4 * kTileW : kBitsWords * 4 * kTileK;
+    auto bits_x = [&](int tw, int kb) { return (MODE == kModeU) ? (kb >> 1) * kBitsWords : tw * kBitsWords; };
+    auto bits_y = [&](int tw, int kb) { return (MODE == kModeU) ? tw * kTileW : kb * kTileK; };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            tc::mbar_init(full_a(s), kExpandWarps);
+        for (int s = 0; s < stages; ++s) {
+            tc::mbar_init(full_a(s), kGroupWarps);
             tc::mbar_init(full_b(s), 1);
             tc::mbar_init(empty(s), 1);
         }
@@ -107,6 +125,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         tc::mbar_init(drain_bar, 1);
         tc::mbar_fence_init();
         tc::tma_prefetch_desc(&tmap_b);
+        if (args.bits_tma) tc::tma_prefetch_desc(&tmap_bits);
     }
     if (warp == 1) {
         tc::tmem_alloc(tmem_slot, kTmemCols);
@@ -124,29 +143,54 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA producer (B)
         if (lane == 0) {
+            // the packed signs of the first `stages` k blocks are weights: load them before
+            // waiting for the activations (the stage's barrier also waits for its B tile)
+            uint32_t pre = 0;
+            if (args.bits_tma) {
+                int tile = blockIdx.x, kb = 0;
+                while (tile < n_tiles && pre < static_cast<uint32_t>(stages)) {
+                    const int tw = tile % args.n_tiles_w;
+                    tc::mbar_expect_tx(full_b(pre), bits_bytes);
+                    tc::tma_load_2d(bits_tile(pre), &tmap_bits, bits_x(tw, kb), bits_y(tw, kb), full_b(pre));
+                    ++pre;
+                    if (++kb == nkb) {
+                        kb = 0;
+                        tile += gridDim.x;
+                    }
+                }
+            }
             pdl_wait();  // activations are written by the grid queued before this one
-            uint32_t it = 0;
+            uint32_t it = 0, ph = 0;
+            int s = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
                 const int tn = tile / args.n_tiles_w;
+                const int tw = tile - tn * args.n_tiles_w;
                 for (int kb = 0; kb < nkb; ++kb, ++it) {
-                    const int s = it % kStages;
-                    const uint32_t ph = (it / kStages) & 1u;
                     if (!(ok = tc::mbar_wait(empty(s), ph ^ 1u, err))) break;
+                    if (args.bits_tma && it >= pre) {
+                        tc::mbar_expect_tx(full_b(s), bits_bytes);
+                        tc::tma_load_2d(bits_tile(s), &tmap_bits, bits_x(tw, kb), bits_y(tw, kb), full_b(s));
+                    }
                     tc::mbar_arrive_expect_tx(full_b(s), b_bytes);
                     tc::tma_load_2d(b_tile(s), &tmap_b, kb * kTileK, tn * tile_n, full_b(s));
+                    if (++s == stages) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
             }
             // drain: every load issued has landed before the CTA may exit
-            const uint32_t first = it > static_cast<uint32_t>(kStages) ? it - kStages : 0u;
-            for (uint32_t j = first; j < it; ++j) tc::mbar_wait(full_b(j % kStages), (j / kStages) & 1u, err);
+            const uint32_t first = it > static_cast<uint32_t>(stages) ? it - stages : 0u;
+            for (uint32_t j = first; j < it; ++j) tc::mbar_wait(full_b(j % stages), (j / stages) & 1u, err);
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer
         if (lane == 0) {
             constexpr bool a_mn = (MODE == kModeV);
             const uint32_t idesc = tc::idesc_f16_f32(kTileW, tile_n, a_mn, false);
-            uint32_t it = 0, tc_count = 0;
+            uint32_t tc_count = 0, ph = 0;
+            int s = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++tc_count) {
                 const int acc = tc_count & 1;
@@ -154,9 +198,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 if (!(ok = tc::mbar_wait(acc_empty(acc), aph ^ 1u, err))) break;
                 tc::tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * 256);
-                for (int kb = 0; kb < nkb; ++kb, ++it) {
-                    const int s = it % kStages;
-                    const uint32_t ph = (it / kStages) & 1u;
+                for (int kb = 0; kb < nkb; ++kb) {
                     if (!(ok = tc::mbar_wait(full_a(s), ph, err))) break;
                     if (!(ok = tc::mbar_wait(full_b(s), ph, err))) break;
                     tc::tc_fence_after();
@@ -174,6 +216,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                         tc::mma_f16_ss(d_tmem, adesc, bdesc, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
                     }
                     tc::mma_commit(empty(s));
+                    if (++s == stages) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
                 if (!ok) break;
                 tc::mma_commit(acc_full(acc));
@@ -184,84 +230,120 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
     } else if (warp < kEpiWarp0) {
         // ---------------------------------------------------------------- A expansion (weights)
-        // 256 threads, one packed word (32 weights) per thread per k block:
-        //  U (K-major): row = t / 2, word 2 kb + (t & 1) -> chunks 4 (t & 1) .. +3 of the row
-        //  V (MN-major): K-row jl, M-group h, word `half` of that group; lanes 0..7 of every
-        //  8-lane group take eight different K-rows so their 16-byte stores hit distinct banks
-        const int t = threadIdx.x - 64;  // 0..255
-        // Each thread's packed word is loaded kPrefetch iterations ahead of its use into a
-        // register ring, so the L2/DRAM latency of the words overlaps the expansion and the
-        // waits of the iterations before.  The load address comes from per-thread constants
-        // and a (tile, k block) cursor that only ever increments (no integer division).
-        int64_t row_off;  // row index within a tile (U) or within a k block (V)
-        int word_off;     // word offset within the k block (U) or within the tile's 4 words (V)
-        if (MODE == kModeU) {
-            row_off = t >> 1;
-            word_off = t & 1;
-        } else {
-            row_off = (t & 7) | ((t >> 5) << 3);
-            word_off = ((t >> 4) & 1) * 2 + ((t >> 3) & 1);
-        }
+        // kExpandGroups groups of warps take alternate k blocks, so that as many stages are
+        // filled at once (a stage's stores, proxy fence and arrival are a latency chain).  A
+        // stage holds 256 packed words; thread tg of a group owns two adjacent ones:
+        //  U (K-major): row tg of the tile, words 2 kb and 2 kb + 1: the row's 64 K values, all
+        //  eight 16-byte chunks of its 128-byte swizzled row
+        //  V (MN-major): K-row jl = (tg & 7) | ((tg >> 4) << 3) of the k block, M-group
+        //  h = (tg >> 3) & 1, words 2h and 2h + 1 of the tile's four (128 M values)
+        // Lanes 0..7 of every 8-lane group take eight different rows, so their 16-byte stores
+        // fall in eight different bank groups.
+        const int grp = (warp - 2) / kGroupWarps;
+        const int tg = threadIdx.x - 64 - grp * 32 * kGroupWarps;  // 0..127
+        const int jl = (tg & 7) | ((tg >> 4) << 3), hgrp = (tg >> 3) & 1;
+        const bool ld_even = (args.ld & 1) == 0;  // 8-byte loads of a word pair are aligned
+        // The pair is loaded kPrefetch of the group's iterations ahead of its use into a
+        // register ring, so the L2/DRAM latency overlaps the expansion and the waits of the
+        // iterations before.  The (tile, k block) cursor only ever increments.
         int pf_tile = blockIdx.x, pf_kb = 0, pf_tw = blockIdx.x % args.n_tiles_w;
-        auto load_next = [&](uint32_t& w) {
-            w = 0u;
+        auto advance = [&]() {
+            if (++pf_kb == nkb) {
+                pf_kb = 0;
+                pf_tile += gridDim.x;
+                pf_tw += gridDim.x;
+                while (pf_tw >= args.n_tiles_w) pf_tw -= args.n_tiles_w;
+            }
+        };
+        for (int i = 0; i < grp; ++i) advance();
+        auto load_next = [&](uint2& w) {
+            w = make_uint2(0u, 0u);
             if (pf_tile < n_tiles) {
                 int64_t row, wcol;
                 bool row_ok;
                 if (MODE == kModeU) {
-                    row = static_cast<int64_t>(pf_tw) * kTileW + row_off;
-                    wcol = static_cast<int64_t>(pf_kb) * 2 + word_off;
+                    row = static_cast<int64_t>(pf_tw) * kTileW + tg;
+                    wcol = 2 * static_cast<int64_t>(pf_kb);
                     row_ok = row < args.rows_w;
                 } else {
-                    row = static_cast<int64_t>(pf_kb) * kTileK + row_off;
-                    wcol = static_cast<int64_t>(pf_tw) * (kTileW / 32) + word_off;
+                    row = static_cast<int64_t>(pf_kb) * kTileK + jl;
+                    wcol = static_cast<int64_t>(pf_tw) * (kTileW / 32) + 2 * hgrp;
                     row_ok = row < args.K;
                 }
-                if (row_ok && wcol < args.nwords) w = __ldg(args.bits + row * args.ld + wcol);
-                if (++pf_kb == nkb) {
-                    pf_kb = 0;
-                    pf_tile += gridDim.x;
-                    pf_tw += gridDim.x;
-                    while (pf_tw >= args.n_tiles_w) pf_tw -= args.n_tiles_w;
+                const uint32_t* src = args.bits + row * args.ld + wcol;
+                if (row_ok) {
+                    if (wcol + 1 < args.nwords) {
+                        if (ld_even) {
+                            w = __ldg(reinterpret_cast<const uint2*>(src));
+                        } else {
+                            w.x = __ldg(src);
+                            w.y = __ldg(src + 1);
+                        }
+                    } else if (wcol < args.nwords) {
+                        w.x = __ldg(src);
+                    }
                 }
             }
+            for (int g = 0; g < kExpandGroups && pf_tile < n_tiles; ++g) advance();
         };
-        constexpr int kPrefetch = 4;
-        uint32_t ring[kPrefetch];
-#pragma unroll
-        for (int i = 0; i < kPrefetch; ++i) load_next(ring[i]);
+        constexpr int kPrefetch = 8;
+        uint2 ring[kPrefetch];
         const int my_tiles = (n_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x);
         const uint32_t total_it = static_cast<uint32_t>(my_tiles > 0 ? my_tiles : 0) * static_cast<uint32_t>(nkb);
-        bool ok = true;
-        for (uint32_t it = 0; it < total_it && ok; ++it) {
-            const int s = it % kStages;
-            const uint32_t ph = (it / kStages) & 1u;
-            const uint32_t wcur = ring[0];
+        // this thread's 128-byte smem row within a stage's A tile, and its swizzle
+        const uint32_t row_off_b = (MODE == kModeU) ? (tg >> 3) * 1024u + (tg & 7) * 128u
+                                                    : ((jl >> 3) * 2 + hgrp) * 1024u + (jl & 7) * 128u;
+        const int swz = (MODE == kModeU) ? (tg & 7) : (jl & 7);
+        // expands this thread's word pair into its 128-byte row of stage s's A tile and
+        // publishes it to the tensor core's (async) proxy
+        auto expand_store = [&](uint2 wcur, int s) {
+            const uint32_t row_addr = a_tile(s) + row_off_b;
 #pragma unroll
-            for (int i = 0; i + 1 < kPrefetch; ++i) ring[i] = ring[i + 1];
-            load_next(ring[kPrefetch - 1]);
-            if (!(ok = tc::mbar_wait(empty(s), ph ^ 1u, err))) break;
-            const uint32_t a = a_tile(s);
-            const uint32_t nw = ~wcur;
-            if (MODE == kModeU) {
-                // half (t & 1) of row t/2 of a K-major SW128 tile: chunks 4 (t & 1) .. +3
-                const int row = t >> 1, c0 = 4 * (t & 1);
-                const uint32_t row_base = a + (row >> 3) * 1024u + (row & 7) * 128u;
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    sts128(row_base + (((c0 + c) ^ (row & 7)) << 4), expand_nbyte_pm1((nw >> (8 * c)) & 0xFFu));
-            } else {
-                const int jl = (t & 7) | ((t >> 5) << 3), half = (t >> 3) & 1, h = (t >> 4) & 1;
-                const uint32_t atom = a + ((jl >> 3) * 2 + h) * 1024u + (jl & 7) * 128u;
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    sts128(atom + (((4 * half + c) ^ (jl & 7)) << 4), expand_nbyte_pm1((nw >> (8 * c)) & 0xFFu));
+            for (int c = 0; c < 8; ++c) {
+                const uint32_t byte = ((c < 4 ? wcur.x : wcur.y) >> (8 * (c & 3))) & 0xFFu;
+                sts128(row_addr + ((c ^ swz) << 4), expand_byte_pm1(byte));
             }
-            // each lane makes its own stores visible to the tensor core's (async) proxy; one
-            // arrive per warp after the warp has converged
             tc::fence_proxy_async_smem();
-            __syncwarp();
+            __syncwarp();  // one arrive per warp after the warp has converged
             if (lane == 0) tc::mbar_arrive(full_a(s));
+        };
+        bool ok = true;
+        int s = grp;  // stage and phase of iteration `it` (grp < 2 <= stages)
+        uint32_t ph = 0;
+        if (args.bits_tma) {
+            // the stage's packed signs land with its B tile: wait for the stage, read them
+            // from shared memory (rows of 16 bytes: 4 words)
+            int cur_kb = grp % nkb;
+            for (uint32_t it = grp; it < total_it && ok; it += kExpandGroups) {
+                if (!(ok = tc::mbar_wait(full_b(s), ph, err))) break;
+                const uint32_t src = bits_tile(s) + ((MODE == kModeU) ? tg * 16u + 8u * (cur_kb & 1) : jl * 16u + 8u * hgrp);
+                uint2 w;
+                asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(w.x), "=r"(w.y) : "r"(src));
+                expand_store(w, s);
+                s += kExpandGroups;
+                while (s >= stages) {
+                    s -= stages;
+                    ph ^= 1u;
+                }
+                cur_kb += kExpandGroups;
+                while (cur_kb >= nkb) cur_kb -= nkb;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < kPrefetch; ++i) load_next(ring[i]);
+            for (uint32_t it = grp; it < total_it && ok; it += kExpandGroups) {
+                const uint2 wcur = ring[0];
+#pragma unroll
+                for (int j = 0; j + 1 < kPrefetch; ++j) ring[j] = ring[j + 1];
+                load_next(ring[kPrefetch - 1]);
+                if (!(ok = tc::mbar_wait(empty(s), ph ^ 1u, err))) break;
+                expand_store(wcur, s);
+                s += kExpandGroups;
+                while (s >= stages) {
+                    s -= stages;
+                    ph ^= 1u;
+                }
+            }
         }
     } else {
         // ---------------------------------------------------------------- epilogue
@@ -315,17 +397,39 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     }
 }
 
-// Z[m][j] = fp16(bf16 x[m][j] * fp16 s2[j]) for j < d_in; row stride ldz.
+// Z[m][j] = fp16(bf16 x[m][j] * fp16 s2[j]) for j < d_in; row stride ldz.  Rows m by grid y,
+// 8 elements (16 bytes) per thread when d_in is a multiple of 8 (rows 16-byte aligned).
+__device__ __forceinline__ uint32_t scale2_f16(uint32_t xb2, uint32_t sh2) {
+    const float a = bf16_bits_to_float(static_cast<uint16_t>(xb2 & 0xFFFFu)) * f16_bits_to_float(static_cast<uint16_t>(sh2 & 0xFFFFu));
+    const float b = bf16_bits_to_float(static_cast<uint16_t>(xb2 >> 16)) * f16_bits_to_float(static_cast<uint16_t>(sh2 >> 16));
+    return static_cast<uint32_t>(__half_as_ushort(__float2half_rn(a))) |
+           (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(b))) << 16);
+}
+
 __global__ void __launch_bounds__(256) scale_convert_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ s2,
                                                            uint16_t* __restrict__ z, int64_t M, int64_t d_in, int64_t ldz) {
     pdl_wait();
-    const int64_t total = M * d_in;
-    for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
-         e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t m = e / d_in;
-        const int64_t j = e - m * d_in;
-        const float v = bf16_bits_to_float(x[e]) * f16_bits_to_float(s2[j]);
-        z[m * ldz + j] = __half_as_ushort(__float2half_rn(v));
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t m = blockIdx.y; m < M; m += gridDim.y) {
+        const uint16_t* xr = x + m * d_in;
+        uint16_t* zr = z + m * ldz;
+        if ((d_in & 7) == 0) {
+            for (int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; v < d_in / 8; v += stride) {
+                const uint4 xv = __ldg(reinterpret_cast<const uint4*>(xr) + v);
+                const uint4 sv = __ldg(reinterpret_cast<const uint4*>(s2) + v);
+                uint4 o;
+                o.x = scale2_f16(xv.x, sv.x);
+                o.y = scale2_f16(xv.y, sv.y);
+                o.z = scale2_f16(xv.z, sv.z);
+                o.w = scale2_f16(xv.w, sv.w);
+                reinterpret_cast<uint4*>(zr)[v] = o;
+            }
+        } else {
+            for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < d_in; j += stride) {
+                const float v = bf16_bits_to_float(xr[j]) * f16_bits_to_float(s2[j]);
+                zr[j] = __half_as_ushort(__float2half_rn(v));
+            }
+        }
     }
 }
 
@@ -341,6 +445,26 @@ struct PrefillPlan {
     int64_t ldz, ldt;
     size_t off_z, off_t, total;
 };
+
+// Tokens per tile (MMA N, a multiple of 16 up to 256) for a GEMM with n_tiles_w weight tiles:
+// the fewest waves of persistent tiles over the SMs, each wave costing about max(N, 192) + 64
+// (the weight expansion puts a floor under a stage's time; splitting N below it buys nothing).
+// Ties go to the larger N.
+int choose_tile_n(int64_t n_tiles_w, int64_t M, int sms) {
+    int best = 16;
+    int64_t best_cost = -1;
+    const int top = static_cast<int>(std::min<int64_t>(256, round_up(M, 16)));
+    for (int tn = 16; tn <= top; tn += 16) {
+        const int64_t tiles = n_tiles_w * ((M + tn - 1) / tn);
+        const int64_t waves = (tiles + sms - 1) / sms;
+        const int64_t cost = waves * (std::max(tn, 192) + 64);
+        if (best_cost < 0 || cost <= best_cost) {
+            best_cost = cost;
+            best = tn;
+        }
+    }
+    return best;
+}
 
 PrefillPlan plan_prefill(const nq_lrb_layer* L, int64_t M) {
     PrefillPlan p{};
@@ -377,18 +501,46 @@ bool make_tmap(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, i
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-size_t umma_smem_bytes(int tile_n) {
+// 2-D uint32 tensor [rows][ld] of packed signs (nwords valid words per row); box = kBitsWords
+// words x box_rows.  Needs a 16-byte aligned base and row stride; false when not encodable.
+bool make_tmap_bits(CUtensorMap* map, const uint32_t* base, int64_t rows, int64_t nwords, int64_t ld, int box_rows) {
+    auto enc = get_encode();
+    if (!enc || (ld % 4) != 0 || (reinterpret_cast<uintptr_t>(base) & 15u) != 0) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(nwords), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * 4)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(nq::kBitsWords), static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+constexpr size_t kUmmaSmemBudget = 220 * 1024;
+
+size_t umma_stage_bytes(int tile_n) {
     const size_t b = static_cast<size_t>(tile_n) * nq::kTileK * 2;
-    const size_t stage = nq::kABytes + ((b + 1023) & ~static_cast<size_t>(1023));
-    return 1024 /* alignment slack */ + nq::kStages * stage + 8 * (3 * nq::kStages + 6) + 16;
+    return nq::kABytes + ((b + 1023) & ~static_cast<size_t>(1023)) + nq::kBitsBytes;
+}
+
+size_t umma_smem_bytes(int tile_n, int stages) {
+    return 1024 /* alignment slack */ + stages * umma_stage_bytes(tile_n) + 8 * (3 * nq::kMaxStages + 6) + 16;
+}
+
+// As many stages as fit the budget: narrow tiles run short stages, and the ring must cover the
+// latency of a tile's TMA load (about a microsecond) to keep the tensor core fed.
+int umma_stages(int tile_n) {
+    int st = nq::kMaxStages;
+    while (st > 2 && umma_smem_bytes(tile_n, st) > kUmmaSmemBudget) --st;
+    return st;
 }
 
 template <int MODE>
-nq_status launch_umma(const nq::PrefillArgs& a, const CUtensorMap& map, cudaStream_t stream, bool pdl) {
+nq_status launch_umma(const nq::PrefillArgs& a, const CUtensorMap& map, const CUtensorMap& bits_map, cudaStream_t stream,
+                      bool pdl) {
     static bool attr_done[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
-    const size_t smem = umma_smem_bytes(256);
+    const size_t smem = kUmmaSmemBudget;
     if (dev >= 0 && dev < 64 && !attr_done[dev]) {
         if (cudaFuncSetAttribute(nq::lrb_umma_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(smem)) != cudaSuccess)
@@ -399,10 +551,12 @@ nq_status launch_umma(const nq::PrefillArgs& a, const CUtensorMap& map, cudaStre
     int grid = nq_host::sm_count();
     if (grid > tiles) grid = tiles;
     nq::PrefillArgs args = a;
-    CUtensorMap tm = map;
-    void* kargs[] = {&tm, &args};
+    args.stages = umma_stages(a.tile_n);
+    CUtensorMap tm = map, tb = bits_map;
+    void* kargs[] = {&tm, &tb, &args};
     return nq_host::launch_pdl(reinterpret_cast<const void*>(nq::lrb_umma_kernel<MODE>), dim3(grid),
-                               dim3(nq::kPrefillThreads), umma_smem_bytes(a.tile_n), stream, kargs, pdl) == cudaSuccess
+                               dim3(nq::kPrefillThreads), umma_smem_bytes(a.tile_n, args.stages), stream, kargs,
+                               pdl) == cudaSuccess
                ? NQ_OK
                : NQ_ERR_LAUNCH;
 }
@@ -417,20 +571,20 @@ nq_status nq_launch_prefill(const nq_lrb_layer* L, const uint16_t* x, uint16_t* 
     uint16_t* z = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + p.off_z);
     uint16_t* t = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + p.off_t);
     unsigned int* err = nq_host::error_word();
-    const int tile_n = M >= 256 ? 256 : static_cast<int>(round_up(M, 16));
 
     {  // Z = fp16(x * s2)
-        int64_t blocks = (M * L->d_in + 255) / 256;
-        const int64_t cap = 4LL * nq_host::sm_count();
-        if (blocks > cap) blocks = cap;
+        const int64_t per_row = (L->d_in % 8 == 0) ? L->d_in / 8 : L->d_in;  // work items per row
+        const unsigned gx = static_cast<unsigned>(std::min<int64_t>((per_row + 255) / 256, 64));
+        const unsigned gy = static_cast<unsigned>(std::min<int64_t>(M, 65535));
         const uint16_t* s2 = L->s2;
         int64_t d_in = L->d_in, ldz = p.ldz;
         void* args[] = {&x, &s2, &z, &M, &d_in, &ldz};
-        if (nq_host::launch_pdl(reinterpret_cast<const void*>(nq::scale_convert_kernel), dim3(static_cast<unsigned>(blocks)),
-                                dim3(256), 0, stream, args, pdl) != cudaSuccess)
+        if (nq_host::launch_pdl(reinterpret_cast<const void*>(nq::scale_convert_kernel), dim3(gx, gy), dim3(256), 0, stream,
+                                args, pdl) != cudaSuccess)
             return NQ_ERR_LAUNCH;
     }
     {  // T = fp16(Z V): weights = V^T (M-extent r, K = d_in), B = Z
+        const int tile_n = choose_tile_n((L->r + nq::kTileW - 1) / nq::kTileW, M, nq_host::sm_count());
         CUtensorMap map;
         if (!make_tmap(&map, z, M, L->d_in, p.ldz, tile_n)) return NQ_ERR_LAUNCH;
         nq::PrefillArgs a{};
@@ -448,10 +602,14 @@ nq_status nq_launch_prefill(const nq_lrb_layer* L, const uint16_t* x, uint16_t* 
         a.ldo = p.ldt;
         a.s1 = nullptr;
         a.err = err;
-        nq_status st = launch_umma<nq::kModeV>(a, map, stream, pdl);
+        CUtensorMap bmap;
+        std::memset(&bmap, 0, sizeof(bmap));
+        a.bits_tma = make_tmap_bits(&bmap, L->V, L->d_in, L->r / 32, L->ldv, nq::kTileK) ? 1 : 0;
+        nq_status st = launch_umma<nq::kModeV>(a, map, bmap, stream, pdl);
         if (st != NQ_OK) return st;
     }
     {  // Y = bf16(s1 * (T U^T)): weights = U (M-extent d_out, K = r), B = T
+        const int tile_n = choose_tile_n((L->d_out + nq::kTileW - 1) / nq::kTileW, M, nq_host::sm_count());
         CUtensorMap map;
         if (!make_tmap(&map, t, M, L->r, p.ldt, tile_n)) return NQ_ERR_LAUNCH;
         nq::PrefillArgs a{};
@@ -469,7 +627,10 @@ nq_status nq_launch_prefill(const nq_lrb_layer* L, const uint16_t* x, uint16_t* 
         a.ldo = L->d_out;
         a.s1 = L->s1;
         a.err = err;
-        nq_status st = launch_umma<nq::kModeU>(a, map, stream, pdl);
+        CUtensorMap bmap;
+        std::memset(&bmap, 0, sizeof(bmap));
+        a.bits_tma = make_tmap_bits(&bmap, L->U, L->d_out, L->r / 32, L->ldu, nq::kTileW) ? 1 : 0;
+        nq_status st = launch_umma<nq::kModeU>(a, map, bmap, stream, pdl);
         if (st != NQ_OK) return st;
     }
     return NQ_OK;

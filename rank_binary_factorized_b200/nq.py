@@ -99,14 +99,26 @@ class Layer:
         self._ws = {}
 
     @classmethod
-    def from_host(cls, U, V, s1_bits, s2_bits, r: int, device="cuda") -> "Layer":
-        """From numpy arrays: uint32 words and fp16 bit patterns (uint16)."""
+    def from_host(cls, U, V, s1_bits, s2_bits, r: int, device="cuda", ld_align_words: int = 4) -> "Layer":
+        """From numpy arrays: uint32 words and fp16 bit patterns (uint16).  Rows of U and V are
+        padded with zero words to a multiple of `ld_align_words` words: at the default 4 (16
+        bytes) the tensor-core path loads the packed signs by TMA; any stride works."""
         import numpy as np
 
         def dev(a, dt):
             return torch.from_numpy(np.ascontiguousarray(a).view(dt)).to(device)
 
-        return cls(dev(U, np.int32), dev(V, np.int32), dev(s1_bits, np.float16), dev(s2_bits, np.float16), r)
+        def words(a):
+            a = np.ascontiguousarray(a)
+            nw = a.shape[1]
+            ld = -(-nw // ld_align_words) * ld_align_words
+            if ld != nw:
+                b = np.zeros((a.shape[0], ld), dtype=a.dtype)
+                b[:, :nw] = a
+                a = b
+            return dev(a, np.int32)
+
+        return cls(words(U), words(V), dev(s1_bits, np.float16), dev(s2_bits, np.float16), r)
 
     def workspace_bytes(self, M: int) -> int:
         return int(_lib.nq_workspace_bytes(ctypes.byref(self.struct), M))

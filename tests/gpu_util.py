@@ -31,8 +31,8 @@ def nq():
     return mod
 
 
-def upload_projection(p, device="cuda"):
-    return nq().Layer.from_host(p.U, p.V, p.s1, p.s2, p.r, device=device)
+def upload_projection(p, device="cuda", ld_align_words=4):
+    return nq().Layer.from_host(p.U, p.V, p.s1, p.s2, p.r, device=device, ld_align_words=ld_align_words)
 
 
 def upload_bf16(bits):

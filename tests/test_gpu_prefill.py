@@ -20,8 +20,8 @@ from tests.gpu_util import (check_tolerance, download_bf16_bits, need_gpu, nq, u
 pytestmark = pytest.mark.gpu
 
 
-def gpu_matmul(p, xb, fn="lrb_matmul"):
-    L = upload_projection(p)
+def gpu_matmul(p, xb, fn="lrb_matmul", ld_align_words=4):
+    L = upload_projection(p, ld_align_words=ld_align_words)
     y = getattr(nq(), fn)(L, upload_bf16(xb))
     nq().sync_status()
     return download_bf16_bits(y)
@@ -44,13 +44,16 @@ def test_tiny_layer_token_counts(M):
     (1, 8, 32, 1, 1, 9),
     (640, 200, 2048, 64, 66, 33),
 ])
-def test_ragged_and_padded(d_out, d_in, r, ldu, ldv, M):
+@pytest.mark.parametrize("align", [1, 4])
+def test_ragged_and_padded(d_out, d_in, r, ldu, ldv, M, align):
+    # align 1 keeps the given row strides (odd ones load the packed signs with plain loads);
+    # align 4 pads them to 16 bytes (the signs arrive by TMA)
     need_gpu()
     p = synth.make_projection("ragged", d_out, d_in, r, seed=402, key=d_out + 3 * d_in, ldu=ldu, ldv=ldv)
     xb = synth.acts_bf16(synth.rng_for(403, d_in, M), (M, d_in))
-    y = gpu_matmul(p, xb)
+    y = gpu_matmul(p, xb, ld_align_words=align)
     y_ref, S = oracle.dense_packed(p.U, p.V, p.s1, p.s2, p.r, xb)
-    check_tolerance(y, y_ref, S, "prefill ragged %r" % ((d_out, d_in, r, ldu, ldv, M),))
+    check_tolerance(y, y_ref, S, "prefill ragged %r align %d" % ((d_out, d_in, r, ldu, ldv, M), align))
 
 
 @pytest.mark.parametrize("d_out,d_in,r,M", [(256, 512, 128, 64), (1024, 2048, 512, 300), (4096, 1024, 1024, 40)])
