@@ -470,7 +470,7 @@ PrefillPlan plan_prefill(const nq_lrb_layer* L, int64_t M) {
     PrefillPlan p{};
     p.ldz = round_up(L->d_in, 8);  // 16-byte aligned rows for TMA
     p.ldt = round_up(L->r, 8);
-    p.off_z = NQ_WS_HEADER_BYTES;  // the header belongs to the decode path's tickets
+    p.off_z = NQ_WS_HEADER_BYTES;  // past the reserved workspace header
     p.off_t = p.off_z + align256(static_cast<size_t>(M * p.ldz) * 2);
     p.total = p.off_t + align256(static_cast<size_t>(M * p.ldt) * 2);
     return p;
