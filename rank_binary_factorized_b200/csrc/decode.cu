@@ -211,37 +211,68 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const S1Params p) 
     pdl_launch_dependents();
     pdl_wait();     // x may be written by the previous grid
 
-    // ---- slice scale: |z_q| < 2^22, z_q = rint(z * 2^shift)
+    // ---- slice scale: |z_q| < 2^22, z_q = rint(z * 2^shift).  The batch rows are the inner,
+    // unrolled loop, so every row's loads of x are in flight together.
+    constexpr int MGS = (NT * 8 + 2) / 3;  // batch rows the B columns can hold (>= M)
     {
-        for (int m = 0; m < p.M; ++m) {
-            const uint16_t* xm = p.x + static_cast<int64_t>(m) * p.d_in;
-            float v = 0.0f;
-            if (s2reg) {
+        float vmax[MGS];
 #pragma unroll
-                for (int i = 0; i < kS2Reg; ++i) {
-                    const int64_t j = j0 + tid + static_cast<int64_t>(i) * kS1Threads;
-                    if (j < j1) {
-                        const float z = s2r[i] * bf16_bits_to_float(xm[j]);
+        for (int m = 0; m < MGS; ++m) vmax[m] = 0.0f;
+        if (s2reg && p.M == 1) {
+#pragma unroll
+            for (int i = 0; i < kS2Reg; ++i) {
+                const int64_t j = j0 + tid + static_cast<int64_t>(i) * kS1Threads;
+                if (j < j1) {
+                    const float z = s2r[i] * bf16_bits_to_float(p.x[j]);
+                    if (p.zstage) {
+                        const int jl = static_cast<int>(j - j0);
+                        zs_s[jl + (jl >> 5)] = z;
+                    }
+                    vmax[0] = fmaxf(vmax[0], fabsf(z));
+                }
+            }
+        } else if (s2reg) {
+#pragma unroll
+            for (int i = 0; i < kS2Reg; ++i) {
+                const int64_t j = j0 + tid + static_cast<int64_t>(i) * kS1Threads;
+                if (j < j1) {
+#pragma unroll
+                    for (int m = 0; m < MGS; ++m) {
+                        if (m < p.M) {
+                            const float z = s2r[i] * bf16_bits_to_float(p.x[static_cast<int64_t>(m) * p.d_in + j]);
+                            if (p.zstage) {
+                                const int jl = static_cast<int>(j - j0);
+                                zs_s[m * zld + jl + (jl >> 5)] = z;
+                            }
+                            vmax[m] = fmaxf(vmax[m], fabsf(z));
+                        }
+                    }
+                }
+            }
+        } else {
+#pragma unroll 4
+            for (int64_t j = j0 + tid; j < j1; j += kS1Threads) {
+                const float s2v = f16_bits_to_float(p.s2[j]);
+#pragma unroll
+                for (int m = 0; m < MGS; ++m) {
+                    if (m < p.M) {
+                        const float z = s2v * bf16_bits_to_float(p.x[static_cast<int64_t>(m) * p.d_in + j]);
                         if (p.zstage) {
                             const int jl = static_cast<int>(j - j0);
                             zs_s[m * zld + jl + (jl >> 5)] = z;
                         }
-                        v = fmaxf(v, fabsf(z));
+                        vmax[m] = fmaxf(vmax[m], fabsf(z));
                     }
-                }
-            } else {
-#pragma unroll 8
-                for (int64_t j = j0 + tid; j < j1; j += kS1Threads) {
-                    const float z = f16_bits_to_float(p.s2[j]) * bf16_bits_to_float(xm[j]);
-                    if (p.zstage) {
-                        const int jl = static_cast<int>(j - j0);
-                        zs_s[m * zld + jl + (jl >> 5)] = z;
-                    }
-                    v = fmaxf(v, fabsf(z));
                 }
             }
-            for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
-            if (lane == 0) s_wmax[warp][m] = v;
+        }
+#pragma unroll
+        for (int m = 0; m < MGS; ++m) {
+            if (m < p.M) {
+                float v = vmax[m];
+                for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+                if (lane == 0) s_wmax[warp][m] = v;
+            }
         }
         for (int e = tid; e < kS1Outs * NT * 8; e += kS1Threads) red[e] = 0;
         if (tid < NQ_MATVEC_MAX_M) s_zsum[tid] = 0ull;
@@ -507,19 +538,40 @@ __global__ void __launch_bounds__(TH, 1) decode_stage2_kernel(const S2Params p) 
     pdl_launch_dependents();
     pdl_wait();  // t comes from stage 1 of this call
 
-    // ---- per-batch-row scale: |t_q| < 2^22 with t_q = rint(t * 2^shift)
+    // ---- per-batch-row scale: |t_q| < 2^22 with t_q = rint(t * 2^shift).  The batch rows are
+    // the inner, unrolled loop, so every row's loads of t are in flight together.
+    constexpr int MGS = (NT * 8 + 2) / 3;  // batch rows the B columns can hold (>= M)
     {
-        for (int m = 0; m < p.M; ++m) {
-            const float* tm = p.t + static_cast<int64_t>(m) * p.r;
-            float v = 0.0f;
+        float vmax[MGS];
+#pragma unroll
+        for (int m = 0; m < MGS; ++m) vmax[m] = 0.0f;
+        if (p.M == 1) {
 #pragma unroll 8
             for (int k = tid; k < p.r; k += kS2Threads) {
-                const float tv = tm[k];
-                if (p.tstage) ts_s[m * (p.r + p.r / 32) + k + (k >> 5)] = tv;
-                v = fmaxf(v, fabsf(tv));
+                const float tv = p.t[k];
+                if (p.tstage) ts_s[k + (k >> 5)] = tv;
+                vmax[0] = fmaxf(vmax[0], fabsf(tv));
             }
-            for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
-            if (lane == 0) s_wmax[warp][m] = v;
+        } else {
+#pragma unroll 4
+            for (int k = tid; k < p.r; k += kS2Threads) {
+#pragma unroll
+                for (int m = 0; m < MGS; ++m) {
+                    if (m < p.M) {
+                        const float tv = p.t[static_cast<int64_t>(m) * p.r + k];
+                        if (p.tstage) ts_s[m * (p.r + p.r / 32) + k + (k >> 5)] = tv;
+                        vmax[m] = fmaxf(vmax[m], fabsf(tv));
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int m = 0; m < MGS; ++m) {
+            if (m < p.M) {
+                float v = vmax[m];
+                for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+                if (lane == 0) s_wmax[warp][m] = v;
+            }
         }
         if (tid < NQ_MATVEC_MAX_M) s_tsum[tid] = 0ull;
         __syncthreads();
@@ -786,7 +838,7 @@ nq_status launch_decode_nt(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y
         q.chunk_mt = chunk;
         size_t smem2 = bt_bytes + chunk * per_mt;
         const size_t t_bytes = static_cast<size_t>(M) * (L->r + L->r / 32) * sizeof(float);
-        q.tstage = (smem2 + t_bytes <= kStage2SmemBudget && t_bytes <= 48 * 1024) ? 1 : 0;
+        q.tstage = (smem2 + t_bytes <= kStage2SmemBudget) ? 1 : 0;
         if (q.tstage) smem2 += t_bytes;
         void* args[] = {&q};
         const bool wide = (NT == 1) && per_cta >= 6;
