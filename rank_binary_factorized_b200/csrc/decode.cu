@@ -139,8 +139,8 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const S1Params p) 
     double* part = reinterpret_cast<double*>(red + kS1Outs * NT * 8);   // inbox [M][per][CS]
     float* zs_s = reinterpret_cast<float*>(part + p.M * (kS1Outs + 16));  // [M][zld] when p.zstage
     const int zld = p.rows_per_slice + p.rows_per_slice / 32;             // one pad word per 32
-    __shared__ int s_shift[NQ_MATVEC_MAX_M];
     __shared__ float s_mul[NQ_MATVEC_MAX_M];
+    __shared__ double s_dinv[NQ_MATVEC_MAX_M];  // 2^-shift: turns the exact integers into values
     __shared__ unsigned long long s_zsum[NQ_MATVEC_MAX_M];
     __shared__ float s_wmax[kS1Threads / 32][NQ_MATVEC_MAX_M];
 
@@ -283,8 +283,8 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const S1Params p) 
             int e = 0;
             frexpf(v, &e);
             const int sh = (v > 0.0f) ? min(max(22 - e, -126), 126) : 0;
-            s_shift[tid] = sh;
             s_mul[tid] = ldexpf(1.0f, sh);
+            s_dinv[tid] = ldexp(1.0, -sh);
         }
         __syncthreads();
     }
@@ -416,28 +416,38 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const S1Params p) 
     // block of rank k / per; every block stores its fp64 partial for k into slot [rank of
     // the sender] of the owner's inbox (distributed shared memory), one cluster barrier
     // publishes the stores, and each owner sums its slots in rank order.
-    const int per = (kS1Outs + CS - 1) / CS;
+    // CS is a power of two (1 .. 16), so is the share per owner; the exact integer times the
+    // power of two 2^-shift is exact in fp64
+    const int lg_per = 8 - (31 - __clz(CS));  // log2(kS1Outs / CS)
+    const int per = 1 << lg_per;
     for (int e = tid; e < p.M * kS1Outs; e += kS1Threads) {
         const int m = e / kS1Outs, kl = e - m * kS1Outs;
         const int* rr = red + kl * (NT * 8) + 3 * m;
         const long long P = static_cast<long long>(rr[0]) + (static_cast<long long>(rr[1]) << 8) +
                             (static_cast<long long>(rr[2]) << 16);
         const long long val = 2 * P - static_cast<long long>(s_zsum[m]);
-        const int owner = kl / per, ko = kl - owner * per;
+        const int owner = kl >> lg_per, ko = kl & (per - 1);
         double* dst = cluster.map_shared_rank(part, owner);
-        dst[(m * per + ko) * CS + q] = ldexp(static_cast<double>(val), -s_shift[m]);
+        dst[(m * per + ko) * CS + q] = static_cast<double>(val) * s_dinv[m];
     }
     cluster.sync();
     {
-        const int k_lo = q * per, k_hi = min(kS1Outs, k_lo + per);
-        for (int e = tid; e < p.M * (k_hi - k_lo); e += kS1Threads) {
-            const int m = e / (k_hi - k_lo), ko = e - m * (k_hi - k_lo);
+        // owner q: its `per` outputs, each the sum of the CS slices' partials in a fixed order
+        // (four interleaved accumulators, then pairwise): a short dependent chain, few registers
+        const int k_lo = q * per;
+        for (int e = tid; e < p.M * per; e += kS1Threads) {
+            const int m = e >> lg_per, ko = e & (per - 1);
             const int64_t k = static_cast<int64_t>(wglob0) * 32 + k_lo + ko;
             if (k < p.r) {
                 const double* src = part + (m * per + ko) * CS;
-                double sum = 0.0;
-                for (int rank = 0; rank < CS; ++rank) sum += src[rank];
-                p.t[static_cast<int64_t>(m) * p.r + k] = static_cast<float>(sum);
+                double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+                for (int rank = 0; rank < CS; rank += 4) {
+                    a0 += src[rank];
+                    if (rank + 1 < CS) a1 += src[rank + 1];
+                    if (rank + 2 < CS) a2 += src[rank + 2];
+                    if (rank + 3 < CS) a3 += src[rank + 3];
+                }
+                p.t[static_cast<int64_t>(m) * p.r + k] = static_cast<float>((a0 + a1) + (a2 + a3));
             }
         }
     }
@@ -494,8 +504,8 @@ __global__ void __launch_bounds__(TH, 1) decode_stage2_kernel(const S2Params p) 
     int* red = reinterpret_cast<int*>(ublk + p.chunk_mt * 16 * p.su);  // [chunk_mt*16][NT*8]
     float* s1_s = reinterpret_cast<float*>(red + p.chunk_mt * 16 * NT * 8);  // [chunk_mt*16]
     float* ts_s = s1_s + p.chunk_mt * 16;                                   // [M][r] when p.tstage
-    __shared__ int s_shift[NQ_MATVEC_MAX_M];
     __shared__ float s_mul[NQ_MATVEC_MAX_M];
+    __shared__ double s_dinv[NQ_MATVEC_MAX_M];  // 2^-shift: turns the exact integers into values
     __shared__ unsigned long long s_tsum[NQ_MATVEC_MAX_M];
     __shared__ float s_wmax[kS2Warps][NQ_MATVEC_MAX_M];
 
@@ -581,8 +591,8 @@ __global__ void __launch_bounds__(TH, 1) decode_stage2_kernel(const S2Params p) 
             int e = 0;
             frexpf(v, &e);  // v < 2^e
             const int sh = (v > 0.0f) ? min(max(22 - e, -126), 126) : 0;
-            s_shift[tid] = sh;
             s_mul[tid] = ldexpf(1.0f, sh);
+            s_dinv[tid] = ldexp(1.0, -sh);
         }
         __syncthreads();
         // t staged with one pad word after every 32 values, so that the table build's
@@ -705,14 +715,14 @@ __global__ void __launch_bounds__(TH, 1) decode_stage2_kernel(const S2Params p) 
 
         // epilogue: y = s1 * 2^-shift * (2 P - Tsum), P = d0 + 2^8 d1 + 2^16 d2
         for (int e = tid; e < nmt * 16 * p.M; e += kS2Threads) {
-            const int row = e / p.M, m = e - row * p.M;
+            const int row = (p.M == 1) ? e : e / p.M, m = e - row * p.M;
             const int64_t i = static_cast<int64_t>(c0) * 16 + row;
             if (i < p.d_out) {
                 const int* rr = red + row * (NT * 8) + 3 * m;
                 const long long P = static_cast<long long>(rr[0]) + (static_cast<long long>(rr[1]) << 8) +
                                     (static_cast<long long>(rr[2]) << 16);
                 const long long val = 2 * P - static_cast<long long>(s_tsum[m]);
-                const double yv = static_cast<double>(s1_s[row]) * ldexp(static_cast<double>(val), -s_shift[m]);
+                const double yv = static_cast<double>(s1_s[row]) * (static_cast<double>(val) * s_dinv[m]);
                 p.y[static_cast<int64_t>(m) * p.d_out + i] = __bfloat16_as_ushort(__double2bfloat16(yv));
             }
         }
