@@ -274,7 +274,8 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const S1Params p) 
                 if (lane == 0) s_wmax[warp][m] = v;
             }
         }
-        for (int e = tid; e < kS1Outs * NT * 8; e += kS1Threads) red[e] = 0;
+        if (kKSplit > 1)  // several warps add into one output; otherwise each stores its own
+            for (int e = tid; e < kS1Outs * NT * 8; e += kS1Threads) red[e] = 0;
         if (tid < NQ_MATVEC_MAX_M) s_zsum[tid] = 0ull;
         __syncthreads();
         if (tid < p.M) {
@@ -353,9 +354,11 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const S1Params p) 
                         if (mm == m) zacc[mm] += qsum;
                 }
                 uint32_t* dst = zq + jq * SWZ + 3 * m;
-                if (3 * m < NT * 8) dst[0] = d0;
-                if (3 * m + 1 < NT * 8) dst[1] = d1;
-                if (3 * m + 2 < NT * 8) dst[2] = d2;
+                if (m < p.M) {  // rows >= M: their D columns are never read
+                    dst[0] = d0;
+                    dst[1] = d1;
+                    dst[2] = d2;
+                }
             }
         }
         __syncthreads();
@@ -408,7 +411,9 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const S1Params p) 
                 for (int e = 0; e < 4; ++e) {
                     const int kl = 32 * wcol + 8 * (2 * h + (e >> 1)) + gid;
                     const int col = nt * 8 + 2 * tig + (e & 1);
-                    atomicAdd(&red[kl * (NT * 8) + col], (acc[0][h][nt][e] >> gid) + (acc[1][h][nt][e] >> gid));
+                    const int v = (acc[0][h][nt][e] >> gid) + (acc[1][h][nt][e] >> gid);
+                    if (kKSplit == 1) red[kl * (NT * 8) + col] = v;
+                    else atomicAdd(&red[kl * (NT * 8) + col], v);
                 }
     }
     __syncthreads();
@@ -632,9 +637,11 @@ __global__ void __launch_bounds__(TH, 1) decode_stage2_kernel(const S2Params p) 
                     }
                     tacc[m] += qsum;
                 }
-                if (3 * m < NT * 8) bt[s2_bidx<NT>(s_, w, 3 * m, ngp)] = d0;
-                if (3 * m + 1 < NT * 8) bt[s2_bidx<NT>(s_, w, 3 * m + 1, ngp)] = d1;
-                if (3 * m + 2 < NT * 8) bt[s2_bidx<NT>(s_, w, 3 * m + 2, ngp)] = d2;
+                if (m < p.M) {  // rows >= M: their D columns are never read
+                    bt[s2_bidx<NT>(s_, w, 3 * m, ngp)] = d0;
+                    bt[s2_bidx<NT>(s_, w, 3 * m + 1, ngp)] = d1;
+                    bt[s2_bidx<NT>(s_, w, 3 * m + 2, ngp)] = d2;
+                }
             }
         }
         // per-warp partial sums into s_tsum; read by the epilogue, after the barriers below
