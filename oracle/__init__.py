@@ -77,6 +77,12 @@ def lib() -> ctypes.CDLL:
                                              _p, _i64, _p, _p]
         L.nq_oracle_factored_packed.restype = ctypes.c_int
         L.nq_oracle_factored_packed.argtypes = [_p, _i64, _p, _i64, _p, _p, _i64, _i64, _i64, _p, _i64, _p]
+        L.nq_oracle_transposed_packed.restype = ctypes.c_int
+        L.nq_oracle_transposed_packed.argtypes = [_p, _i64, _p, _i64, _p, _p, _i64, _i64, _i64, _p, _i64,
+                                                  _p, _i64, _p, _p]
+        L.nq_oracle_scale_grads_packed.restype = ctypes.c_int
+        L.nq_oracle_scale_grads_packed.argtypes = [_p, _i64, _p, _i64, _p, _p, _i64, _i64, _i64, _p, _p, _i64,
+                                                   _p, _p, _p, _p]
         L.nq_oracle_silu_mul.restype = None
         L.nq_oracle_silu_mul.argtypes = [_p, _p, _i64, _p]
         L.nq_oracle_round_bf16.restype = None
@@ -214,6 +220,49 @@ def dense_packed(Uw, Vw, s1_f16, s2_f16, r: int, x_bf16, rows=None):
     if rc != 0:
         raise ValueError("nq_oracle_dense_packed failed (%d)" % rc)
     return y, S
+
+
+def transposed_packed(Uw, Vw, s1_f16, s2_f16, r: int, ybar_bf16, cols=None):
+    """The layer's transpose, xbar[b][j] = sum_i W_ij ybar[b][i] (Phase 3 scale-only
+    calibration backpropagates through the frozen factors), on the packed layout.  ``cols``
+    selects output columns j (all d_in when None).  Returns (xbar, S), each [B][n_cols]."""
+    Uw = _c(Uw, np.uint32)
+    Vw = _c(Vw, np.uint32)
+    s1 = _c(s1_f16, np.uint16)
+    s2 = _c(s2_f16, np.uint16)
+    yb = _c(np.atleast_2d(ybar_bf16), np.uint16)
+    d_out, d_in, B = Uw.shape[0], Vw.shape[0], yb.shape[0]
+    cols_arr = None if cols is None else _c(cols, np.int64)
+    n = d_in if cols is None else cols_arr.size
+    xbar = np.empty((B, n), dtype=np.float64)
+    S = np.empty((B, n), dtype=np.float64)
+    rc = lib().nq_oracle_transposed_packed(_ptr(Uw), Uw.shape[1], _ptr(Vw), Vw.shape[1], _ptr(s1), _ptr(s2), d_out,
+                                           d_in, r, _ptr(yb), B, None if cols_arr is None else _ptr(cols_arr), n,
+                                           _ptr(xbar), _ptr(S))
+    if rc != 0:
+        raise ValueError("nq_oracle_transposed_packed failed (%d)" % rc)
+    return xbar, S
+
+
+def scale_grads_packed(Uw, Vw, s1_f16, s2_f16, r: int, x_bf16, ybar_bf16):
+    """dL/ds1 and dL/ds2 for L = sum_b <ybar_b, y_b>, with the magnitudes of their terms.
+    Returns (g1 [d_out], S1 [d_out], g2 [d_in], S2 [d_in]), fp64."""
+    Uw = _c(Uw, np.uint32)
+    Vw = _c(Vw, np.uint32)
+    s1 = _c(s1_f16, np.uint16)
+    s2 = _c(s2_f16, np.uint16)
+    x = _c(np.atleast_2d(x_bf16), np.uint16)
+    yb = _c(np.atleast_2d(ybar_bf16), np.uint16)
+    d_out, d_in, B = Uw.shape[0], Vw.shape[0], x.shape[0]
+    if yb.shape != (B, d_out) or x.shape != (B, d_in):
+        raise ValueError("x must be [B][d_in] and ybar [B][d_out]")
+    g1, S1 = np.empty(d_out), np.empty(d_out)
+    g2, S2 = np.empty(d_in), np.empty(d_in)
+    rc = lib().nq_oracle_scale_grads_packed(_ptr(Uw), Uw.shape[1], _ptr(Vw), Vw.shape[1], _ptr(s1), _ptr(s2), d_out,
+                                            d_in, r, _ptr(x), _ptr(yb), B, _ptr(g1), _ptr(S1), _ptr(g2), _ptr(S2))
+    if rc != 0:
+        raise ValueError("nq_oracle_scale_grads_packed failed (%d)" % rc)
+    return g1, S1, g2, S2
 
 
 def factored_packed(Uw, Vw, s1_f16, s2_f16, r: int, x_bf16) -> np.ndarray:

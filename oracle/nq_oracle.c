@@ -274,6 +274,102 @@ ORACLE_API int nq_oracle_factored_packed(const uint32_t* U, int64_t ldu, const u
 }
 
 /* ---------------------------------------------------------------------------------
+ * Products through the frozen factors for scale-only calibration (section 3, "Phase 3:
+ * Scale-Only Model Reconstruction": U and V stay fixed while s1 and s2 are optimised, so
+ * the training step needs the layer's transpose and the derivatives of its output with
+ * respect to the two scale vectors).  Both follow from the section 2 equation read
+ * elementwise, W_ij = s1_i G_ij s2_j, y[b][i] = sum_j W_ij x[b][j]:
+ *
+ *   transpose:   xbar[b][j] = sum_i W_ij ybar[b][i]
+ *   scale grads: for L = sum_b sum_i ybar[b][i] y[b][i] (ybar the cotangent of y),
+ *                dL/ds1_i = sum_b ybar[b][i] sum_j G_ij s2_j x[b][j]
+ *                dL/ds2_j = sum_b x[b][j]    sum_i G_ij s1_i ybar[b][i]
+ * --------------------------------------------------------------------------------- */
+
+/* The transpose on the packed layout, for a chosen subset of output columns j (cols ==
+ * NULL means all d_in, in order).  ybar [B][d_out] bf16 bits; xbar, S [B][n_cols], with
+ * S[b][n] = sum_i |W_ij ybar[b][i]|. */
+ORACLE_API int nq_oracle_transposed_packed(const uint32_t* U, int64_t ldu, const uint32_t* V, int64_t ldv,
+                                           const uint16_t* s1_f16, const uint16_t* s2_f16, int64_t d_out,
+                                           int64_t d_in, int64_t r, const uint16_t* ybar_bf16, int64_t B,
+                                           const int64_t* cols, int64_t n_cols, double* xbar, double* S) {
+    if (r % 32 != 0 || ldu < r / 32 || ldv < r / 32) return -1;
+    if (cols == NULL) n_cols = d_in;
+    double* s1 = (double*)malloc(sizeof(double) * (size_t)(d_out > 0 ? d_out : 1));
+    double* yb = (double*)malloc(sizeof(double) * (size_t)(B * d_out > 0 ? B * d_out : 1));
+    if (!s1 || !yb) {
+        free(s1);
+        free(yb);
+        return -2;
+    }
+    for (int64_t i = 0; i < d_out; ++i) s1[i] = nq_oracle_f16_to_double(s1_f16[i]);
+    for (int64_t e = 0; e < B * d_out; ++e) yb[e] = nq_oracle_bf16_to_double(ybar_bf16[e]);
+    for (int64_t n = 0; n < n_cols; ++n) {
+        int64_t j = cols ? cols[n] : n;
+        if (j < 0 || j >= d_in) {
+            free(s1);
+            free(yb);
+            return -1;
+        }
+        double s2 = nq_oracle_f16_to_double(s2_f16[j]);
+        for (int64_t b = 0; b < B; ++b) {
+            xbar[b * n_cols + n] = 0.0;
+            if (S) S[b * n_cols + n] = 0.0;
+        }
+        for (int64_t i = 0; i < d_out; ++i) {
+            double w = s1[i] * (double)gram_entry_packed(U + i * ldu, V + j * ldv, r) * s2;
+            for (int64_t b = 0; b < B; ++b) {
+                double term = w * yb[b * d_out + i];
+                xbar[b * n_cols + n] += term;
+                if (S) S[b * n_cols + n] += fabs(term);
+            }
+        }
+    }
+    free(s1);
+    free(yb);
+    return 0;
+}
+
+/* Both scale gradients on the packed layout, with the magnitudes of their terms:
+ * g1, S1 [d_out]; g2, S2 [d_in].  x [B][d_in], ybar [B][d_out] bf16 bits. */
+ORACLE_API int nq_oracle_scale_grads_packed(const uint32_t* U, int64_t ldu, const uint32_t* V, int64_t ldv,
+                                            const uint16_t* s1_f16, const uint16_t* s2_f16, int64_t d_out,
+                                            int64_t d_in, int64_t r, const uint16_t* x_bf16,
+                                            const uint16_t* ybar_bf16, int64_t B, double* g1, double* S1,
+                                            double* g2, double* S2) {
+    if (r % 32 != 0 || ldu < r / 32 || ldv < r / 32) return -1;
+    double* x = (double*)malloc(sizeof(double) * (size_t)(B * d_in > 0 ? B * d_in : 1));
+    double* yb = (double*)malloc(sizeof(double) * (size_t)(B * d_out > 0 ? B * d_out : 1));
+    if (!x || !yb) {
+        free(x);
+        free(yb);
+        return -2;
+    }
+    for (int64_t e = 0; e < B * d_in; ++e) x[e] = nq_oracle_bf16_to_double(x_bf16[e]);
+    for (int64_t e = 0; e < B * d_out; ++e) yb[e] = nq_oracle_bf16_to_double(ybar_bf16[e]);
+    for (int64_t i = 0; i < d_out; ++i) g1[i] = S1[i] = 0.0;
+    for (int64_t j = 0; j < d_in; ++j) g2[j] = S2[j] = 0.0;
+    for (int64_t i = 0; i < d_out; ++i) {
+        double s1 = nq_oracle_f16_to_double(s1_f16[i]);
+        for (int64_t j = 0; j < d_in; ++j) {
+            double g = (double)gram_entry_packed(U + i * ldu, V + j * ldv, r);
+            double s2 = nq_oracle_f16_to_double(s2_f16[j]);
+            for (int64_t b = 0; b < B; ++b) {
+                double t1 = yb[b * d_out + i] * g * s2 * x[b * d_in + j];
+                double t2 = x[b * d_in + j] * g * s1 * yb[b * d_out + i];
+                g1[i] += t1;
+                S1[i] += fabs(t1);
+                g2[j] += t2;
+                S2[j] += fabs(t2);
+            }
+        }
+    }
+    free(x);
+    free(yb);
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------------
  * SiLU-gated product between the gate/up and down projections of a Llama MLP block.  This
  * is not on the pages; it is the MLP composition of the 7B/70B workloads:
  *   h = bf16( silu(g) * u ),  silu(g) = g / (1 + exp(-g)),  in fp64 before the rounding.

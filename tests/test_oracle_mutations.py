@@ -33,9 +33,26 @@ MUTATIONS = [
     ("v = ldexp((double)(1024 + f), e - 25);", "v = ldexp((double)(1024 + f), e - 24);"),
 ]
 
+# mistakes in the calibration products, caught by their own pins
+CAL = "test_oracle_calibration.py"
+MUTATIONS += [
+    # transpose: a dropped s2
+    ("double w = s1[i] * (double)gram_entry_packed(U + i * ldu, V + j * ldv, r) * s2;",
+     "double w = s1[i] * (double)gram_entry_packed(U + i * ldu, V + j * ldv, r);", CAL),
+    # transpose: the cotangent read at the wrong row
+    ("double term = w * yb[b * d_out + i];", "double term = w * yb[b * d_out + (d_out - 1 - i)];", CAL),
+    # dL/ds1: a dropped s2
+    ("double t1 = yb[b * d_out + i] * g * s2 * x[b * d_in + j];",
+     "double t1 = yb[b * d_out + i] * g * x[b * d_in + j];", CAL),
+    # dL/ds2: s2 where s1 belongs
+    ("double t2 = x[b * d_in + j] * g * s1 * yb[b * d_out + i];",
+     "double t2 = x[b * d_in + j] * g * s2 * yb[b * d_out + i];", CAL),
+]
+MUTATIONS = [m if len(m) == 3 else (m[0], m[1], "test_oracle.py") for m in MUTATIONS]
 
-@pytest.mark.parametrize("old,new", MUTATIONS)
-def test_pins_fail_on_planted_mistake(tmp_path, old, new):
+
+@pytest.mark.parametrize("old,new,pins", MUTATIONS)
+def test_pins_fail_on_planted_mistake(tmp_path, old, new, pins):
     src = open(SRC).read()
     assert old in src, "mutation anchor not found"
     mutant = tmp_path / "mutant.c"
@@ -44,6 +61,6 @@ def test_pins_fail_on_planted_mistake(tmp_path, old, new):
     subprocess.check_call(["gcc", "-std=c11", "-O2", "-fPIC", "-shared", "-o", str(so), str(mutant), "-lm"])
     env = dict(os.environ, NQ_ORACLE_SO=str(so))
     proc = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
-                           os.path.join(ROOT, "tests", "test_oracle.py")],
+                           os.path.join(ROOT, "tests", pins)],
                           cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
     assert proc.returncode != 0, "pins passed on a planted mistake: " + new
