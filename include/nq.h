@@ -101,8 +101,9 @@ NQ_API nq_status nq_pack_signs(const float* latent, int64_t rows, int64_t r, int
                         int64_t ld_words, void* stream);
 
 /*
- * nq_workspace_bytes -- device scratch a call with M activation rows needs (for both
- * nq_lrb_matvec and nq_lrb_matmul through nq_layer_forward).  Returns 0 for an invalid
+ * nq_workspace_bytes -- device scratch a call with M activation rows needs (for
+ * nq_lrb_matvec, nq_lrb_matmul, nq_layer_forward, nq_lrb_transposed and
+ * nq_lrb_scale_grads alike).  Returns 0 for an invalid
  * layer or M.  The workspace must stay untouched by other work while the call runs.  Its
  * first 4096 bytes hold counters that read zero between calls (the library restores them
  * before each call ends); the rest is scratch.  So one workspace can be reused by
@@ -135,6 +136,38 @@ NQ_API nq_status nq_lrb_matmul(const nq_lrb_layer* L, const uint16_t* x, uint16_
 /* nq_layer_forward -- M <= NQ_MATVEC_MAX_M: nq_lrb_matvec; otherwise nq_lrb_matmul. */
 NQ_API nq_status nq_layer_forward(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y, int64_t M, void* ws,
                            size_t ws_bytes, void* stream);
+
+/*
+ * Calibration products.  Page "NanoQuant: Efficient Sub-1-Bit Quantization of Large Language
+ * Models", section 3, "Phase 3: Scale-Only Model Reconstruction": with U and V frozen and
+ * packed, only s1 and s2 are optimised, so a training step needs the layer's transpose (to
+ * carry the output gradient to the layer's input) and the gradients with respect to the two
+ * scale vectors.  Both come from the section 2 equation read elementwise,
+ * W_ij = s1_i (sum_k U_ik V_jk) s2_j.
+ *
+ * nq_lrb_transposed -- xbar[m][j] = bf16( sum_i W_ij ybar[m][i] )
+ *                                = bf16( s2_j sum_k V_jk sum_i U_ik s1_i ybar[m][i] ).
+ *   ybar [M][d_out] bf16 (the cotangent of y), xbar [M][d_in] bf16.  Computed as the forward
+ *   product of the layer with (U, s1, d_out) and (V, s2, d_in) exchanged: M <= NQ_MATVEC_MAX_M
+ *   on the decode path, larger M on the tensor cores, with the same numerics as
+ *   nq_lrb_matvec and nq_lrb_matmul respectively.  ws: nq_workspace_bytes(L, M) bytes.
+ */
+NQ_API nq_status nq_lrb_transposed(const nq_lrb_layer* L, const uint16_t* ybar, uint16_t* xbar, int64_t M, void* ws,
+                                   size_t ws_bytes, void* stream);
+
+/*
+ * nq_lrb_scale_grads -- for L = sum_m sum_i ybar[m][i] y[m][i], y = the layer applied to x:
+ *   g_s1[i] = dL/ds1_i = sum_m ybar[m][i] sum_k U_ik t[m][k],  t[m] = V^T (s2 . x[m])
+ *   g_s2[j] = dL/ds2_j = sum_m x[m][j]    sum_k V_jk u[m][k],  u[m] = U^T (s1 . ybar[m])
+ *   x [M][d_in] and ybar [M][d_out] bf16; g_s1 [d_out] and g_s2 [d_in] fp32, overwritten
+ *   (16-byte aligned).  M <= NQ_MATVEC_MAX_M: the decode kernels' exact integer sums of the
+ *   23-bit quantised activations, weighted by the cotangent and summed over m in fp64.
+ *   Larger M: the tensor-core products (fp16 operands, fp32 accumulation), weighted and summed
+ *   over tokens in fp64, token tiles in a fixed order: run-to-run identical.
+ *   ws: nq_workspace_bytes(L, M) bytes.
+ */
+NQ_API nq_status nq_lrb_scale_grads(const nq_lrb_layer* L, const uint16_t* x, const uint16_t* ybar, int64_t M,
+                                    float* g_s1, float* g_s2, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * nq_silu_mul -- h[e] = bf16( silu(g[e]) * u[e] ), silu(g) = g / (1 + exp(-g)), fp32 math,

@@ -11,11 +11,9 @@ __device__ unsigned int g_error_word = 0u;
 
 // kernels' host launchers (defined next to each kernel)
 nq_status nq_launch_pack(const float*, int64_t, int64_t, int64_t, uint32_t*, int64_t, cudaStream_t);
-nq_status nq_launch_decode(const nq_lrb_layer*, const uint16_t*, uint16_t*, int64_t, void*, cudaStream_t, bool);
 size_t nq_decode_workspace_bytes(int64_t d_in, int64_t r, int64_t M);
 size_t nq_decode_stage2_smem(int64_t r, int64_t M);
 nq_status nq_launch_silu_mul(const uint16_t*, const uint16_t*, uint16_t*, int64_t, cudaStream_t, bool);
-nq_status nq_launch_prefill(const nq_lrb_layer*, const uint16_t*, uint16_t*, int64_t, void*, cudaStream_t, bool);
 size_t nq_prefill_workspace_bytes(const nq_lrb_layer*, int64_t M);
 
 namespace {
@@ -72,6 +70,21 @@ nq_status check_io(const uint16_t* x, const uint16_t* y, void* ws) {
     if (!x || !y || !ws) return NQ_ERR_NULL;
     if (!aligned16(x) || !aligned16(y) || !aligned16(ws)) return NQ_ERR_ALIGN;
     return NQ_OK;
+}
+
+// The layer with the roles of (U, s1, d_out) and (V, s2, d_in) exchanged: its forward product
+// is the transpose of L's, since W_ij = s1_i G_ij s2_j and G_ij = G^T_ji.
+nq_lrb_layer exchanged(const nq_lrb_layer* L) {
+    nq_lrb_layer T = *L;
+    T.d_out = L->d_in;
+    T.d_in = L->d_out;
+    T.U = L->V;
+    T.ldu = L->ldv;
+    T.V = L->U;
+    T.ldv = L->ldu;
+    T.s1 = L->s2;
+    T.s2 = L->s1;
+    return T;
 }
 
 }  // namespace
@@ -167,7 +180,11 @@ nq_status nq_pack_signs(const float* latent, int64_t rows, int64_t r, int64_t ld
 
 size_t nq_workspace_bytes(const nq_lrb_layer* L, int64_t M) {
     if (check_layer(L) != NQ_OK || M < 1) return 0;
+    // one workspace serves the forward product, the transpose and the scale gradients
+    const nq_lrb_layer T = exchanged(L);
     size_t bytes = nq_prefill_workspace_bytes(L, M);
+    const size_t bytes_t = nq_prefill_workspace_bytes(&T, M);
+    if (bytes_t > bytes) bytes = bytes_t;
     if (M <= NQ_MATVEC_MAX_M) {
         const size_t dec = nq_decode_workspace_bytes(L->d_in, L->r, M);
         if (dec > bytes) bytes = dec;
@@ -204,6 +221,47 @@ nq_status nq_layer_forward(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y
                            size_t ws_bytes, void* stream) {
     if (M >= 1 && M <= NQ_MATVEC_MAX_M) return nq_lrb_matvec(L, x, y, M, ws, ws_bytes, stream);
     return nq_lrb_matmul(L, x, y, M, ws, ws_bytes, stream);
+}
+
+nq_status nq_lrb_transposed(const nq_lrb_layer* L, const uint16_t* ybar, uint16_t* xbar, int64_t M, void* ws,
+                            size_t ws_bytes, void* stream) {
+    nq_status st = check_layer(L);
+    if (st != NQ_OK) return st;
+    if (M < 1) return NQ_ERR_SHAPE;
+    if (M <= NQ_MATVEC_MAX_M && nq_decode_stage2_smem(L->r, M) > kMaxDecodeSmem) return NQ_ERR_SHAPE;
+    if ((st = check_io(ybar, xbar, ws)) != NQ_OK) return st;
+    if (ws_bytes < nq_workspace_bytes(L, M)) return NQ_ERR_WORKSPACE;
+    DeviceInfo* d = current_device();
+    if (!d || !d->ok) return NQ_ERR_DEVICE;
+    const nq_lrb_layer T = exchanged(L);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (M <= NQ_MATVEC_MAX_M) return nq_launch_decode(&T, ybar, xbar, M, ws, s, pdl_enabled());
+    return nq_launch_prefill(&T, ybar, xbar, M, ws, s, pdl_enabled());
+}
+
+nq_status nq_lrb_scale_grads(const nq_lrb_layer* L, const uint16_t* x, const uint16_t* ybar, int64_t M, float* g_s1,
+                             float* g_s2, void* ws, size_t ws_bytes, void* stream) {
+    nq_status st = check_layer(L);
+    if (st != NQ_OK) return st;
+    if (M < 1) return NQ_ERR_SHAPE;
+    if (M <= NQ_MATVEC_MAX_M && nq_decode_stage2_smem(L->r, M) > kMaxDecodeSmem) return NQ_ERR_SHAPE;
+    if ((st = check_io(x, ybar, ws)) != NQ_OK) return st;
+    if (!g_s1 || !g_s2) return NQ_ERR_NULL;
+    if (!aligned16(g_s1) || !aligned16(g_s2)) return NQ_ERR_ALIGN;
+    if (ws_bytes < nq_workspace_bytes(L, M)) return NQ_ERR_WORKSPACE;
+    DeviceInfo* d = current_device();
+    if (!d || !d->ok) return NQ_ERR_DEVICE;
+    const nq_lrb_layer T = exchanged(L);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool pdl = pdl_enabled();
+    // dL/ds1 from the layer with cotangent ybar; dL/ds2 from the exchanged layer, whose
+    // intermediate is U^T (s1 . ybar), with cotangent x
+    if (M <= NQ_MATVEC_MAX_M) {
+        if ((st = nq_launch_decode(L, x, nullptr, M, ws, s, pdl, ybar, g_s1)) != NQ_OK) return st;
+        return nq_launch_decode(&T, ybar, nullptr, M, ws, s, pdl, x, g_s2);
+    }
+    if ((st = nq_launch_prefill(L, x, nullptr, M, ws, s, pdl, ybar, g_s1)) != NQ_OK) return st;
+    return nq_launch_prefill(&T, ybar, nullptr, M, ws, s, pdl, x, g_s2);
 }
 
 nq_status nq_silu_mul(const uint16_t* g, const uint16_t* u, uint16_t* h, int64_t n, void* stream) {

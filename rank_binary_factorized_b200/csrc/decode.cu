@@ -486,6 +486,10 @@ struct S2Params {
     int mt_total;        // 16-row M-tiles of U
     int chunk_mt;        // M-tiles staged in shared memory at a time
     int tstage;          // t (M x r fp32) is copied into shared memory for the table build
+    // gradient mode (grad != nullptr): instead of y, grad[i] = sum_m cot[m][i] (U t_m)_i, the
+    // derivative of sum_m <cot_m, y_m> with respect to s1_i; cot [M][d_out] bf16, grad fp32
+    const uint16_t* cot;
+    float* grad;
 };
 
 // B table layout: the two B-fragment words of lane (gid, tig) for bit offset s, word group g
@@ -721,7 +725,26 @@ __global__ void __launch_bounds__(TH, 1) decode_stage2_kernel(const S2Params p) 
         __syncthreads();
 
         // epilogue: y = s1 * 2^-shift * (2 P - Tsum), P = d0 + 2^8 d1 + 2^16 d2
-        for (int e = tid; e < nmt * 16 * p.M; e += kS2Threads) {
+        if (p.grad) {
+            // (U t_m)_i = 2^-shift (2 P - Tsum), weighted by the cotangent and summed over m in
+            // order, in fp64
+            for (int row = tid; row < nmt * 16; row += kS2Threads) {
+                const int64_t i = static_cast<int64_t>(c0) * 16 + row;
+                if (i < p.d_out) {
+                    double g = 0.0;
+                    for (int m = 0; m < p.M; ++m) {
+                        const int* rr = red + row * (NT * 8) + 3 * m;
+                        const long long P = static_cast<long long>(rr[0]) + (static_cast<long long>(rr[1]) << 8) +
+                                            (static_cast<long long>(rr[2]) << 16);
+                        const long long val = 2 * P - static_cast<long long>(s_tsum[m]);
+                        g += static_cast<double>(bf16_bits_to_float(p.cot[static_cast<int64_t>(m) * p.d_out + i])) *
+                             (static_cast<double>(val) * s_dinv[m]);
+                    }
+                    p.grad[i] = static_cast<float>(g);
+                }
+            }
+        }
+        for (int e = tid; e < (p.grad ? 0 : nmt * 16 * p.M); e += kS2Threads) {
             const int row = (p.M == 1) ? e : e / p.M, m = e - row * p.M;
             const int64_t i = static_cast<int64_t>(c0) * 16 + row;
             if (i < p.d_out) {
@@ -800,6 +823,7 @@ void set_attrs_once() {
 
 template <int NT>
 nq_status launch_decode_nt(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y, int M, void* ws,
+                           const uint16_t* cot, float* grad,
                            cudaStream_t stream, bool pdl) {
     float* t = reinterpret_cast<float*>(static_cast<char*>(ws) + kWsHeader);
     {
@@ -837,6 +861,8 @@ nq_status launch_decode_nt(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y
         q.s1 = L->s1;
         q.t = t;
         q.y = y;
+        q.cot = cot;
+        q.grad = grad;
         q.M = M;
         q.d_out = L->d_out;
         q.r = static_cast<int>(L->r);
@@ -888,11 +914,11 @@ size_t nq_decode_stage2_smem(int64_t r, int64_t M) {
 }
 
 nq_status nq_launch_decode(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y, int64_t M, void* ws,
-                           cudaStream_t stream, bool pdl) {
+                           cudaStream_t stream, bool pdl, const uint16_t* cot, float* grad) {
     const int m = static_cast<int>(M);
     switch (ntiles_for(M)) {
-        case 1: return launch_decode_nt<1>(L, x, y, m, ws, stream, pdl);
-        case 2: return launch_decode_nt<2>(L, x, y, m, ws, stream, pdl);
-        default: return launch_decode_nt<3>(L, x, y, m, ws, stream, pdl);
+        case 1: return launch_decode_nt<1>(L, x, y, m, ws, cot, grad, stream, pdl);
+        case 2: return launch_decode_nt<2>(L, x, y, m, ws, cot, grad, stream, pdl);
+        default: return launch_decode_nt<3>(L, x, y, m, ws, cot, grad, stream, pdl);
     }
 }

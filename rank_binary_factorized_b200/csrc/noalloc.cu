@@ -16,7 +16,6 @@
 // the library holds this many bytes until the process exits.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[NQ_NOALLOC_SCRATCH_BYTES];
 
-nq_status nq_launch_decode(const nq_lrb_layer*, const uint16_t*, uint16_t*, int64_t, void*, cudaStream_t, bool);
 size_t nq_decode_workspace_bytes(int64_t d_in, int64_t r, int64_t M);
 size_t nq_decode_stage2_smem(int64_t r, int64_t M);
 

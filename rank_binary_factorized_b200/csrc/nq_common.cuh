@@ -64,3 +64,13 @@ cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem, cudaS
 cudaError_t launch_ex(const void* fn, dim3 grid, dim3 block, size_t smem, cudaStream_t s, void** args, bool pdl,
                       int cluster_y);
 }  // namespace nq_host
+
+// Decode path (decode.cu): y = layer(x) for M <= NQ_MATVEC_MAX_M; with grad != nullptr it
+// writes grad[i] = sum_m cot[m][i] (U t_m)_i (the s1-gradient of sum_m <cot_m, y_m>) instead
+// of y.
+nq_status nq_launch_decode(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y, int64_t M, void* ws,
+                           cudaStream_t stream, bool pdl, const uint16_t* cot = nullptr, float* grad = nullptr);
+// Prefill path (prefill.cu): Y = layer(x) on the tensor cores; with grad != nullptr it writes
+// grad[i] = sum_m cot[m][i] (T U^T)[m][i] instead of Y.
+nq_status nq_launch_prefill(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y, int64_t M, void* ws,
+                            cudaStream_t stream, bool pdl, const uint16_t* cot = nullptr, float* grad = nullptr);

@@ -61,6 +61,11 @@ struct PrefillArgs {
     const uint16_t* s1;    // mode U
     unsigned int* err;
     int bits_tma;          // packed signs arrive by TMA (row stride a multiple of 16 bytes)
+    // gradient mode (mode U, gpart != nullptr): no Y; for every token tile tn and row w,
+    // gpart[tn][w] = sum over the tile's tokens of cot[tok][w] * (T U^T)[tok][w] (fp64)
+    const uint16_t* cot;   // [M][ldcot] bf16
+    int64_t ldcot;
+    double* gpart;         // [n_tiles_n][rows_w]
 };
 
 // fp16 +1 = 0x3C00, -1 = 0xBC00; two elements per 32-bit word, element 2i in the low half.
@@ -363,6 +368,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             const bool row_ok = wrow < args.rows_w;
             float scale = 1.0f;
             if (MODE == kModeU && row_ok) scale = f16_bits_to_float(args.s1[wrow]);
+            const bool grad = (MODE == kModeU) && args.gpart != nullptr;
+            double g = 0.0;
             for (int c0 = 0; c0 < tile_n; c0 += 32) {
                 uint32_t v[32];
                 tc::tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * 256 + c0, v);
@@ -373,7 +380,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                         const int64_t tok = static_cast<int64_t>(tn) * tile_n + c0 + j;
                         if (c0 + j < tile_n && tok < args.M) {
                             const float f = __uint_as_float(v[j]);
-                            if (MODE == kModeU) {
+                            if (grad) {
+                                g += static_cast<double>(bf16_bits_to_float(args.cot[tok * args.ldcot + wrow])) * f;
+                            } else if (MODE == kModeU) {
                                 static_cast<uint16_t*>(args.out)[tok * args.ldo + wrow] = float_to_bf16_bits(scale * f);
                             } else {
                                 static_cast<uint16_t*>(args.out)[tok * args.ldo + wrow] =
@@ -383,6 +392,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     }
                 }
             }
+            if (grad && row_ok) args.gpart[static_cast<int64_t>(tn) * args.rows_w + wrow] = g;
             tc::tc_fence_before();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(acc_empty(acc));
@@ -433,6 +443,18 @@ __global__ void __launch_bounds__(256) scale_convert_kernel(const uint16_t* __re
     }
 }
 
+// grad[i] = sum over token tiles tn (in order) of gpart[tn][i], fp64, rounded to fp32.
+__global__ void __launch_bounds__(256) grad_reduce_kernel(const double* __restrict__ gpart, int64_t n_tiles,
+                                                         int64_t rows, float* __restrict__ grad) {
+    pdl_wait();
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < rows;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        double g = 0.0;
+        for (int64_t tn = 0; tn < n_tiles; ++tn) g += gpart[tn * rows + i];
+        grad[i] = static_cast<float>(g);
+    }
+}
+
 }  // namespace nq
 
 // ------------------------------------------------------------------------------ host side
@@ -443,7 +465,8 @@ int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
 
 struct PrefillPlan {
     int64_t ldz, ldt;
-    size_t off_z, off_t, total;
+    int tile_n1, tile_n2;  // token tiles of GEMM 1 and GEMM 2
+    size_t off_z, off_t, off_g, total;
 };
 
 // Tokens per tile (MMA N, a multiple of 16 up to 256) for a GEMM with n_tiles_w weight tiles:
@@ -468,11 +491,17 @@ int choose_tile_n(int64_t n_tiles_w, int64_t M, int sms) {
 
 PrefillPlan plan_prefill(const nq_lrb_layer* L, int64_t M) {
     PrefillPlan p{};
+    const int sms = nq_host::sm_count();
+    p.tile_n1 = choose_tile_n((L->r + nq::kTileW - 1) / nq::kTileW, M, sms);
+    p.tile_n2 = choose_tile_n((L->d_out + nq::kTileW - 1) / nq::kTileW, M, sms);
     p.ldz = round_up(L->d_in, 8);  // 16-byte aligned rows for TMA
     p.ldt = round_up(L->r, 8);
     p.off_z = NQ_WS_HEADER_BYTES;  // past the reserved workspace header
     p.off_t = p.off_z + align256(static_cast<size_t>(M * p.ldz) * 2);
-    p.total = p.off_t + align256(static_cast<size_t>(M * p.ldt) * 2);
+    p.off_g = p.off_t + align256(static_cast<size_t>(M * p.ldt) * 2);
+    // gradient mode: fp64 partial per (token tile of GEMM 2, row)
+    const int64_t n_tn2 = (M + p.tile_n2 - 1) / p.tile_n2;
+    p.total = p.off_g + align256(static_cast<size_t>(n_tn2 * L->d_out) * sizeof(double));
     return p;
 }
 
@@ -566,7 +595,7 @@ nq_status launch_umma(const nq::PrefillArgs& a, const CUtensorMap& map, const CU
 size_t nq_prefill_workspace_bytes(const nq_lrb_layer* L, int64_t M) { return plan_prefill(L, M).total; }
 
 nq_status nq_launch_prefill(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y, int64_t M, void* ws,
-                            cudaStream_t stream, bool pdl) {
+                            cudaStream_t stream, bool pdl, const uint16_t* cot, float* grad) {
     const PrefillPlan p = plan_prefill(L, M);
     uint16_t* z = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + p.off_z);
     uint16_t* t = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + p.off_t);
@@ -584,7 +613,7 @@ nq_status nq_launch_prefill(const nq_lrb_layer* L, const uint16_t* x, uint16_t* 
             return NQ_ERR_LAUNCH;
     }
     {  // T = fp16(Z V): weights = V^T (M-extent r, K = d_in), B = Z
-        const int tile_n = choose_tile_n((L->r + nq::kTileW - 1) / nq::kTileW, M, nq_host::sm_count());
+        const int tile_n = p.tile_n1;
         CUtensorMap map;
         if (!make_tmap(&map, z, M, L->d_in, p.ldz, tile_n)) return NQ_ERR_LAUNCH;
         nq::PrefillArgs a{};
@@ -609,7 +638,7 @@ nq_status nq_launch_prefill(const nq_lrb_layer* L, const uint16_t* x, uint16_t* 
         if (st != NQ_OK) return st;
     }
     {  // Y = bf16(s1 * (T U^T)): weights = U (M-extent d_out, K = r), B = T
-        const int tile_n = choose_tile_n((L->d_out + nq::kTileW - 1) / nq::kTileW, M, nq_host::sm_count());
+        const int tile_n = p.tile_n2;
         CUtensorMap map;
         if (!make_tmap(&map, t, M, L->r, p.ldt, tile_n)) return NQ_ERR_LAUNCH;
         nq::PrefillArgs a{};
@@ -627,11 +656,26 @@ nq_status nq_launch_prefill(const nq_lrb_layer* L, const uint16_t* x, uint16_t* 
         a.ldo = L->d_out;
         a.s1 = L->s1;
         a.err = err;
+        double* gpart = reinterpret_cast<double*>(static_cast<char*>(ws) + p.off_g);
+        if (grad) {
+            a.out = nullptr;
+            a.cot = cot;
+            a.ldcot = L->d_out;
+            a.gpart = gpart;
+        }
         CUtensorMap bmap;
         std::memset(&bmap, 0, sizeof(bmap));
         a.bits_tma = make_tmap_bits(&bmap, L->U, L->d_out, L->r / 32, L->ldu, nq::kTileW) ? 1 : 0;
         nq_status st = launch_umma<nq::kModeU>(a, map, bmap, stream, pdl);
         if (st != NQ_OK) return st;
+        if (grad) {  // sum the token tiles' partials per row, in order
+            int64_t n_tiles = a.n_tiles_n, rows = L->d_out;
+            const unsigned blocks = static_cast<unsigned>(std::min<int64_t>((rows + 255) / 256, 4LL * nq_host::sm_count()));
+            void* args[] = {&gpart, &n_tiles, &rows, &grad};
+            if (nq_host::launch_pdl(reinterpret_cast<const void*>(nq::grad_reduce_kernel), dim3(blocks), dim3(256), 0,
+                                    stream, args, pdl) != cudaSuccess)
+                return NQ_ERR_LAUNCH;
+        }
     }
     return NQ_OK;
 }

@@ -49,6 +49,10 @@ for _name in ("nq_lrb_matvec", "nq_lrb_matmul", "nq_layer_forward"):
     getattr(_lib, _name).argtypes = [ctypes.POINTER(nq_lrb_layer), _p, _p, _i64, _p, ctypes.c_size_t, _p]
 _lib.nq_silu_mul.restype = ctypes.c_int
 _lib.nq_silu_mul.argtypes = [_p, _p, _p, _i64, _p]
+_lib.nq_lrb_transposed.restype = ctypes.c_int
+_lib.nq_lrb_transposed.argtypes = [ctypes.POINTER(nq_lrb_layer), _p, _p, _i64, _p, ctypes.c_size_t, _p]
+_lib.nq_lrb_scale_grads.restype = ctypes.c_int
+_lib.nq_lrb_scale_grads.argtypes = [ctypes.POINTER(nq_lrb_layer), _p, _p, _i64, _p, _p, _p, ctypes.c_size_t, _p]
 _lib.nq_sync_status.restype = ctypes.c_int
 _lib.nq_sync_status.argtypes = [_p]
 _lib.nq_status_string.restype = ctypes.c_char_p
@@ -175,6 +179,31 @@ def lrb_matmul(layer: Layer, x: torch.Tensor, y=None, ws=None, stream=None) -> t
 
 def layer_forward(layer: Layer, x: torch.Tensor, y=None, ws=None, stream=None) -> torch.Tensor:
     return _forward("nq_layer_forward", layer, x, y, ws, stream)
+
+
+def lrb_transposed(layer: Layer, ybar: torch.Tensor, xbar=None, ws=None, stream=None) -> torch.Tensor:
+    """xbar = the layer's transpose applied to ybar ([M][d_out] bf16 -> [M][d_in] bf16)."""
+    M = int(ybar.shape[0])
+    if xbar is None:
+        xbar = torch.empty((M, layer.d_in), dtype=torch.bfloat16, device=ybar.device)
+    if ws is None:
+        ws = layer.workspace(M)
+    _check("nq_lrb_transposed", _lib.nq_lrb_transposed(ctypes.byref(layer.struct), _ptr(ybar), _ptr(xbar), M,
+                                                       _ptr(ws), ws.numel(), _stream_ptr(stream)))
+    return xbar
+
+
+def lrb_scale_grads(layer: Layer, x: torch.Tensor, ybar: torch.Tensor, ws=None, stream=None):
+    """(dL/ds1 [d_out], dL/ds2 [d_in]) fp32 for L = sum <ybar, layer(x)>."""
+    M = int(x.shape[0])
+    g1 = torch.empty(layer.d_out, dtype=torch.float32, device=x.device)
+    g2 = torch.empty(layer.d_in, dtype=torch.float32, device=x.device)
+    if ws is None:
+        ws = layer.workspace(M)
+    _check("nq_lrb_scale_grads", _lib.nq_lrb_scale_grads(ctypes.byref(layer.struct), _ptr(x), _ptr(ybar), M,
+                                                         _ptr(g1), _ptr(g2), _ptr(ws), ws.numel(),
+                                                         _stream_ptr(stream)))
+    return g1, g2
 
 
 def silu_mul(g: torch.Tensor, u: torch.Tensor, h=None, stream=None) -> torch.Tensor:

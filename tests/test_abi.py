@@ -60,7 +60,7 @@ def _call(nq, fn, L, x=0x50000, y=0x60000, M=1, ws=0x70000, ws_bytes=1 << 30):
     return getattr(lib, fn)(ctypes.byref(L) if L is not None else None, x, y, M, ws, ws_bytes, None)
 
 
-@pytest.mark.parametrize("fn", ["nq_lrb_matvec", "nq_lrb_matmul", "nq_layer_forward"])
+@pytest.mark.parametrize("fn", ["nq_lrb_matvec", "nq_lrb_matmul", "nq_layer_forward", "nq_lrb_transposed"])
 def test_forward_argument_errors(nq, fn):
     assert _call(nq, fn, None) == NQ["NULL"]
     assert _call(nq, fn, _layer(nq, U=0)) == NQ["NULL"]
@@ -77,6 +77,35 @@ def test_forward_argument_errors(nq, fn):
     assert _call(nq, fn, _layer(nq, V=0x20004)) == NQ["ALIGN"]
     assert _call(nq, fn, _layer(nq), x=0x50002) == NQ["ALIGN"]
     assert _call(nq, fn, _layer(nq), ws_bytes=16) == NQ["WORKSPACE"]
+
+
+def test_scale_grads_argument_errors(nq):
+    lib = nq.raw_lib()
+
+    def call(L, x=0x50000, ybar=0x60000, M=1, g1=0x80000, g2=0x90000, ws=0x70000, ws_bytes=1 << 30):
+        return lib.nq_lrb_scale_grads(ctypes.byref(L) if L is not None else None, x, ybar, M, g1, g2, ws, ws_bytes,
+                                      None)
+
+    assert call(None) == NQ["NULL"]
+    assert call(_layer(nq, V=0)) == NQ["NULL"]
+    assert call(_layer(nq), ybar=0) == NQ["NULL"]
+    assert call(_layer(nq), g1=0) == NQ["NULL"]
+    assert call(_layer(nq), g2=0) == NQ["NULL"]
+    assert call(_layer(nq, r=48)) == NQ["SHAPE"]
+    assert call(_layer(nq), M=0) == NQ["SHAPE"]
+    assert call(_layer(nq), g2=0x90004) == NQ["ALIGN"]
+    assert call(_layer(nq), x=0x50008) == NQ["ALIGN"]
+    assert call(_layer(nq), ws_bytes=16) == NQ["WORKSPACE"]
+
+
+def test_workspace_covers_both_directions(nq):
+    """One workspace serves the forward product, the transpose and the scale gradients: the
+    size is the same for a layer and for the layer with its two sides exchanged."""
+    lib = nq.raw_lib()
+    for M in (1, 8, 64, 2048):
+        a = lib.nq_workspace_bytes(ctypes.byref(_layer(nq, d_out=28672, d_in=8192, r=3520)), M)
+        b = lib.nq_workspace_bytes(ctypes.byref(_layer(nq, d_out=8192, d_in=28672, r=3520)), M)
+        assert a == b > 0
 
 
 def test_matvec_rejects_large_batch(nq):
