@@ -47,7 +47,8 @@ def parse_args():
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--headline-only", action="store_true", help="skip the other workloads")
     ap.add_argument("--only", default=None,
-                    help="run just these extra sections (comma list of attn7b_b8, mlp7b, layer70b, prefill, pack) "
+                    help="run just these extra sections (comma list of attn7b_b8, mlp7b, layer70b, prefill, pack, "
+                         "calib) "
                          "after the headline; implies no CPU baseline")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU oracle sample budget")
     return ap.parse_args()
@@ -359,6 +360,8 @@ def extras(torch, nq, stream, args, hbm_gbs, bf16_tf, bf16_tf_sus, peak_src):
         out["prefill70b_gate"] = _extra_prefill(torch, nq, stream, steps, bf16_tf)
     if on("pack"):
         out["pack_70b_gate_U"] = _extra_pack(torch, nq, stream, steps, warm, hbm_gbs)
+    if on("calib"):
+        out.update(_extra_calib(torch, nq, stream, steps, warm, hbm_gbs, bf16_tf))
     nq.sync_status(stream)
     return out
 
@@ -438,6 +441,50 @@ def _extra_prefill(torch, nq, stream, steps, bf16_tf):
                           "frac_bf16": round(flops / us / 1e6 / bf16_tf, 4)}
         del g
     return pre
+
+
+def _extra_calib(torch, nq, stream, steps, warm, hbm_gbs, bf16_tf):
+    """Scale-only calibration products: the layer transpose at decode batch 1 and the two
+    scale gradients at batch 8 (7B attention shape, distinct instances > 3x L2), and the
+    scale gradients of the 70B gate at M = 2048 on the tensor cores."""
+    out = {}
+    (_, do, di, r), = synth.WORKLOADS[HEADLINE]
+    for (key, M) in (("transposed_attn7b_b1", 1), ("scale_grads_attn7b_b8", 8)):
+        lb = decode_bytes(do, di, r, M)
+        ch = Chain(torch, nq, do, di, r, M, n_instances(lb), seed=synth.workload_seed(HEADLINE) + 70 + M)
+        ybar = torch.zeros((M, do), dtype=torch.bfloat16, device="cuda").normal_()
+        xbar = torch.empty((M, di), dtype=torch.bfloat16, device="cuda")
+        if M == 1:
+            def run():
+                for L in ch.layers:
+                    nq.lrb_transposed(L, ybar, xbar, ws=ch.ws, stream=stream)
+        else:
+            def run():
+                for L in ch.layers:
+                    nq.lrb_scale_grads(L, ch.x0, ybar, ws=ch.ws, stream=stream)
+        g = graph_of(torch, run, stream)
+        ms = timed_replays(torch, g, stream, steps, warm)
+        us = ms * 1e3 / (steps * ch.n)
+        moved = lb if M == 1 else 2 * lb  # the gradients read every weight twice (two passes)
+        out[key] = {"us_per_layer": round(us, 3), "GB_s": round(moved / us / 1e3, 1),
+                    "frac_hbm": round(moved / us / 1e3 / hbm_gbs, 4),
+                    "l2": "no flush: %d distinct layers > 3x L2" % ch.n}
+        del g, ch
+    (_, do, di, r), = synth.WORKLOADS["prefill70b"]
+    p = synth.make_projection("gate", do, di, r, seed=synth.workload_seed("prefill70b"))
+    L = nq.Layer.from_host(p.U, p.V, p.s1, p.s2, r)
+    M = 2048
+    x = torch.zeros((M, di), dtype=torch.bfloat16, device="cuda").normal_()
+    ybar = torch.zeros((M, do), dtype=torch.bfloat16, device="cuda").normal_()
+    ws = L.workspace(M)
+    g = graph_of(torch, lambda: nq.lrb_scale_grads(L, x, ybar, ws=ws, stream=stream), stream)
+    ms = timed_replays(torch, g, stream, 3, 2)
+    us = ms * 1e3 / 3
+    flops = 2 * 2.0 * M * r * (di + do)  # two passes of the two products
+    out["scale_grads_prefill70b_gate_M2048"] = {"us": round(us, 2), "TFLOP_s": round(flops / us / 1e6, 2),
+                                                "frac_bf16": round(flops / us / 1e6 / bf16_tf, 4)}
+    del g
+    return out
 
 
 def _extra_pack(torch, nq, stream, steps, warm, hbm_gbs):
