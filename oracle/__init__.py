@@ -83,6 +83,11 @@ def lib() -> ctypes.CDLL:
         L.nq_oracle_scale_grads_packed.restype = ctypes.c_int
         L.nq_oracle_scale_grads_packed.argtypes = [_p, _i64, _p, _i64, _p, _p, _i64, _i64, _i64, _p, _p, _i64,
                                                    _p, _p, _p, _p]
+        L.nq_oracle_double_to_f16.restype = ctypes.c_uint16
+        L.nq_oracle_double_to_f16.argtypes = [ctypes.c_double]
+        L.nq_oracle_from_latent.restype = ctypes.c_int
+        L.nq_oracle_from_latent.argtypes = [_p, _i64, _p, _i64, _i64, _i64, _i64, _p, _i64, _p, _i64, _p, _p, _p,
+                                            _p, _p]
         L.nq_oracle_silu_mul.restype = None
         L.nq_oracle_silu_mul.argtypes = [_p, _p, _i64, _p]
         L.nq_oracle_round_bf16.restype = None
@@ -263,6 +268,35 @@ def scale_grads_packed(Uw, Vw, s1_f16, s2_f16, r: int, x_bf16, ybar_bf16):
     if rc != 0:
         raise ValueError("nq_oracle_scale_grads_packed failed (%d)" % rc)
     return g1, S1, g2, S2
+
+
+def double_to_f16(values) -> np.ndarray:
+    """fp64 values -> fp16 bit patterns (round to nearest, ties to even)."""
+    v = np.asarray(values, dtype=np.float64).ravel()
+    return np.array([lib().nq_oracle_double_to_f16(float(a)) for a in v], dtype=np.uint16).reshape(np.shape(values))
+
+
+def from_latent(Uh, Vh, ldu=None, ldv=None):
+    """Balance the latent proxies (eta), extract the mean-absolute-value scales and pack the
+    signs.  Returns (U words, V words, s1 fp16 bits, s2 fp16 bits, eta, s1 fp64, s2 fp64)."""
+    Uh = _c(Uh, np.float32)
+    Vh = _c(Vh, np.float32)
+    d_out, r = Uh.shape
+    d_in = Vh.shape[0]
+    ldu = r // 32 if ldu is None else ldu
+    ldv = r // 32 if ldv is None else ldv
+    U = np.zeros((d_out, ldu), dtype=np.uint32)
+    V = np.zeros((d_in, ldv), dtype=np.uint32)
+    s1 = np.zeros(d_out, dtype=np.uint16)
+    s2 = np.zeros(d_in, dtype=np.uint16)
+    eta = np.zeros(1)
+    s1d = np.zeros(d_out)
+    s2d = np.zeros(d_in)
+    rc = lib().nq_oracle_from_latent(_ptr(Uh), r, _ptr(Vh), r, d_out, d_in, r, _ptr(U), ldu, _ptr(V), ldv, _ptr(s1),
+                                     _ptr(s2), _ptr(eta), _ptr(s1d), _ptr(s2d))
+    if rc != 0:
+        raise ValueError("nq_oracle_from_latent failed (%d)" % rc)
+    return U, V, s1, s2, float(eta[0]), s1d, s2d
 
 
 def factored_packed(Uw, Vw, s1_f16, s2_f16, r: int, x_bf16) -> np.ndarray:

@@ -77,6 +77,29 @@ ORACLE_API double nq_oracle_bf16_to_double(uint16_t b) {
 /* fp64 -> bfloat16, round to nearest, ties to even, directly from the real value (no
  * intermediate binary32 rounding).  bfloat16 keeps 8 significant bits; its smallest normal
  * is 2^-126 and its quantum below that is 2^-133. */
+/* fp64 -> IEEE binary16 (1 sign, 5 exponent bits with bias 15, 10 fraction bits), round to
+ * nearest, ties to even: keep 11 significant bits (quantum 2^(e-11) for a in [2^(e-1), 2^e)),
+ * never finer than the subnormal quantum 2^-24; results of 65536 and above overflow to inf. */
+ORACLE_API uint16_t nq_oracle_double_to_f16(double v) {
+    if (isnan(v)) return 0x7E00;
+    uint16_t sign = signbit(v) ? 0x8000 : 0;
+    double a = fabs(v);
+    if (isinf(a)) return sign | 0x7C00;
+    if (a == 0.0) return sign;
+    int e;
+    frexp(a, &e); /* a = m * 2^e, 0.5 <= m < 1 */
+    int qexp = e - 11;
+    if (qexp < -24) qexp = -24;
+    double q = nearbyint(ldexp(a, -qexp)); /* default rounding mode: to nearest, ties even */
+    double rv = ldexp(q, qexp);
+    if (rv >= 65536.0) return sign | 0x7C00;
+    if (rv < ldexp(1.0, -14)) return sign | (uint16_t)ldexp(rv, 24); /* subnormal (1024 -> 0x0400) */
+    int e2;
+    double m2 = frexp(rv, &e2); /* rv = m2 * 2^e2, 0.5 <= m2 < 1: exponent field e2 - 1 + 15 */
+    uint16_t frac = (uint16_t)(ldexp(m2, 11) - 1024.0);
+    return sign | (uint16_t)((e2 + 14) << 10) | frac;
+}
+
 ORACLE_API uint16_t nq_oracle_double_to_bf16(double v) {
     if (isnan(v)) return 0x7FC0;
     uint16_t sign = signbit(v) ? 0x8000 : 0;
@@ -366,6 +389,56 @@ ORACLE_API int nq_oracle_scale_grads_packed(const uint32_t* U, int64_t ldu, cons
     }
     free(x);
     free(yb);
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------------
+ * From latent factors to a packed layer (section 3, "Step 2", "Magnitude Balancing and Scale
+ * Extraction", then "Phase 3" packing): for the continuous proxies Uh [d_out][r] and
+ * Vh [d_in][r],
+ *     eta = sqrt( ||Vh||_F / ||Uh||_F ),   U := eta Uh,   V := Vh / eta,
+ *     s1_i = mean over k of |U_ik|,        s2_j = mean over k of |V_jk|,
+ * and the binary factors are sign(U), sign(V), packed as nq_oracle_pack does.  Readings:
+ * the mean runs over the r entries of a row; eta = 1 when either norm is zero; s1, s2 are
+ * stored as fp16 (round to nearest even).  Outputs: packed U, V; s1, s2 as fp16 bits and,
+ * when the pointers are not NULL, eta and the fp64 scales before rounding.
+ * --------------------------------------------------------------------------------- */
+ORACLE_API int nq_oracle_from_latent(const float* Uh, int64_t ld_uh, const float* Vh, int64_t ld_vh, int64_t d_out,
+                                     int64_t d_in, int64_t r, uint32_t* U, int64_t ldu, uint32_t* V, int64_t ldv,
+                                     uint16_t* s1_f16, uint16_t* s2_f16, double* eta_out, double* s1_out,
+                                     double* s2_out) {
+    if (d_out < 0 || d_in < 0 || r <= 0 || r % 32 != 0 || ld_uh < r || ld_vh < r || ldu < r / 32 || ldv < r / 32)
+        return -1;
+    double su = 0.0, sv = 0.0;
+    for (int64_t i = 0; i < d_out; ++i)
+        for (int64_t k = 0; k < r; ++k) su += (double)Uh[i * ld_uh + k] * (double)Uh[i * ld_uh + k];
+    for (int64_t j = 0; j < d_in; ++j)
+        for (int64_t k = 0; k < r; ++k) sv += (double)Vh[j * ld_vh + k] * (double)Vh[j * ld_vh + k];
+    const double nu = sqrt(su), nv = sqrt(sv);
+    const double eta = (nu > 0.0 && nv > 0.0) ? sqrt(nv / nu) : 1.0;
+    if (eta_out) *eta_out = eta;
+    for (int64_t i = 0; i < d_out; ++i) {
+        double acc = 0.0;
+        for (int64_t w = 0; w < ldu; ++w) U[i * ldu + w] = 0u;
+        for (int64_t k = 0; k < r; ++k) {
+            double b = eta * (double)Uh[i * ld_uh + k];
+            acc += fabs(b);
+            if (b >= 0.0) U[i * ldu + k / 32] |= 1u << (k % 32);
+        }
+        if (s1_out) s1_out[i] = acc / (double)r;
+        s1_f16[i] = nq_oracle_double_to_f16(acc / (double)r);
+    }
+    for (int64_t j = 0; j < d_in; ++j) {
+        double acc = 0.0;
+        for (int64_t w = 0; w < ldv; ++w) V[j * ldv + w] = 0u;
+        for (int64_t k = 0; k < r; ++k) {
+            double b = (double)Vh[j * ld_vh + k] / eta;
+            acc += fabs(b);
+            if (b >= 0.0) V[j * ldv + k / 32] |= 1u << (k % 32);
+        }
+        if (s2_out) s2_out[j] = acc / (double)r;
+        s2_f16[j] = nq_oracle_double_to_f16(acc / (double)r);
+    }
     return 0;
 }
 

@@ -48,6 +48,20 @@ MUTATIONS += [
     ("double t2 = x[b * d_in + j] * g * s1 * yb[b * d_out + i];",
      "double t2 = x[b * d_in + j] * g * s2 * yb[b * d_out + i];", CAL),
 ]
+CONV = "test_oracle_converter.py"
+MUTATIONS += [
+    # balancing with the norm ratio inverted
+    ("const double eta = (nu > 0.0 && nv > 0.0) ? sqrt(nv / nu) : 1.0;",
+     "const double eta = (nu > 0.0 && nv > 0.0) ? sqrt(nu / nv) : 1.0;", CONV),
+    # mean of the signed values instead of their magnitudes
+    ("            acc += fabs(b);\n            if (b >= 0.0) U", "            acc += b;\n            if (b >= 0.0) U", CONV),
+    # the mean divided by the row count instead of the row length
+    ("if (s1_out) s1_out[i] = acc / (double)r;\n        s1_f16[i] = nq_oracle_double_to_f16(acc / (double)r);",
+     "if (s1_out) s1_out[i] = acc / (double)d_out;\n        s1_f16[i] = nq_oracle_double_to_f16(acc / (double)d_out);",
+     CONV),
+    # fp16 encoder with the exponent field one too large
+    ("return sign | (uint16_t)((e2 + 14) << 10) | frac;", "return sign | (uint16_t)((e2 + 15) << 10) | frac;", CONV),
+]
 MUTATIONS = [m if len(m) == 3 else (m[0], m[1], "test_oracle.py") for m in MUTATIONS]
 
 
