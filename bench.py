@@ -484,6 +484,16 @@ def _extra_calib(torch, nq, stream, steps, warm, hbm_gbs, bf16_tf):
     out["scale_grads_prefill70b_gate_M2048"] = {"us": round(us, 2), "TFLOP_s": round(flops / us / 1e6, 2),
                                                 "frac_bf16": round(flops / us / 1e6 / bf16_tf, 4)}
     del g
+    # latent factors -> packed layer (balancing, scales, signs) for the 70B gate projection
+    Uh = torch.randn((do, r), dtype=torch.float32, device="cuda")
+    Vh = torch.randn((di, r), dtype=torch.float32, device="cuda")
+    g = graph_of(torch, lambda: nq.lrb_from_latent(Uh, Vh, stream=stream), stream)
+    ms = timed_replays(torch, g, stream, steps, warm)
+    us = ms * 1e3 / steps
+    moved = 4 * (do + di) * r + (do + di) * r // 8 + 2 * (do + di)  # fp32 in, bits and fp16 scales out
+    out["from_latent_70b_gate"] = {"us": round(us, 2), "GB_s": round(moved / us / 1e3, 1),
+                                   "frac_hbm": round(moved / us / 1e3 / hbm_gbs, 4)}
+    del g
     return out
 
 

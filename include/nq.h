@@ -138,6 +138,25 @@ NQ_API nq_status nq_layer_forward(const nq_lrb_layer* L, const uint16_t* x, uint
                            size_t ws_bytes, void* stream);
 
 /*
+ * nq_lrb_from_latent -- a packed layer from its latent factors.  Page "NanoQuant: Efficient
+ * Sub-1-Bit Quantization of Large Language Models", section 3, "Magnitude Balancing and Scale
+ * Extraction", then "Phase 3" packing.  For the continuous proxies Uh [d_out][ld_uh] and
+ * Vh [d_in][ld_vh] (fp32, r columns each):
+ *     eta = sqrt( ||Vh||_F / ||Uh||_F )   (1 when either norm is 0),
+ *     U := eta Uh,  V := Vh / eta,  s1_i = mean_k |U_ik|,  s2_j = mean_k |V_jk|,
+ * and the binary factors sign(U), sign(V) packed as nq_pack_signs does (eta > 0, so the signs
+ * are those of Uh, Vh).  Outputs (device, caller-owned): U [d_out][ldu], V [d_in][ldv] words,
+ * s1 [d_out], s2 [d_in] fp16 bit patterns (round to nearest even), and eta (one double; may be
+ * NULL).  Norms and means are summed in fp64 in a fixed order (run-to-run identical).
+ * ws: nq_from_latent_workspace_bytes(d_out, d_in, r, ldu, ldv) bytes.
+ */
+NQ_API size_t nq_from_latent_workspace_bytes(int64_t d_out, int64_t d_in, int64_t r, int64_t ldu, int64_t ldv);
+NQ_API nq_status nq_lrb_from_latent(const float* Uh, int64_t ld_uh, const float* Vh, int64_t ld_vh, int64_t d_out,
+                                    int64_t d_in, int64_t r, uint32_t* U, int64_t ldu, uint32_t* V, int64_t ldv,
+                                    uint16_t* s1, uint16_t* s2, double* eta, void* ws, size_t ws_bytes,
+                                    void* stream);
+
+/*
  * Calibration products.  Page "NanoQuant: Efficient Sub-1-Bit Quantization of Large Language
  * Models", section 3, "Phase 3: Scale-Only Model Reconstruction": with U and V frozen and
  * packed, only s1 and s2 are optimised, so a training step needs the layer's transpose (to

@@ -15,6 +15,10 @@ size_t nq_decode_workspace_bytes(int64_t d_in, int64_t r, int64_t M);
 size_t nq_decode_stage2_smem(int64_t r, int64_t M);
 nq_status nq_launch_silu_mul(const uint16_t*, const uint16_t*, uint16_t*, int64_t, cudaStream_t, bool);
 size_t nq_prefill_workspace_bytes(const nq_lrb_layer*, int64_t M);
+size_t nq_from_latent_ws(int64_t d_out, int64_t d_in, int64_t ldu, int64_t ldv);
+nq_status nq_launch_from_latent(const float* Uh, int64_t ld_uh, const float* Vh, int64_t ld_vh, int64_t d_out,
+                                int64_t d_in, int64_t r, uint32_t* U, int64_t ldu, uint32_t* V, int64_t ldv,
+                                uint16_t* s1, uint16_t* s2, double* eta, void* ws, cudaStream_t stream);
 
 namespace {
 
@@ -262,6 +266,27 @@ nq_status nq_lrb_scale_grads(const nq_lrb_layer* L, const uint16_t* x, const uin
     }
     if ((st = nq_launch_prefill(L, x, nullptr, M, ws, s, pdl, ybar, g_s1)) != NQ_OK) return st;
     return nq_launch_prefill(&T, ybar, nullptr, M, ws, s, pdl, x, g_s2);
+}
+
+size_t nq_from_latent_workspace_bytes(int64_t d_out, int64_t d_in, int64_t r, int64_t ldu, int64_t ldv) {
+    if (d_out < 1 || d_in < 1 || r < 32 || (r % 32) != 0 || r > NQ_MAX_RANK || ldu < r / 32 || ldv < r / 32) return 0;
+    return nq_from_latent_ws(d_out, d_in, ldu, ldv);
+}
+
+nq_status nq_lrb_from_latent(const float* Uh, int64_t ld_uh, const float* Vh, int64_t ld_vh, int64_t d_out,
+                             int64_t d_in, int64_t r, uint32_t* U, int64_t ldu, uint32_t* V, int64_t ldv,
+                             uint16_t* s1, uint16_t* s2, double* eta, void* ws, size_t ws_bytes, void* stream) {
+    if (d_out < 1 || d_in < 1 || r < 32 || (r % 32) != 0 || r > NQ_MAX_RANK) return NQ_ERR_SHAPE;
+    if (ld_uh < r || ld_vh < r || ldu < r / 32 || ldv < r / 32) return NQ_ERR_SHAPE;
+    if (!Uh || !Vh || !U || !V || !s1 || !s2 || !ws) return NQ_ERR_NULL;
+    if (!aligned16(Uh) || !aligned16(Vh) || !aligned16(U) || !aligned16(V) || !aligned16(s1) || !aligned16(s2) ||
+        !aligned16(ws) || (eta && (reinterpret_cast<uintptr_t>(eta) & 7u) != 0))
+        return NQ_ERR_ALIGN;
+    if (ws_bytes < nq_from_latent_ws(d_out, d_in, ldu, ldv)) return NQ_ERR_WORKSPACE;
+    DeviceInfo* d = current_device();
+    if (!d || !d->ok) return NQ_ERR_DEVICE;
+    return nq_launch_from_latent(Uh, ld_uh, Vh, ld_vh, d_out, d_in, r, U, ldu, V, ldv, s1, s2, eta, ws,
+                                 static_cast<cudaStream_t>(stream));
 }
 
 nq_status nq_silu_mul(const uint16_t* g, const uint16_t* u, uint16_t* h, int64_t n, void* stream) {

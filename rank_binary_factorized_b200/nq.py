@@ -51,6 +51,11 @@ _lib.nq_silu_mul.restype = ctypes.c_int
 _lib.nq_silu_mul.argtypes = [_p, _p, _p, _i64, _p]
 _lib.nq_lrb_transposed.restype = ctypes.c_int
 _lib.nq_lrb_transposed.argtypes = [ctypes.POINTER(nq_lrb_layer), _p, _p, _i64, _p, ctypes.c_size_t, _p]
+_lib.nq_from_latent_workspace_bytes.restype = ctypes.c_size_t
+_lib.nq_from_latent_workspace_bytes.argtypes = [_i64, _i64, _i64, _i64, _i64]
+_lib.nq_lrb_from_latent.restype = ctypes.c_int
+_lib.nq_lrb_from_latent.argtypes = [_p, _i64, _p, _i64, _i64, _i64, _i64, _p, _i64, _p, _i64, _p, _p, _p, _p,
+                                    ctypes.c_size_t, _p]
 _lib.nq_lrb_scale_grads.restype = ctypes.c_int
 _lib.nq_lrb_scale_grads.argtypes = [ctypes.POINTER(nq_lrb_layer), _p, _p, _i64, _p, _p, _p, ctypes.c_size_t, _p]
 _lib.nq_sync_status.restype = ctypes.c_int
@@ -204,6 +209,31 @@ def lrb_scale_grads(layer: Layer, x: torch.Tensor, ybar: torch.Tensor, ws=None, 
                                                          _ptr(g1), _ptr(g2), _ptr(ws), ws.numel(),
                                                          _stream_ptr(stream)))
     return g1, g2
+
+
+def lrb_from_latent(Uh: torch.Tensor, Vh: torch.Tensor, r: int | None = None, ld_align_words: int = 4,
+                    stream=None):
+    """A device Layer from fp32 latent proxies Uh [d_out][r], Vh [d_in][r]: magnitude balancing,
+    mean-absolute-value scales, packed signs.  Returns (Layer, eta as a 0-d fp64 tensor)."""
+    if Uh.dtype != torch.float32 or Vh.dtype != torch.float32 or Uh.stride(1) != 1 or Vh.stride(1) != 1:
+        raise ValueError("latents must be float32 with unit column stride")
+    r = int(Uh.shape[1]) if r is None else int(r)
+    d_out, d_in = int(Uh.shape[0]), int(Vh.shape[0])
+    ld = -(-(r // 32) // ld_align_words) * ld_align_words
+    dev = Uh.device
+    U = torch.empty((d_out, ld), dtype=torch.int32, device=dev)
+    V = torch.empty((d_in, ld), dtype=torch.int32, device=dev)
+    s1 = torch.empty(d_out, dtype=torch.float16, device=dev)
+    s2 = torch.empty(d_in, dtype=torch.float16, device=dev)
+    eta = torch.empty((), dtype=torch.float64, device=dev)
+    need = int(_lib.nq_from_latent_workspace_bytes(d_out, d_in, r, ld, ld))
+    if need == 0:
+        raise NQError("nq_from_latent_workspace_bytes", 2)
+    ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    _check("nq_lrb_from_latent", _lib.nq_lrb_from_latent(_ptr(Uh), int(Uh.stride(0)), _ptr(Vh), int(Vh.stride(0)),
+                                                         d_out, d_in, r, _ptr(U), ld, _ptr(V), ld, _ptr(s1),
+                                                         _ptr(s2), _ptr(eta), _ptr(ws), need, _stream_ptr(stream)))
+    return Layer(U, V, s1, s2, r), eta
 
 
 def silu_mul(g: torch.Tensor, u: torch.Tensor, h=None, stream=None) -> torch.Tensor:

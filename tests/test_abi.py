@@ -108,6 +108,27 @@ def test_workspace_covers_both_directions(nq):
         assert a == b > 0
 
 
+def test_from_latent_argument_errors(nq):
+    lib = nq.raw_lib()
+
+    def call(Uh=0x10000, ld_uh=64, Vh=0x20000, ld_vh=64, d_out=8, d_in=8, r=64, U=0x30000, ldu=2, V=0x40000, ldv=2,
+             s1=0x50000, s2=0x60000, eta=0, ws=0x70000, ws_bytes=1 << 20):
+        return lib.nq_lrb_from_latent(Uh, ld_uh, Vh, ld_vh, d_out, d_in, r, U, ldu, V, ldv, s1, s2, eta, ws, ws_bytes,
+                                      None)
+
+    assert call(r=48) == NQ["SHAPE"]
+    assert call(ld_uh=32) == NQ["SHAPE"]
+    assert call(ldv=1) == NQ["SHAPE"]
+    assert call(d_in=0) == NQ["SHAPE"]
+    assert call(Uh=0) == NQ["NULL"]
+    assert call(s2=0) == NQ["NULL"]
+    assert call(V=0x40004) == NQ["ALIGN"]
+    assert call(eta=0x80004) == NQ["ALIGN"]
+    assert call(ws_bytes=16) == NQ["WORKSPACE"]
+    assert lib.nq_from_latent_workspace_bytes(8, 8, 64, 2, 2) > 0
+    assert lib.nq_from_latent_workspace_bytes(8, 8, 48, 2, 2) == 0
+
+
 def test_matvec_rejects_large_batch(nq):
     assert _call(nq, "nq_lrb_matvec", _layer(nq), M=nq.MATVEC_MAX_M + 1) == NQ["SHAPE"]
 
