@@ -48,7 +48,7 @@ def parse_args():
     ap.add_argument("--headline-only", action="store_true", help="skip the other workloads")
     ap.add_argument("--only", default=None,
                     help="run just these extra sections (comma list of attn7b_b8, mlp7b, layer70b, prefill, pack, "
-                         "calib) "
+                         "calib, model70b) "
                          "after the headline; implies no CPU baseline")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU oracle sample budget")
     return ap.parse_args()
@@ -362,6 +362,8 @@ def extras(torch, nq, stream, args, hbm_gbs, bf16_tf, bf16_tf_sus, peak_src):
         out["pack_70b_gate_U"] = _extra_pack(torch, nq, stream, steps, warm, hbm_gbs)
     if on("calib"):
         out.update(_extra_calib(torch, nq, stream, steps, warm, hbm_gbs, bf16_tf))
+    if on("model70b"):
+        out["model70b_decode_b1"] = _extra_model70b(torch, nq, stream, hbm_gbs)
     nq.sync_status(stream)
     return out
 
@@ -495,6 +497,56 @@ def _extra_calib(torch, nq, stream, steps, warm, hbm_gbs, bf16_tf):
                                    "frac_hbm": round(moved / us / 1e3 / hbm_gbs, 4)}
     del g
     return out
+
+
+def _extra_model70b(torch, nq, stream, hbm_gbs, n_layers=80):
+    """One token (batch 1) through the LRB projections of 80 Llama-2-70B decoder layers
+    (q, k, v, o, gate, up, down + SiLU.mul each; attention core and norms are not LRB
+    matmuls).  Random packed signs and scales generated on the device: every layer distinct."""
+    shapes = synth.WORKLOADS["layer70b"]
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(synth.workload_seed("layer70b") + 80)
+
+    def words(rows, r):
+        ld = -(-(r // 32) // 4) * 4
+        return torch.randint(-2 ** 31, 2 ** 31 - 1, (rows, ld), dtype=torch.int32, device="cuda", generator=gen)
+
+    def scales(n):
+        return (0.02 * torch.randn(n, device="cuda", generator=gen).abs()).half()
+
+    layers = []
+    for _ in range(n_layers):
+        layers.append({name: nq.Layer(words(do, r), words(di, r), scales(do), scales(di), r)
+                       for (name, do, di, r) in shapes})
+    need = max(L.workspace_bytes(1) for bl in layers for L in bl.values())
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    dmodel = shapes[0][2]
+    x = torch.zeros((1, dmodel), dtype=torch.bfloat16, device="cuda").normal_()
+    bufs = {name: torch.empty((1, do), dtype=torch.bfloat16, device="cuda") for (name, do, di, r) in shapes}
+    h = torch.empty((1, layers[0]["gate"].d_out), dtype=torch.bfloat16, device="cuda")
+
+    def token():
+        xx = x
+        for bl in layers:
+            for name in ("q", "k", "v"):
+                nq.layer_forward(bl[name], xx, bufs[name], ws=ws, stream=stream)
+            nq.layer_forward(bl["o"], bufs["q"], bufs["o"], ws=ws, stream=stream)  # stands in for attention
+            nq.layer_forward(bl["gate"], bufs["o"], bufs["gate"], ws=ws, stream=stream)
+            nq.layer_forward(bl["up"], bufs["o"], bufs["up"], ws=ws, stream=stream)
+            nq.silu_mul(bufs["gate"], bufs["up"], h, stream=stream)
+            nq.layer_forward(bl["down"], h, bufs["down"], ws=ws, stream=stream)
+            xx = bufs["down"]
+
+    g = graph_of(torch, token, stream)
+    ms = timed_replays(torch, g, stream, 10, 3)
+    us = ms * 1e3 / 10
+    wbytes = sum(L.U.numel() * 4 + L.V.numel() * 4 + 2 * (L.d_out + L.d_in) for bl in layers for L in bl.values())
+    alg = n_layers * sum(decode_bytes(do, di, r, 1) for (_, do, di, r) in shapes)
+    del g, layers
+    return {"layers": n_layers, "weights_GB": round(wbytes / 1e9, 3), "us_per_token": round(us, 1),
+            "tokens_per_s": round(1e6 / us, 1), "GB_s": round(alg / us / 1e3, 1),
+            "frac_hbm": round(alg / us / 1e3 / hbm_gbs, 4),
+            "note": "LRB projections + SiLU.mul only; o takes q's output in place of attention"}
 
 
 def _extra_pack(torch, nq, stream, steps, warm, hbm_gbs):
