@@ -32,18 +32,30 @@ __global__ void __launch_bounds__(256) pack_stats_kernel(const float* __restrict
         const int64_t w0 = (task - row * tasks_per_row) * 32;
         const float* src = latent + row * ld_latent + w0 * 32 + lane;
         float v[32];
+        if (w0 + 32 <= words) {  // a full task: no bounds to check
 #pragma unroll
-        for (int u = 0; u < 32; ++u) v[u] = (w0 + u < words) ? __ldcs(src + u * 32) : 0.0f;
-        uint32_t mine = 0;
+            for (int u = 0; u < 32; ++u) v[u] = __ldcs(src + u * 32);
+        } else {
+#pragma unroll
+            for (int u = 0; u < 32; ++u) v[u] = (w0 + u < words) ? __ldcs(src + u * 32) : 0.0f;
+        }
+        // word u is the same in every lane; lane u keeps it (binary select on the lane bits)
+        uint32_t b[32];
         double sa = 0.0, sq = 0.0;
 #pragma unroll
         for (int u = 0; u < 32; ++u) {
-            const uint32_t word = __ballot_sync(0xffffffffu, v[u] >= 0.0f);  // NaN >= 0 is false
-            if (lane == u) mine = word;
+            b[u] = __ballot_sync(0xffffffffu, v[u] >= 0.0f);  // NaN >= 0 is false
             const double d = static_cast<double>(v[u]);
             sa += fabs(d);
             sq += d * d;
         }
+#pragma unroll
+        for (int lvl = 0, n = 16; lvl < 5; ++lvl, n >>= 1) {
+            const bool hi = (lane >> lvl) & 1;
+#pragma unroll
+            for (int i = 0; i < n; ++i) b[i] = hi ? b[2 * i + 1] : b[2 * i];
+        }
+        const uint32_t mine = b[0];
         for (int off = 16; off > 0; off >>= 1) {
             sa += __shfl_xor_sync(0xffffffffu, sa, off);
             sq += __shfl_xor_sync(0xffffffffu, sq, off);
