@@ -189,6 +189,21 @@ NQ_API nq_status nq_lrb_scale_grads(const nq_lrb_layer* L, const uint16_t* x, co
                                     float* g_s1, float* g_s2, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * nq_layer_forward_group -- y[l] = layer l applied to x, for 1 <= n <= NQ_MAX_GROUP projections
+ * that share their input (a transformer's q, k, v, or its gate and up): every layer must have
+ * the same d_in; d_out and r may differ.  For M <= NQ_MATVEC_MAX_M the group runs as one
+ * launch of each decode stage (the layers' blocks side by side), which saves a kernel pair's
+ * fixed latency per extra member; numerics as nq_lrb_matvec, except that the row slices of V
+ * over which x is quantised follow the group's total size.  Larger M runs nq_lrb_matmul once
+ * per layer.  y: array of n output pointers ([M][d_out_l] bf16 each); ws:
+ * nq_group_workspace_bytes(layers, n, M) bytes (0 for an invalid group).
+ */
+#define NQ_MAX_GROUP 4
+NQ_API size_t nq_group_workspace_bytes(const nq_lrb_layer* const* layers, int n, int64_t M);
+NQ_API nq_status nq_layer_forward_group(const nq_lrb_layer* const* layers, int n, const uint16_t* x,
+                                        uint16_t* const* y, int64_t M, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * nq_silu_mul -- h[e] = bf16( silu(g[e]) * u[e] ), silu(g) = g / (1 + exp(-g)), fp32 math,
  * for the Llama MLP block built from LRB projections (gate, up -> h -> down).  Not part of
  * the factorisation itself.  g, u, h: n bf16 values each, device.

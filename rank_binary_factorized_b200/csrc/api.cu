@@ -1,6 +1,7 @@
 // api.cu -- the C ABI declared in include/nq.h: argument validation, device checks,
 // workspace planning and dispatch to the kernels.  No allocation, no synchronisation (except
 // nq_sync_status), no fallback: a device that is not sm_100 gets NQ_ERR_DEVICE.
+#include <algorithm>
 #include <mutex>
 
 #include "nq_common.cuh"
@@ -225,6 +226,38 @@ nq_status nq_layer_forward(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y
                            size_t ws_bytes, void* stream) {
     if (M >= 1 && M <= NQ_MATVEC_MAX_M) return nq_lrb_matvec(L, x, y, M, ws, ws_bytes, stream);
     return nq_lrb_matmul(L, x, y, M, ws, ws_bytes, stream);
+}
+
+size_t nq_group_workspace_bytes(const nq_lrb_layer* const* layers, int n, int64_t M) {
+    if (!layers || n < 1 || n > NQ_MAX_GROUP || M < 1) return 0;
+    size_t bytes = 0;
+    for (int l = 0; l < n; ++l) {
+        if (check_layer(layers[l]) != NQ_OK || layers[l]->d_in != layers[0]->d_in) return 0;
+        bytes = std::max(bytes, nq_workspace_bytes(layers[l], M));
+    }
+    if (M <= NQ_MATVEC_MAX_M) bytes = std::max(bytes, nq_decode_group_workspace_bytes(layers, n, M));
+    return bytes;
+}
+
+nq_status nq_layer_forward_group(const nq_lrb_layer* const* layers, int n, const uint16_t* x, uint16_t* const* y,
+                                 int64_t M, void* ws, size_t ws_bytes, void* stream) {
+    if (!layers || !y) return NQ_ERR_NULL;
+    if (n < 1 || n > NQ_MAX_GROUP || M < 1) return NQ_ERR_SHAPE;
+    nq_status st;
+    for (int l = 0; l < n; ++l) {
+        if ((st = check_layer(layers[l])) != NQ_OK) return st;
+        if (layers[l]->d_in != layers[0]->d_in) return NQ_ERR_SHAPE;
+        if (M <= NQ_MATVEC_MAX_M && nq_decode_stage2_smem(layers[l]->r, M) > kMaxDecodeSmem) return NQ_ERR_SHAPE;
+        if ((st = check_io(x, y[l], ws)) != NQ_OK) return st;
+    }
+    if (ws_bytes < nq_group_workspace_bytes(layers, n, M)) return NQ_ERR_WORKSPACE;
+    DeviceInfo* d = current_device();
+    if (!d || !d->ok) return NQ_ERR_DEVICE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (M <= NQ_MATVEC_MAX_M) return nq_launch_decode_group(layers, n, x, y, M, ws, s, pdl_enabled());
+    for (int l = 0; l < n; ++l)
+        if ((st = nq_launch_prefill(layers[l], x, y[l], M, ws, s, pdl_enabled())) != NQ_OK) return st;
+    return NQ_OK;
 }
 
 nq_status nq_lrb_transposed(const nq_lrb_layer* L, const uint16_t* ybar, uint16_t* xbar, int64_t M, void* ws,

@@ -18,6 +18,8 @@
 // weights before it waits for the previous grid.
 #include <cooperative_groups.h>
 
+#include <algorithm>
+
 #include "nq_common.cuh"
 
 namespace nq {
@@ -107,6 +109,15 @@ struct S1Params {
     int64_t upf_bytes;    // prefetched into L2 for stage 2, 1/grid of them per block
 };
 
+// Up to kMaxGroup projections that share their input x are launched as one grid: block
+// column c belongs to member l when chunk_off[l] <= c < chunk_off[l + 1].
+constexpr int kMaxGroup = NQ_MAX_GROUP;
+struct S1Group {
+    S1Params p[kMaxGroup];
+    int chunk_off[kMaxGroup + 1];
+    int n;
+};
+
 template <int NT>
 struct S1Layout {
     static constexpr int SWZ = (NT == 1) ? 8 : 24;  // words per quad row of the z table
@@ -124,13 +135,20 @@ __device__ __forceinline__ void byte_transpose4(uint32_t w0, uint32_t w1, uint32
     o[3] = __byte_perm(t1, t3, 0x7632);
 }
 
-template <int NT, int TH>
-__global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const S1Params p) {
+// GN: 1 for a single layer (member 0, resolved at compile time), kMaxGroup for a group.
+template <int NT, int TH, int GN>
+__global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const __grid_constant__ S1Group grp) {
     constexpr int kS1Threads = TH;
     constexpr int kKSplit = kS1Threads / (32 * kS1Words);  // warps per word column
     namespace cg = cooperative_groups;
     constexpr int SWZ = S1Layout<NT>::SWZ;
     extern __shared__ __align__(16) uint32_t smem1[];
+    int li = 0;  // the member of the group this block works for
+    if (GN > 1)
+        while (li + 1 < grp.n && static_cast<int>(blockIdx.x) >= grp.chunk_off[li + 1]) ++li;
+    const S1Params& p = grp.p[li];
+    const int chunk = blockIdx.x - grp.chunk_off[li];
+    const int n_chunks = grp.chunk_off[li + 1] - grp.chunk_off[li];
     const int nq_rows = p.jc_rows / 4;  // quads per pass
     const int nkb = p.jc_rows / 32;     // K steps per pass
     uint32_t* aws = smem1;                          // [8 words][nkb][2][4][4]
@@ -147,7 +165,7 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const S1Params p) 
     cg::cluster_group cluster = cg::this_cluster();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int gid = lane >> 2, tig = lane & 3;
-    const int chunk = blockIdx.x;
+
     const int q = blockIdx.y;  // slice index == rank in the cluster
     const int CS = gridDim.y;
     const int64_t j0 = static_cast<int64_t>(q) * p.rows_per_slice;
@@ -190,7 +208,7 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const S1Params p) 
 
     // stage 2's weights: start their way from HBM into L2 now, so that stage 2 reads them there
     if (tid == 0 && p.upf_bytes > 0) {
-        const int G = gridDim.x * gridDim.y, b = blockIdx.y * gridDim.x + blockIdx.x;
+        const int G = n_chunks * gridDim.y, b = blockIdx.y * n_chunks + chunk;
         const int64_t share = ((p.upf_bytes + G - 1) / G + 15) & ~static_cast<int64_t>(15);
         const int64_t beg = static_cast<int64_t>(b) * share, end = min(beg + share, p.upf_bytes);
         for (int64_t off = beg; off < end; off += 32768)
@@ -492,6 +510,13 @@ struct S2Params {
     float* grad;
 };
 
+// Stage-2 blocks [cta_off[l], cta_off[l + 1]) work for member l of the group.
+struct S2Group {
+    S2Params p[kMaxGroup];
+    int cta_off[kMaxGroup + 1];
+    int n;
+};
+
 // B table layout: the two B-fragment words of lane (gid, tig) for bit offset s, word group g
 // (8 words) and column tile nt sit next to each other, lanes in order, so one 64-bit load per
 // lane and MMA reads 256 contiguous bytes:
@@ -503,11 +528,17 @@ __device__ __forceinline__ int s2_bidx(int s_, int w, int col, int ng) {
     return ((((s_ * ng + g) * NT + (col >> 3)) * 32 + 4 * (col & 7) + tg) * 2 + half);
 }
 
-template <int NT, int TH>
-__global__ void __launch_bounds__(TH, 1) decode_stage2_kernel(const S2Params p) {
+template <int NT, int TH, int GN>
+__global__ void __launch_bounds__(TH, 1) decode_stage2_kernel(const __grid_constant__ S2Group grp) {
     constexpr int kS2Threads = TH;
     constexpr int kS2Warps = kS2Threads / 32;
     extern __shared__ __align__(16) uint32_t smem2[];
+    int li = 0;  // the member of the group this block works for
+    if (GN > 1)
+        while (li + 1 < grp.n && static_cast<int>(blockIdx.x) >= grp.cta_off[li + 1]) ++li;
+    const S2Params& p = grp.p[li];
+    const int bid = blockIdx.x - grp.cta_off[li];
+    const int G = grp.cta_off[li + 1] - grp.cta_off[li];
     uint32_t* bt = smem2;                                  // 8 * nwp * NT*8 words (s2_bidx)
     uint32_t* ublk = bt + 8 * p.nwp * NT * 8;              // [chunk_mt*16][su]
     int* red = reinterpret_cast<int*>(ublk + p.chunk_mt * 16 * p.su);  // [chunk_mt*16][NT*8]
@@ -519,9 +550,9 @@ __global__ void __launch_bounds__(TH, 1) decode_stage2_kernel(const S2Params p) 
     __shared__ float s_wmax[kS2Warps][NQ_MATVEC_MAX_M];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int G = gridDim.x;
-    const int mt0 = static_cast<int>((static_cast<int64_t>(blockIdx.x) * p.mt_total) / G);
-    const int mt1 = static_cast<int>((static_cast<int64_t>(blockIdx.x + 1) * p.mt_total) / G);
+
+    const int mt0 = static_cast<int>((static_cast<int64_t>(bid) * p.mt_total) / G);
+    const int mt1 = static_cast<int>((static_cast<int64_t>(bid + 1) * p.mt_total) / G);
 
     // stage the rows of U of M-tiles [a, b) into ublk (row stride su); weights only, so this
     // may run before the previous grid has finished
@@ -782,11 +813,15 @@ struct S1Plan {
     size_t smem;
 };
 
-S1Plan plan_stage1(int64_t d_in, int64_t r, int64_t M) {
+int chunks_of(int64_t r) { return static_cast<int>((r / 32 + nq::kS1Words - 1) / nq::kS1Words); }
+
+// Stage-1 shape for a grid of `total_chunks` word chunks over d_in rows: the cluster size CS
+// (row slices per chunk) shrinks as the chunk count grows, so that the grid stays near one
+// block per SM; rows per slice and the staging pass follow.
+S1Plan plan_stage1(int64_t d_in, int total_chunks, int64_t M) {
     S1Plan p{};
-    const int64_t nw = r / 32;
-    p.n_chunks = static_cast<int>((nw + nq::kS1Words - 1) / nq::kS1Words);
-    int cs = p.n_chunks <= 8 ? 16 : (p.n_chunks <= 18 ? 8 : (p.n_chunks <= 37 ? 4 : 2));
+    p.n_chunks = total_chunks;
+    int cs = total_chunks <= 8 ? 16 : (total_chunks <= 18 ? 8 : (total_chunks <= 37 ? 4 : 2));
     while (cs > 1 && static_cast<int64_t>(cs) * 32 > d_in) cs >>= 1;
     p.CS = cs;
     p.rows_per_slice = static_cast<int>(((d_in + cs - 1) / cs + 31) / 32 * 32);
@@ -807,89 +842,129 @@ S1Plan plan_stage1(int64_t d_in, int64_t r, int64_t M) {
 
 size_t decode_ws_bytes(int64_t r, int64_t M) { return kWsHeader + align256(static_cast<size_t>(M * r) * sizeof(float)); }
 
-template <int NT, int TH1, int TH2>
+template <int NT, int TH1, int TH2, int GN>
 void set_attrs_once() {
     static bool done[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || done[dev]) return;
-    cudaFuncSetAttribute(nq::decode_stage1_kernel<NT, TH1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(nq::decode_stage1_kernel<NT, TH1, GN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(kStage1SmemBudget));
-    cudaFuncSetAttribute(nq::decode_stage1_kernel<NT, TH1>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    cudaFuncSetAttribute(nq::decode_stage2_kernel<NT, TH2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(nq::decode_stage1_kernel<NT, TH1, GN>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    cudaFuncSetAttribute(nq::decode_stage2_kernel<NT, TH2, GN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(kStage2SmemBudget));
     done[dev] = true;
 }
 
-template <int NT>
-nq_status launch_decode_nt(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y, int M, void* ws,
-                           const uint16_t* cot, float* grad,
-                           cudaStream_t stream, bool pdl) {
-    float* t = reinterpret_cast<float*>(static_cast<char*>(ws) + kWsHeader);
+// One launch of each stage for n projections that share x (n = 1: a single layer).
+template <int NT, int GN>
+nq_status launch_decode_group_nt(const nq_lrb_layer* const* Ls, int n, const uint16_t* x, uint16_t* const* ys, int M,
+                                 void* ws, const uint16_t* cot, float* grad, cudaStream_t stream, bool pdl) {
+    // t of member l follows the earlier members' t in the workspace
+    float* t[nq::kMaxGroup];
+    size_t off = kWsHeader;
+    for (int l = 0; l < n; ++l) {
+        t[l] = reinterpret_cast<float*>(static_cast<char*>(ws) + off);
+        off += align256(static_cast<size_t>(M) * Ls[l]->r * sizeof(float));
+    }
     {
-        const S1Plan sp = plan_stage1(L->d_in, L->r, M);
-        nq::S1Params q{};
-        q.V = L->V;
-        q.ldv = L->ldv;
-        q.s2 = L->s2;
-        q.x = x;
-        q.t = t;
-        q.M = M;
-        q.d_in = L->d_in;
-        q.r = static_cast<int>(L->r);
-        q.nw = static_cast<int>(L->r / 32);
-        q.rows_per_slice = sp.rows_per_slice;
-        q.jc_rows = sp.jc_rows;
-        q.zstage = sp.zstage;
-        q.upf = L->U;
-        // U up to the last valid word of its last row, rounded down to 16 bytes
-        q.upf_bytes = (((L->d_out - 1) * L->ldu + L->r / 32) * 4) & ~static_cast<int64_t>(15);
-        void* args[] = {&q};
+        int total = 0;
+        for (int l = 0; l < n; ++l) total += chunks_of(Ls[l]->r);
+        const S1Plan sp = plan_stage1(Ls[0]->d_in, total, M);
+        nq::S1Group g{};
+        g.n = n;
+        int acc = 0;
+        for (int l = 0; l < n; ++l) {
+            const nq_lrb_layer* L = Ls[l];
+            nq::S1Params& q = g.p[l];
+            q.V = L->V;
+            q.ldv = L->ldv;
+            q.s2 = L->s2;
+            q.x = x;
+            q.t = t[l];
+            q.M = M;
+            q.d_in = L->d_in;
+            q.r = static_cast<int>(L->r);
+            q.nw = static_cast<int>(L->r / 32);
+            q.rows_per_slice = sp.rows_per_slice;
+            q.jc_rows = sp.jc_rows;
+            q.zstage = sp.zstage;
+            q.upf = L->U;
+            // U up to the last valid word of its last row, rounded down to 16 bytes
+            q.upf_bytes = (((L->d_out - 1) * L->ldu + L->r / 32) * 4) & ~static_cast<int64_t>(15);
+            g.chunk_off[l] = acc;
+            acc += chunks_of(L->r);
+        }
+        g.chunk_off[n] = acc;
+        void* args[] = {&g};
         const bool wide = (NT <= 2) && sp.rows_per_slice >= 1024;
-        const void* fn = wide ? reinterpret_cast<const void*>(nq::decode_stage1_kernel<NT, (NT <= 2 ? 512 : 256)>)
-                              : reinterpret_cast<const void*>(nq::decode_stage1_kernel<NT, 256>);
-        if (wide) set_attrs_once<NT, (NT <= 2 ? 512 : 256), 256>();
-        else set_attrs_once<NT, 256, 256>();
-        if (nq_host::launch_ex(fn, dim3(sp.n_chunks, sp.CS), dim3(wide ? 512 : 256), sp.smem, stream, args, pdl,
-                               sp.CS) != cudaSuccess)
+        const void* fn = wide ? reinterpret_cast<const void*>(nq::decode_stage1_kernel<NT, (NT <= 2 ? 512 : 256), GN>)
+                              : reinterpret_cast<const void*>(nq::decode_stage1_kernel<NT, 256, GN>);
+        if (wide) set_attrs_once<NT, (NT <= 2 ? 512 : 256), 256, GN>();
+        else set_attrs_once<NT, 256, 256, GN>();
+        if (nq_host::launch_ex(fn, dim3(acc, sp.CS), dim3(wide ? 512 : 256), sp.smem, stream, args, pdl, sp.CS) !=
+            cudaSuccess)
             return NQ_ERR_LAUNCH;
     }
     {
-        nq::S2Params q{};
-        q.U = L->U;
-        q.ldu = L->ldu;
-        q.s1 = L->s1;
-        q.t = t;
-        q.y = y;
-        q.cot = cot;
-        q.grad = grad;
-        q.M = M;
-        q.d_out = L->d_out;
-        q.r = static_cast<int>(L->r);
-        q.nw = static_cast<int>(L->r / 32);
-        q.nwp = (q.nw + 7) / 8 * 8;
-        q.su = q.nwp + ((4 - q.nwp % 32) + 32) % 32;
-        q.mt_total = static_cast<int>((L->d_out + 15) / 16);
-        int grid = nq_host::sm_count();
-        if (grid > q.mt_total) grid = q.mt_total;
-        const int per_cta = (q.mt_total + grid - 1) / grid;
-        const size_t bt_bytes = static_cast<size_t>(8) * q.nwp * NT * 8 * 4;
-        const size_t per_mt = static_cast<size_t>(16) * q.su * 4 + static_cast<size_t>(16) * NT * 8 * 4 + 16 * 4;
-        int chunk = per_cta;
-        if (bt_bytes + chunk * per_mt > kStage2SmemBudget) chunk = static_cast<int>((kStage2SmemBudget - bt_bytes) / per_mt);
-        if (chunk < 1) return NQ_ERR_SHAPE;
-        q.chunk_mt = chunk;
-        size_t smem2 = bt_bytes + chunk * per_mt;
-        const size_t t_bytes = static_cast<size_t>(M) * (L->r + L->r / 32) * sizeof(float);
-        q.tstage = (smem2 + t_bytes <= kStage2SmemBudget) ? 1 : 0;
-        if (q.tstage) smem2 += t_bytes;
-        void* args[] = {&q};
-        const bool wide = (NT == 1) && per_cta >= 6;
-        const void* fn = wide ? reinterpret_cast<const void*>(nq::decode_stage2_kernel<NT, (NT == 1 ? 512 : 256)>)
-                              : reinterpret_cast<const void*>(nq::decode_stage2_kernel<NT, 256>);
-        if (wide) set_attrs_once<NT, 256, (NT == 1 ? 512 : 256)>();
-        else set_attrs_once<NT, 256, 256>();
-        if (nq_host::launch_ex(fn, dim3(grid), dim3(wide ? 512 : 256), smem2, stream, args, pdl, 1) != cudaSuccess)
+        // the SMs are shared among the members in proportion to their weight words
+        const int sms = nq_host::sm_count();
+        double wsum = 0.0;
+        int mt[nq::kMaxGroup], nwp[nq::kMaxGroup], grid[nq::kMaxGroup];
+        for (int l = 0; l < n; ++l) {
+            mt[l] = static_cast<int>((Ls[l]->d_out + 15) / 16);
+            nwp[l] = static_cast<int>((Ls[l]->r / 32 + 7) / 8 * 8);
+            wsum += static_cast<double>(mt[l]) * nwp[l];
+        }
+        nq::S2Group g{};
+        g.n = n;
+        size_t smem = 0;
+        int min_per_cta = 1 << 30, acc = 0;
+        for (int l = 0; l < n; ++l) {
+            const nq_lrb_layer* L = Ls[l];
+            int gl = static_cast<int>(sms * (static_cast<double>(mt[l]) * nwp[l]) / wsum + 0.5);
+            gl = std::max(1, std::min(gl, mt[l]));
+            grid[l] = gl;
+            nq::S2Params& q = g.p[l];
+            q.U = L->U;
+            q.ldu = L->ldu;
+            q.s1 = L->s1;
+            q.t = t[l];
+            q.y = ys ? ys[l] : nullptr;
+            q.cot = cot;
+            q.grad = grad;
+            q.M = M;
+            q.d_out = L->d_out;
+            q.r = static_cast<int>(L->r);
+            q.nw = static_cast<int>(L->r / 32);
+            q.nwp = nwp[l];
+            q.su = q.nwp + ((4 - q.nwp % 32) + 32) % 32;
+            q.mt_total = mt[l];
+            const int per_cta = (q.mt_total + gl - 1) / gl;
+            min_per_cta = std::min(min_per_cta, per_cta);
+            const size_t bt_bytes = static_cast<size_t>(8) * q.nwp * NT * 8 * 4;
+            const size_t per_mt = static_cast<size_t>(16) * q.su * 4 + static_cast<size_t>(16) * NT * 8 * 4 + 16 * 4;
+            int chunk = per_cta;
+            if (bt_bytes + chunk * per_mt > kStage2SmemBudget)
+                chunk = static_cast<int>((kStage2SmemBudget - bt_bytes) / per_mt);
+            if (chunk < 1) return NQ_ERR_SHAPE;
+            q.chunk_mt = chunk;
+            size_t smem2 = bt_bytes + chunk * per_mt;
+            const size_t t_bytes = static_cast<size_t>(M) * (L->r + L->r / 32) * sizeof(float);
+            q.tstage = (smem2 + t_bytes <= kStage2SmemBudget) ? 1 : 0;
+            if (q.tstage) smem2 += t_bytes;
+            smem = std::max(smem, smem2);
+            g.cta_off[l] = acc;
+            acc += gl;
+        }
+        g.cta_off[n] = acc;
+        void* args[] = {&g};
+        const bool wide = (NT == 1) && min_per_cta >= 6;
+        const void* fn = wide ? reinterpret_cast<const void*>(nq::decode_stage2_kernel<NT, (NT == 1 ? 512 : 256), GN>)
+                              : reinterpret_cast<const void*>(nq::decode_stage2_kernel<NT, 256, GN>);
+        if (wide) set_attrs_once<NT, 256, (NT == 1 ? 512 : 256), GN>();
+        else set_attrs_once<NT, 256, 256, GN>();
+        if (nq_host::launch_ex(fn, dim3(acc), dim3(wide ? 512 : 256), smem, stream, args, pdl, 1) != cudaSuccess)
             return NQ_ERR_LAUNCH;
     }
     return NQ_OK;
@@ -913,12 +988,31 @@ size_t nq_decode_stage2_smem(int64_t r, int64_t M) {
     return need <= kStage2SmemBudget ? need : kStage2SmemBudget + 1;
 }
 
+nq_status nq_launch_decode_group(const nq_lrb_layer* const* Ls, int n, const uint16_t* x, uint16_t* const* ys,
+                                 int64_t M, void* ws, cudaStream_t stream, bool pdl, const uint16_t* cot,
+                                 float* grad) {
+    const int m = static_cast<int>(M);
+    if (n == 1) {
+        switch (ntiles_for(M)) {
+            case 1: return launch_decode_group_nt<1, 1>(Ls, n, x, ys, m, ws, cot, grad, stream, pdl);
+            case 2: return launch_decode_group_nt<2, 1>(Ls, n, x, ys, m, ws, cot, grad, stream, pdl);
+            default: return launch_decode_group_nt<3, 1>(Ls, n, x, ys, m, ws, cot, grad, stream, pdl);
+        }
+    }
+    switch (ntiles_for(M)) {
+        case 1: return launch_decode_group_nt<1, nq::kMaxGroup>(Ls, n, x, ys, m, ws, cot, grad, stream, pdl);
+        case 2: return launch_decode_group_nt<2, nq::kMaxGroup>(Ls, n, x, ys, m, ws, cot, grad, stream, pdl);
+        default: return launch_decode_group_nt<3, nq::kMaxGroup>(Ls, n, x, ys, m, ws, cot, grad, stream, pdl);
+    }
+}
+
 nq_status nq_launch_decode(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y, int64_t M, void* ws,
                            cudaStream_t stream, bool pdl, const uint16_t* cot, float* grad) {
-    const int m = static_cast<int>(M);
-    switch (ntiles_for(M)) {
-        case 1: return launch_decode_nt<1>(L, x, y, m, ws, cot, grad, stream, pdl);
-        case 2: return launch_decode_nt<2>(L, x, y, m, ws, cot, grad, stream, pdl);
-        default: return launch_decode_nt<3>(L, x, y, m, ws, cot, grad, stream, pdl);
-    }
+    return nq_launch_decode_group(&L, 1, x, &y, M, ws, stream, pdl, cot, grad);
+}
+
+size_t nq_decode_group_workspace_bytes(const nq_lrb_layer* const* Ls, int n, int64_t M) {
+    size_t off = kWsHeader;
+    for (int l = 0; l < n; ++l) off += align256(static_cast<size_t>(M) * Ls[l]->r * sizeof(float));
+    return off;
 }

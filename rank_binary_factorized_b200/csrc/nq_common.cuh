@@ -70,6 +70,11 @@ cudaError_t launch_ex(const void* fn, dim3 grid, dim3 block, size_t smem, cudaSt
 // of y.
 nq_status nq_launch_decode(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y, int64_t M, void* ws,
                            cudaStream_t stream, bool pdl, const uint16_t* cot = nullptr, float* grad = nullptr);
+// Decode path for n <= 4 projections sharing x, one launch per stage (decode.cu).
+nq_status nq_launch_decode_group(const nq_lrb_layer* const* Ls, int n, const uint16_t* x, uint16_t* const* ys,
+                                 int64_t M, void* ws, cudaStream_t stream, bool pdl, const uint16_t* cot = nullptr,
+                                 float* grad = nullptr);
+size_t nq_decode_group_workspace_bytes(const nq_lrb_layer* const* Ls, int n, int64_t M);
 // Prefill path (prefill.cu): Y = layer(x) on the tensor cores; with grad != nullptr it writes
 // grad[i] = sum_m cot[m][i] (T U^T)[m][i] instead of Y.
 nq_status nq_launch_prefill(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y, int64_t M, void* ws,

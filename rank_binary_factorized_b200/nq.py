@@ -56,6 +56,11 @@ _lib.nq_from_latent_workspace_bytes.argtypes = [_i64, _i64, _i64, _i64, _i64]
 _lib.nq_lrb_from_latent.restype = ctypes.c_int
 _lib.nq_lrb_from_latent.argtypes = [_p, _i64, _p, _i64, _i64, _i64, _i64, _p, _i64, _p, _i64, _p, _p, _p, _p,
                                     ctypes.c_size_t, _p]
+_lib.nq_group_workspace_bytes.restype = ctypes.c_size_t
+_lib.nq_group_workspace_bytes.argtypes = [ctypes.POINTER(ctypes.POINTER(nq_lrb_layer)), ctypes.c_int, _i64]
+_lib.nq_layer_forward_group.restype = ctypes.c_int
+_lib.nq_layer_forward_group.argtypes = [ctypes.POINTER(ctypes.POINTER(nq_lrb_layer)), ctypes.c_int, _p,
+                                        ctypes.POINTER(_p), _i64, _p, ctypes.c_size_t, _p]
 _lib.nq_lrb_scale_grads.restype = ctypes.c_int
 _lib.nq_lrb_scale_grads.argtypes = [ctypes.POINTER(nq_lrb_layer), _p, _p, _i64, _p, _p, _p, ctypes.c_size_t, _p]
 _lib.nq_sync_status.restype = ctypes.c_int
@@ -234,6 +239,33 @@ def lrb_from_latent(Uh: torch.Tensor, Vh: torch.Tensor, r: int | None = None, ld
                                                          d_out, d_in, r, _ptr(U), ld, _ptr(V), ld, _ptr(s1),
                                                          _ptr(s2), _ptr(eta), _ptr(ws), need, _stream_ptr(stream)))
     return Layer(U, V, s1, s2, r), eta
+
+
+def _layer_array(layers):
+    arr = (ctypes.POINTER(nq_lrb_layer) * len(layers))()
+    for i, L in enumerate(layers):
+        arr[i] = ctypes.pointer(L.struct)
+    return arr
+
+
+def group_workspace_bytes(layers, M: int) -> int:
+    return int(_lib.nq_group_workspace_bytes(_layer_array(layers), len(layers), M))
+
+
+def layer_forward_group(layers, x: torch.Tensor, ys=None, ws=None, stream=None):
+    """y_l = layers[l](x) for projections sharing x (one decode launch per stage for M <= 8)."""
+    M = int(x.shape[0])
+    if ys is None:
+        ys = [torch.empty((M, L.d_out), dtype=torch.bfloat16, device=x.device) for L in layers]
+    if ws is None:
+        need = group_workspace_bytes(layers, M)
+        if need == 0:
+            raise NQError("nq_group_workspace_bytes", 2)
+        ws = torch.zeros(need, dtype=torch.uint8, device=x.device)
+    yp = (_p * len(ys))(*[_ptr(y) for y in ys])
+    _check("nq_layer_forward_group", _lib.nq_layer_forward_group(_layer_array(layers), len(layers), _ptr(x), yp, M,
+                                                                 _ptr(ws), ws.numel(), _stream_ptr(stream)))
+    return ys
 
 
 def silu_mul(g: torch.Tensor, u: torch.Tensor, h=None, stream=None) -> torch.Tensor:

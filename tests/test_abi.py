@@ -129,6 +129,20 @@ def test_from_latent_argument_errors(nq):
     assert lib.nq_from_latent_workspace_bytes(8, 8, 48, 2, 2) == 0
 
 
+def test_group_argument_errors(nq):
+    lib = nq.raw_lib()
+    Ls = [_layer(nq), _layer(nq, d_out=32, r=32), _layer(nq, d_in=64)]
+    arr = (ctypes.POINTER(nq.nq_lrb_layer) * 3)(*[ctypes.pointer(L) for L in Ls])
+    ys = (ctypes.c_void_p * 3)(0x60000, 0x61000, 0x62000)
+    assert lib.nq_layer_forward_group(arr, 2, 0x50000, ys, 1, 0x70000, 1 << 30, None) != NQ["SHAPE"]
+    assert lib.nq_layer_forward_group(arr, 3, 0x50000, ys, 1, 0x70000, 1 << 30, None) == NQ["SHAPE"]  # d_in differs
+    assert lib.nq_layer_forward_group(arr, 0, 0x50000, ys, 1, 0x70000, 1 << 30, None) == NQ["SHAPE"]
+    assert lib.nq_layer_forward_group(arr, 5, 0x50000, ys, 1, 0x70000, 1 << 30, None) == NQ["SHAPE"]
+    assert lib.nq_layer_forward_group(arr, 2, 0x50000, ys, 1, 0x70000, 16, None) == NQ["WORKSPACE"]
+    assert lib.nq_group_workspace_bytes(arr, 2, 1) > 0
+    assert lib.nq_group_workspace_bytes(arr, 3, 1) == 0
+
+
 def test_matvec_rejects_large_batch(nq):
     assert _call(nq, "nq_lrb_matvec", _layer(nq), M=nq.MATVEC_MAX_M + 1) == NQ["SHAPE"]
 
