@@ -83,6 +83,9 @@ def lib() -> ctypes.CDLL:
         L.nq_oracle_scale_grads_packed.restype = ctypes.c_int
         L.nq_oracle_scale_grads_packed.argtypes = [_p, _i64, _p, _i64, _p, _p, _i64, _i64, _i64, _p, _p, _i64,
                                                    _p, _p, _p, _p]
+        L.nq_oracle_sign_grads_packed.restype = ctypes.c_int
+        L.nq_oracle_sign_grads_packed.argtypes = [_p, _i64, _p, _i64, _p, _p, _i64, _i64, _i64, _p, _p, _i64,
+                                                  _p, _i64, _p, _i64, _p, _i64, _p, _p, _p, _p]
         L.nq_oracle_double_to_f16.restype = ctypes.c_uint16
         L.nq_oracle_double_to_f16.argtypes = [ctypes.c_double]
         L.nq_oracle_from_latent.restype = ctypes.c_int
@@ -268,6 +271,37 @@ def scale_grads_packed(Uw, Vw, s1_f16, s2_f16, r: int, x_bf16, ybar_bf16):
     if rc != 0:
         raise ValueError("nq_oracle_scale_grads_packed failed (%d)" % rc)
     return g1, S1, g2, S2
+
+
+def sign_grads_packed(Uw, Vw, s1_f16, s2_f16, r: int, x_bf16, ybar_bf16, rows_u=None, rows_v=None, ks=None):
+    """dL/dU and dL/dV (the gradients the identity straight-through estimator hands to the
+    latent factors) for L = sum_b <ybar_b, y_b>, with the magnitudes of their terms.
+    ``rows_u``, ``rows_v`` and ``ks`` select rows of U, rows of V and rank columns (all when
+    None).  Returns (gU, SU [n_rows_u][n_ks], gV, SV [n_rows_v][n_ks]), fp64."""
+    Uw = _c(Uw, np.uint32)
+    Vw = _c(Vw, np.uint32)
+    s1 = _c(s1_f16, np.uint16)
+    s2 = _c(s2_f16, np.uint16)
+    x = _c(np.atleast_2d(x_bf16), np.uint16)
+    yb = _c(np.atleast_2d(ybar_bf16), np.uint16)
+    d_out, d_in, B = Uw.shape[0], Vw.shape[0], x.shape[0]
+    if yb.shape != (B, d_out) or x.shape != (B, d_in):
+        raise ValueError("x must be [B][d_in] and ybar [B][d_out]")
+    ru = None if rows_u is None else _c(rows_u, np.int64)
+    rv = None if rows_v is None else _c(rows_v, np.int64)
+    kk = None if ks is None else _c(ks, np.int64)
+    nu = d_out if ru is None else ru.size
+    nv = d_in if rv is None else rv.size
+    nk = r if kk is None else kk.size
+    gU, SU = np.empty((nu, nk)), np.empty((nu, nk))
+    gV, SV = np.empty((nv, nk)), np.empty((nv, nk))
+    opt = lambda a: None if a is None else _ptr(a)
+    rc = lib().nq_oracle_sign_grads_packed(_ptr(Uw), Uw.shape[1], _ptr(Vw), Vw.shape[1], _ptr(s1), _ptr(s2), d_out,
+                                           d_in, r, _ptr(x), _ptr(yb), B, opt(ru), nu, opt(rv), nv, opt(kk), nk,
+                                           _ptr(gU), _ptr(SU), _ptr(gV), _ptr(SV))
+    if rc != 0:
+        raise ValueError("nq_oracle_sign_grads_packed failed (%d)" % rc)
+    return gU, SU, gV, SV
 
 
 def double_to_f16(values) -> np.ndarray:

@@ -393,6 +393,101 @@ ORACLE_API int nq_oracle_scale_grads_packed(const uint32_t* U, int64_t ldu, cons
 }
 
 /* ---------------------------------------------------------------------------------
+ * Gradients with respect to the two sign factors (section 3, "Step 3: Factorized Component
+ * Refinement": the latent factors are refined through sign() with straight-through
+ * estimators).  For L = sum_b sum_i ybar[b][i] y[b][i] the section 2 equation, read
+ * elementwise, gives
+ *     dL/dU_ik = sum_b sum_j ybar[b][i] s1_i V_jk s2_j x[b][j]
+ *     dL/dV_jk = sum_b sum_i x[b][j] s2_j U_ik s1_i ybar[b][i]
+ * and the straight-through estimator passes them to the latent entries unchanged (the pages
+ * name no variant; the reading taken is the identity estimator).  Every term is an exact
+ * fp64 product (8 + 11 + 1 + 11 + 8 significant bits), so only the sums round.
+ *
+ * Entries (rows_u[a], ks[c]) of dL/dU and (rows_v[a], ks[c]) of dL/dV are evaluated (a NULL
+ * list means every row, or every k, in order), with the magnitudes of their terms:
+ * gU, SU [n_rows_u][n_ks]; gV, SV [n_rows_v][n_ks].  x [B][d_in], ybar [B][d_out] bf16 bits.
+ * --------------------------------------------------------------------------------- */
+static int sign_of_packed(const uint32_t* row, int64_t k) { return ((row[k / 32] >> (k % 32)) & 1u) ? 1 : -1; }
+
+ORACLE_API int nq_oracle_sign_grads_packed(const uint32_t* U, int64_t ldu, const uint32_t* V, int64_t ldv,
+                                           const uint16_t* s1_f16, const uint16_t* s2_f16, int64_t d_out,
+                                           int64_t d_in, int64_t r, const uint16_t* x_bf16,
+                                           const uint16_t* ybar_bf16, int64_t B, const int64_t* rows_u,
+                                           int64_t n_rows_u, const int64_t* rows_v, int64_t n_rows_v,
+                                           const int64_t* ks, int64_t n_ks, double* gU, double* SU, double* gV,
+                                           double* SV) {
+    if (r % 32 != 0 || ldu < r / 32 || ldv < r / 32) return -1;
+    if (rows_u == NULL) n_rows_u = d_out;
+    if (rows_v == NULL) n_rows_v = d_in;
+    if (ks == NULL) n_ks = r;
+    double* x = (double*)malloc(sizeof(double) * (size_t)(B * d_in > 0 ? B * d_in : 1));
+    double* yb = (double*)malloc(sizeof(double) * (size_t)(B * d_out > 0 ? B * d_out : 1));
+    if (!x || !yb) {
+        free(x);
+        free(yb);
+        return -2;
+    }
+    for (int64_t e = 0; e < B * d_in; ++e) x[e] = nq_oracle_bf16_to_double(x_bf16[e]);
+    for (int64_t e = 0; e < B * d_out; ++e) yb[e] = nq_oracle_bf16_to_double(ybar_bf16[e]);
+    int rc = 0;
+    for (int64_t a = 0; a < n_rows_u && rc == 0; ++a) {
+        const int64_t i = rows_u ? rows_u[a] : a;
+        if (i < 0 || i >= d_out) {
+            rc = -1;
+            break;
+        }
+        const double s1 = nq_oracle_f16_to_double(s1_f16[i]);
+        for (int64_t c = 0; c < n_ks; ++c) {
+            const int64_t k = ks ? ks[c] : c;
+            if (k < 0 || k >= r) {
+                rc = -1;
+                break;
+            }
+            double g = 0.0, S = 0.0;
+            for (int64_t b = 0; b < B; ++b) {
+                for (int64_t j = 0; j < d_in; ++j) {
+                    double term = yb[b * d_out + i] * s1 * (double)sign_of_packed(V + j * ldv, k) *
+                                  nq_oracle_f16_to_double(s2_f16[j]) * x[b * d_in + j];
+                    g += term;
+                    S += fabs(term);
+                }
+            }
+            if (gU) gU[a * n_ks + c] = g;
+            if (SU) SU[a * n_ks + c] = S;
+        }
+    }
+    for (int64_t a = 0; a < n_rows_v && rc == 0; ++a) {
+        const int64_t j = rows_v ? rows_v[a] : a;
+        if (j < 0 || j >= d_in) {
+            rc = -1;
+            break;
+        }
+        const double s2 = nq_oracle_f16_to_double(s2_f16[j]);
+        for (int64_t c = 0; c < n_ks; ++c) {
+            const int64_t k = ks ? ks[c] : c;
+            if (k < 0 || k >= r) {
+                rc = -1;
+                break;
+            }
+            double g = 0.0, S = 0.0;
+            for (int64_t b = 0; b < B; ++b) {
+                for (int64_t i = 0; i < d_out; ++i) {
+                    double term = x[b * d_in + j] * s2 * (double)sign_of_packed(U + i * ldu, k) *
+                                  nq_oracle_f16_to_double(s1_f16[i]) * yb[b * d_out + i];
+                    g += term;
+                    S += fabs(term);
+                }
+            }
+            if (gV) gV[a * n_ks + c] = g;
+            if (SV) SV[a * n_ks + c] = S;
+        }
+    }
+    free(x);
+    free(yb);
+    return rc;
+}
+
+/* ---------------------------------------------------------------------------------
  * From latent factors to a packed layer (section 3, "Step 2", "Magnitude Balancing and Scale
  * Extraction", then "Phase 3" packing): for the continuous proxies Uh [d_out][r] and
  * Vh [d_in][r],

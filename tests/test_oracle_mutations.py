@@ -62,6 +62,17 @@ MUTATIONS += [
     # fp16 encoder with the exponent field one too large
     ("return sign | (uint16_t)((e2 + 14) << 10) | frac;", "return sign | (uint16_t)((e2 + 15) << 10) | frac;", CONV),
 ]
+SGR = "test_oracle_sign_grads.py"
+MUTATIONS += [
+    # dL/dU: a dropped s1
+    ("double term = yb[b * d_out + i] * s1 * (double)sign_of_packed(V + j * ldv, k) *",
+     "double term = yb[b * d_out + i] * (double)sign_of_packed(V + j * ldv, k) *", SGR),
+    # dL/dV: the neighbouring rank column of U
+    ("double term = x[b * d_in + j] * s2 * (double)sign_of_packed(U + i * ldu, k) *",
+     "double term = x[b * d_in + j] * s2 * (double)sign_of_packed(U + i * ldu, (k + 1) % r) *", SGR),
+    # the packed bits read as 0/1 instead of -1/+1
+    ("return ((row[k / 32] >> (k % 32)) & 1u) ? 1 : -1;", "return ((row[k / 32] >> (k % 32)) & 1u) ? 1 : 0;", SGR),
+]
 MUTATIONS = [m if len(m) == 3 else (m[0], m[1], "test_oracle.py") for m in MUTATIONS]
 
 
