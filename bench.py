@@ -71,10 +71,20 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
 
 
+HOST_SIDE_MARKER = "// ------------------------------------------------------------------------------ host side"
+
+
+def device_source_sha(path: str) -> str:
+    """Hash of a kernel file's device part (everything before its host-side marker), so that
+    host-only edits keep a capture valid and any kernel edit invalidates it."""
+    import hashlib
+    text = open(path).read()
+    return hashlib.sha256(text.split(HOST_SIDE_MARKER)[0].encode()).hexdigest()[:16]
+
+
 def profile_traffic(kernel_key: str):
     """DRAM bytes per launch recorded from an ncu capture in profiles/ (None if absent or
-    if the kernel source changed since: the summary records the source hash)."""
-    import hashlib
+    if the kernel source changed since: the summary records the device-code hash)."""
     for path in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
         text = open(path).read()
         tag = "traffic[%s]:" % kernel_key
@@ -83,9 +93,7 @@ def profile_traffic(kernel_key: str):
         line = [ln for ln in text.splitlines() if ln.startswith(tag)][0]
         fields = dict(kv.split("=") for kv in line[len(tag):].split())
         src = os.path.join(ROOT, fields["source"])
-        if not os.path.exists(src):
-            return None
-        if hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] != fields["sha"]:
+        if not os.path.exists(src) or device_source_sha(src) != fields["device_sha"]:
             return None
         return float(fields["bytes"])
     return None
@@ -566,7 +574,8 @@ def _extra_pack(torch, nq, stream, steps, warm, hbm_gbs):
     us = ms * 1e3 / steps
     pbytes = 4 * rows * rr + rows * rr // 8
     del g
-    return {"us": round(us, 2), "GB_s": round(pbytes / us / 1e3, 1), "frac_hbm": round(pbytes / us / 1e3 / hbm_gbs, 4)}
+    return {"us": round(us, 2), "GB_s": round(pbytes / us / 1e3, 1), "frac_hbm": round(pbytes / us / 1e3 / hbm_gbs, 4),
+            "traffic": profile_traffic("pack_gate70b_u")}
 
 
 # --------------------------------------------------------------------------- CPU oracle

@@ -859,14 +859,17 @@ void set_attrs_once() {
 // One launch of each stage for n projections that share x (n = 1: a single layer).
 template <int NT, int GN>
 nq_status launch_decode_group_nt(const nq_lrb_layer* const* Ls, int n, const uint16_t* x, uint16_t* const* ys, int M,
-                                 void* ws, const uint16_t* cot, float* grad, cudaStream_t stream, bool pdl) {
-    // t of member l follows the earlier members' t in the workspace
+                                 void* ws, const uint16_t* cot, float* grad, cudaStream_t stream, bool pdl,
+                                 float* t_only = nullptr) {
+    // t of member l follows the earlier members' t in the workspace; with t_only (one layer),
+    // stage 1 alone runs and writes t there
     float* t[nq::kMaxGroup];
     size_t off = kWsHeader;
     for (int l = 0; l < n; ++l) {
-        t[l] = reinterpret_cast<float*>(static_cast<char*>(ws) + off);
+        t[l] = ws ? reinterpret_cast<float*>(static_cast<char*>(ws) + off) : nullptr;
         off += align256(static_cast<size_t>(M) * Ls[l]->r * sizeof(float));
     }
+    if (t_only) t[0] = t_only;
     {
         int total = 0;
         for (int l = 0; l < n; ++l) total += chunks_of(Ls[l]->r);
@@ -891,7 +894,7 @@ nq_status launch_decode_group_nt(const nq_lrb_layer* const* Ls, int n, const uin
             q.zstage = sp.zstage;
             q.upf = L->U;
             // U up to the last valid word of its last row, rounded down to 16 bytes
-            q.upf_bytes = (((L->d_out - 1) * L->ldu + L->r / 32) * 4) & ~static_cast<int64_t>(15);
+            q.upf_bytes = t_only ? 0 : (((L->d_out - 1) * L->ldu + L->r / 32) * 4) & ~static_cast<int64_t>(15);
             g.chunk_off[l] = acc;
             acc += chunks_of(L->r);
         }
@@ -906,6 +909,7 @@ nq_status launch_decode_group_nt(const nq_lrb_layer* const* Ls, int n, const uin
             cudaSuccess)
             return NQ_ERR_LAUNCH;
     }
+    if (t_only) return NQ_OK;
     {
         // the SMs are shared among the members in proportion to their weight words
         const int sms = nq_host::sm_count();
@@ -1009,6 +1013,16 @@ nq_status nq_launch_decode_group(const nq_lrb_layer* const* Ls, int n, const uin
 nq_status nq_launch_decode(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y, int64_t M, void* ws,
                            cudaStream_t stream, bool pdl, const uint16_t* cot, float* grad) {
     return nq_launch_decode_group(&L, 1, x, &y, M, ws, stream, pdl, cot, grad);
+}
+
+nq_status nq_launch_decode_stage1(const nq_lrb_layer* L, const uint16_t* x, int64_t M, float* t, cudaStream_t stream,
+                                  bool pdl) {
+    const int m = static_cast<int>(M);
+    switch (ntiles_for(M)) {
+        case 1: return launch_decode_group_nt<1, 1>(&L, 1, x, nullptr, m, nullptr, nullptr, nullptr, stream, pdl, t);
+        case 2: return launch_decode_group_nt<2, 1>(&L, 1, x, nullptr, m, nullptr, nullptr, nullptr, stream, pdl, t);
+        default: return launch_decode_group_nt<3, 1>(&L, 1, x, nullptr, m, nullptr, nullptr, nullptr, stream, pdl, t);
+    }
 }
 
 size_t nq_decode_group_workspace_bytes(const nq_lrb_layer* const* Ls, int n, int64_t M) {

@@ -79,3 +79,12 @@ size_t nq_decode_group_workspace_bytes(const nq_lrb_layer* const* Ls, int n, int
 // grad[i] = sum_m cot[m][i] (T U^T)[m][i] instead of Y.
 nq_status nq_launch_prefill(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y, int64_t M, void* ws,
                             cudaStream_t stream, bool pdl, const uint16_t* cot = nullptr, float* grad = nullptr);
+// GEMM 1 alone (prefill.cu): Z = fp16(x . s2) and T = fp16(Z V) into the workspace at the
+// offsets nq_prefill_stage1_layout gives (bytes = the extent of the region).
+void nq_prefill_stage1_layout(const nq_lrb_layer* L, int64_t M, size_t* off_z, int64_t* ldz, size_t* off_t,
+                              int64_t* ldt, size_t* bytes);
+nq_status nq_launch_prefill_stage1(const nq_lrb_layer* L, const uint16_t* x, int64_t M, void* ws, cudaStream_t stream,
+                                   bool pdl);
+// Stage 1 alone (decode.cu): t = V^T (s2 . x) [M][r] fp32 into t, M <= NQ_MATVEC_MAX_M.
+nq_status nq_launch_decode_stage1(const nq_lrb_layer* L, const uint16_t* x, int64_t M, float* t, cudaStream_t stream,
+                                  bool pdl);

@@ -61,6 +61,7 @@ __global__ void __launch_bounds__(256) pack_signs_kernel(const float* __restrict
 
 }  // namespace nq
 
+// ------------------------------------------------------------------------------ host side
 nq_status nq_launch_pack(const float* latent, int64_t rows, int64_t r, int64_t ld_latent, uint32_t* packed,
                          int64_t ld_words, cudaStream_t stream) {
     const int64_t tasks = rows * ((ld_words + 31) / 32);

@@ -592,15 +592,20 @@ nq_status launch_umma(const nq::PrefillArgs& a, const CUtensorMap& map, const CU
 
 }  // namespace
 
+namespace nq_host {
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() { return get_encode(); }
+}  // namespace nq_host
+
 size_t nq_prefill_workspace_bytes(const nq_lrb_layer* L, int64_t M) { return plan_prefill(L, M).total; }
 
-nq_status nq_launch_prefill(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y, int64_t M, void* ws,
-                            cudaStream_t stream, bool pdl, const uint16_t* cot, float* grad) {
-    const PrefillPlan p = plan_prefill(L, M);
+namespace {
+
+// Z = fp16(x . s2) and T = fp16(Z V) of layer L into the workspace ws, laid out by plan p.
+nq_status launch_stage1(const nq_lrb_layer* L, const uint16_t* x, int64_t M, void* ws, const PrefillPlan& p,
+                        cudaStream_t stream, bool pdl) {
     uint16_t* z = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + p.off_z);
     uint16_t* t = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + p.off_t);
     unsigned int* err = nq_host::error_word();
-
     {  // Z = fp16(x * s2)
         const int64_t per_row = (L->d_in % 8 == 0) ? L->d_in / 8 : L->d_in;  // work items per row
         const unsigned gx = static_cast<unsigned>(std::min<int64_t>((per_row + 255) / 256, 64));
@@ -634,9 +639,34 @@ nq_status nq_launch_prefill(const nq_lrb_layer* L, const uint16_t* x, uint16_t* 
         CUtensorMap bmap;
         std::memset(&bmap, 0, sizeof(bmap));
         a.bits_tma = make_tmap_bits(&bmap, L->V, L->d_in, L->r / 32, L->ldv, nq::kTileK) ? 1 : 0;
-        nq_status st = launch_umma<nq::kModeV>(a, map, bmap, stream, pdl);
-        if (st != NQ_OK) return st;
+        return launch_umma<nq::kModeV>(a, map, bmap, stream, pdl);
     }
+}
+
+}  // namespace
+
+void nq_prefill_stage1_layout(const nq_lrb_layer* L, int64_t M, size_t* off_z, int64_t* ldz, size_t* off_t,
+                              int64_t* ldt, size_t* bytes) {
+    const PrefillPlan p = plan_prefill(L, M);
+    *off_z = p.off_z;
+    *ldz = p.ldz;
+    *off_t = p.off_t;
+    *ldt = p.ldt;
+    *bytes = p.off_g;
+}
+
+nq_status nq_launch_prefill_stage1(const nq_lrb_layer* L, const uint16_t* x, int64_t M, void* ws, cudaStream_t stream,
+                                   bool pdl) {
+    return launch_stage1(L, x, M, ws, plan_prefill(L, M), stream, pdl);
+}
+
+nq_status nq_launch_prefill(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y, int64_t M, void* ws,
+                            cudaStream_t stream, bool pdl, const uint16_t* cot, float* grad) {
+    const PrefillPlan p = plan_prefill(L, M);
+    uint16_t* t = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + p.off_t);
+    unsigned int* err = nq_host::error_word();
+    nq_status st0 = launch_stage1(L, x, M, ws, p, stream, pdl);
+    if (st0 != NQ_OK) return st0;
     {  // Y = bf16(s1 * (T U^T)): weights = U (M-extent d_out, K = r), B = T
         const int tile_n = p.tile_n2;
         CUtensorMap map;
