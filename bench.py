@@ -498,6 +498,7 @@ def _extra_calib(torch, nq, stream, steps, warm, hbm_gbs, bf16_tf):
     out["scale_grads_prefill70b_gate_M2048"] = {"us": round(us, 2), "TFLOP_s": round(flops / us / 1e6, 2),
                                                 "frac_bf16": round(flops / us / 1e6 / bf16_tf, 4)}
     del g
+    out.update(_extra_sign_grads(torch, nq, stream, steps, warm, hbm_gbs, bf16_tf, L, p))
     # latent factors -> packed layer (balancing, scales, signs) for the 70B gate projection
     Uh = torch.randn((do, r), dtype=torch.float32, device="cuda")
     Vh = torch.randn((di, r), dtype=torch.float32, device="cuda")
@@ -508,6 +509,48 @@ def _extra_calib(torch, nq, stream, steps, warm, hbm_gbs, bf16_tf):
     out["from_latent_70b_gate"] = {"us": round(us, 2), "GB_s": round(moved / us / 1e3, 1),
                                    "frac_hbm": round(moved / us / 1e3 / hbm_gbs, 4)}
     del g
+    return out
+
+
+def _extra_sign_grads(torch, nq, stream, steps, warm, hbm_gbs, bf16_tf, L70, p70):
+    """Gradients with respect to the sign factors (the refinement step's straight-through
+    backward): the 7B attention shape at batch 1 (distinct layer instances, one fp32 gradient
+    pair of 2 x 4096 x 2048 written per call) and the 70B gate at M = 64 and 2048."""
+    out = {}
+    (_, do, di, r), = synth.WORKLOADS[HEADLINE]
+    ch = Chain(torch, nq, do, di, r, 1, 16, seed=synth.workload_seed(HEADLINE) + 90)
+    ybar = torch.zeros((1, do), dtype=torch.bfloat16, device="cuda").normal_()
+    gU = torch.empty((do, r), dtype=torch.float32, device="cuda")
+    gV = torch.empty((di, r), dtype=torch.float32, device="cuda")
+    ws = torch.empty(nq.sign_grads_workspace_bytes(ch.layers[0], 1), dtype=torch.uint8, device="cuda")
+
+    def run():
+        for Lc in ch.layers:
+            nq.lrb_sign_grads(Lc, ch.x0, ybar, gU=gU, gV=gV, ws=ws, stream=stream)
+    g = graph_of(torch, run, stream)
+    ms = timed_replays(torch, g, stream, steps, warm)
+    us = ms * 1e3 / (steps * ch.n)
+    moved = r * (do + di) // 8 + 4 * r * (do + di) + 2 * (do + di) + 4 * (do + di)  # bits, fp32 out, scales, acts
+    out["sign_grads_attn7b_b1"] = {"us_per_layer": round(us, 3), "GB_s": round(moved / us / 1e3, 1),
+                                   "frac_hbm": round(moved / us / 1e3 / hbm_gbs, 4),
+                                   "note": "16 distinct layers; output 2 x 32 MB fp32 per call"}
+    del g, ch
+    (_, do, di, r), = synth.WORKLOADS["prefill70b"]
+    gU = torch.empty((do, r), dtype=torch.float32, device="cuda")
+    gV = torch.empty((di, r), dtype=torch.float32, device="cuda")
+    for M in (64, 2048):
+        x = torch.zeros((M, di), dtype=torch.bfloat16, device="cuda").normal_()
+        ybar = torch.zeros((M, do), dtype=torch.bfloat16, device="cuda").normal_()
+        ws = torch.empty(nq.sign_grads_workspace_bytes(L70, M), dtype=torch.uint8, device="cuda")
+        g = graph_of(torch, lambda: nq.lrb_sign_grads(L70, x, ybar, gU=gU, gV=gV, ws=ws, stream=stream), stream)
+        ms = timed_replays(torch, g, stream, 3, 2)
+        us = ms * 1e3 / 3
+        flops = 4.0 * M * r * (di + do)  # two GEMM 1 passes and the two outer products
+        wbytes = 4 * r * (do + di)
+        out["sign_grads_prefill70b_gate_M%d" % M] = {
+            "us": round(us, 2), "TFLOP_s": round(flops / us / 1e6, 2), "frac_bf16": round(flops / us / 1e6 / bf16_tf, 4),
+            "out_GB_s": round(wbytes / us / 1e3, 1), "out_frac_hbm": round(wbytes / us / 1e3 / hbm_gbs, 4)}
+        del g
     return out
 
 

@@ -189,6 +189,29 @@ NQ_API nq_status nq_lrb_scale_grads(const nq_lrb_layer* L, const uint16_t* x, co
                                     float* g_s1, float* g_s2, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Gradients with respect to the sign factors.  Page "NanoQuant: Efficient Sub-1-Bit
+ * Quantization of Large Language Models", section 3, "Step 3: Factorized Component
+ * Refinement": the latent factors are refined through sign() with straight-through
+ * estimators.  For L = sum_m sum_i ybar[m][i] y[m][i] (y = the layer applied to x):
+ *   gU[i][k] = dL/dU_ik = s1_i sum_m ybar[m][i] t[m][k],  t[m] = V^T (s2 . x[m])
+ *   gV[j][k] = dL/dV_jk = s2_j sum_m x[m][j]    u[m][k],  u[m] = U^T (s1 . ybar[m])
+ * The identity straight-through estimator passes these to the latent entries unchanged
+ * (the pages name no variant); a clipped estimator is the caller's mask on gU, gV.
+ *   x [M][d_in], ybar [M][d_out] bf16; gU [d_out][ldgu] and gV [d_in][ldgv] fp32, columns
+ *   0..r-1 overwritten, pad columns untouched.  ldgu, ldgv >= r and multiples of 4; gU, gV
+ *   16-byte aligned (NQ_ERR_ALIGN otherwise).
+ *   M <= NQ_MATVEC_MAX_M: t and u from the decode stage 1 (exact integer sums of the 23-bit
+ *   quantised activations, fp32), the sum over m in fp32 on the CUDA cores.  Larger M: t and u
+ *   from the tensor-core GEMM 1 (fp16 operands s2 . x and s1 . ybar, fp16 t, u), the sum over
+ *   m on the tensor cores (fp16 operands, fp32 accumulation).
+ *   ws: nq_sign_grads_workspace_bytes(L, M) bytes (0 for an invalid layer or M < 1).
+ */
+NQ_API size_t nq_sign_grads_workspace_bytes(const nq_lrb_layer* L, int64_t M);
+NQ_API nq_status nq_lrb_sign_grads(const nq_lrb_layer* L, const uint16_t* x, const uint16_t* ybar, int64_t M,
+                                   float* gU, int64_t ldgu, float* gV, int64_t ldgv, void* ws, size_t ws_bytes,
+                                   void* stream);
+
+/*
  * nq_layer_forward_group -- y[l] = layer l applied to x, for 1 <= n <= NQ_MAX_GROUP projections
  * that share their input (a transformer's q, k, v, or its gate and up): every layer must have
  * the same d_in; d_out and r may differ.  For M <= NQ_MATVEC_MAX_M the group runs as one

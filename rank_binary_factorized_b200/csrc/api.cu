@@ -20,6 +20,10 @@ size_t nq_from_latent_ws(int64_t d_out, int64_t d_in, int64_t ldu, int64_t ldv);
 nq_status nq_launch_from_latent(const float* Uh, int64_t ld_uh, const float* Vh, int64_t ld_vh, int64_t d_out,
                                 int64_t d_in, int64_t r, uint32_t* U, int64_t ldu, uint32_t* V, int64_t ldv,
                                 uint16_t* s1, uint16_t* s2, double* eta, void* ws, cudaStream_t stream);
+size_t nq_sign_grads_ws(const nq_lrb_layer* L, const nq_lrb_layer* X, int64_t M);
+nq_status nq_launch_sign_grads(const nq_lrb_layer* L, const nq_lrb_layer* X, const uint16_t* x, const uint16_t* ybar,
+                               int64_t M, float* gU, int64_t ldgu, float* gV, int64_t ldgv, void* ws,
+                               cudaStream_t stream, bool pdl);
 
 namespace {
 
@@ -299,6 +303,29 @@ nq_status nq_lrb_scale_grads(const nq_lrb_layer* L, const uint16_t* x, const uin
     }
     if ((st = nq_launch_prefill(L, x, nullptr, M, ws, s, pdl, ybar, g_s1)) != NQ_OK) return st;
     return nq_launch_prefill(&T, ybar, nullptr, M, ws, s, pdl, x, g_s2);
+}
+
+size_t nq_sign_grads_workspace_bytes(const nq_lrb_layer* L, int64_t M) {
+    if (check_layer(L) != NQ_OK || M < 1) return 0;
+    const nq_lrb_layer T = exchanged(L);
+    return nq_sign_grads_ws(L, &T, M);
+}
+
+nq_status nq_lrb_sign_grads(const nq_lrb_layer* L, const uint16_t* x, const uint16_t* ybar, int64_t M, float* gU,
+                            int64_t ldgu, float* gV, int64_t ldgv, void* ws, size_t ws_bytes, void* stream) {
+    nq_status st = check_layer(L);
+    if (st != NQ_OK) return st;
+    if (M < 1) return NQ_ERR_SHAPE;
+    if ((st = check_io(x, ybar, ws)) != NQ_OK) return st;
+    if (!gU || !gV) return NQ_ERR_NULL;
+    if (ldgu < L->r || ldgv < L->r) return NQ_ERR_SHAPE;
+    if (!aligned16(gU) || !aligned16(gV) || (ldgu % 4) != 0 || (ldgv % 4) != 0) return NQ_ERR_ALIGN;
+    const nq_lrb_layer T = exchanged(L);
+    if (ws_bytes < nq_sign_grads_ws(L, &T, M)) return NQ_ERR_WORKSPACE;
+    DeviceInfo* d = current_device();
+    if (!d || !d->ok) return NQ_ERR_DEVICE;
+    return nq_launch_sign_grads(L, &T, x, ybar, M, gU, ldgu, gV, ldgv, ws, static_cast<cudaStream_t>(stream),
+                                pdl_enabled());
 }
 
 size_t nq_from_latent_workspace_bytes(int64_t d_out, int64_t d_in, int64_t r, int64_t ldu, int64_t ldv) {

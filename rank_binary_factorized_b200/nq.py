@@ -64,6 +64,11 @@ _lib.nq_layer_forward_group.argtypes = [ctypes.POINTER(ctypes.POINTER(nq_lrb_lay
 _lib.nq_lrb_scale_grads.restype = ctypes.c_int
 _lib.nq_lrb_scale_grads.argtypes = [ctypes.POINTER(nq_lrb_layer), _p, _p, _i64, _p, _p, _p, ctypes.c_size_t, _p]
 _lib.nq_sync_status.restype = ctypes.c_int
+_lib.nq_sign_grads_workspace_bytes.restype = ctypes.c_size_t
+_lib.nq_sign_grads_workspace_bytes.argtypes = [ctypes.POINTER(nq_lrb_layer), _i64]
+_lib.nq_lrb_sign_grads.restype = ctypes.c_int
+_lib.nq_lrb_sign_grads.argtypes = [ctypes.POINTER(nq_lrb_layer), _p, _p, _i64, _p, _i64, _p, _i64, _p, ctypes.c_size_t,
+                                   _p]
 _lib.nq_sync_status.argtypes = [_p]
 _lib.nq_status_string.restype = ctypes.c_char_p
 _lib.nq_status_string.argtypes = [ctypes.c_int]
@@ -214,6 +219,34 @@ def lrb_scale_grads(layer: Layer, x: torch.Tensor, ybar: torch.Tensor, ws=None, 
                                                          _ptr(g1), _ptr(g2), _ptr(ws), ws.numel(),
                                                          _stream_ptr(stream)))
     return g1, g2
+
+
+def sign_grads_workspace_bytes(layer: Layer, M: int) -> int:
+    n = int(_lib.nq_sign_grads_workspace_bytes(ctypes.byref(layer.struct), int(M)))
+    if n == 0:
+        raise NQError("nq_sign_grads_workspace_bytes", 2)
+    return n
+
+
+def lrb_sign_grads(layer: Layer, x: torch.Tensor, ybar: torch.Tensor, gU=None, gV=None, ws=None, stream=None):
+    """(dL/dU [d_out][r], dL/dV [d_in][r]) fp32 for L = sum <ybar, layer(x)>: the gradients the
+    identity straight-through estimator passes to the latent factors.  gU, gV may be given
+    ([rows][ld] fp32 with ld >= r a multiple of 4); only their first r columns are written."""
+    M = int(x.shape[0])
+    r = layer.r
+    if gU is None:
+        gU = torch.empty((layer.d_out, r), dtype=torch.float32, device=x.device)
+    if gV is None:
+        gV = torch.empty((layer.d_in, r), dtype=torch.float32, device=x.device)
+    for g in (gU, gV):
+        if g.dtype != torch.float32 or g.dim() != 2 or g.stride(1) != 1:
+            raise ValueError("gradients must be 2-D float32 with unit column stride")
+    if ws is None:
+        ws = torch.empty(sign_grads_workspace_bytes(layer, M), dtype=torch.uint8, device=x.device)
+    _check("nq_lrb_sign_grads", _lib.nq_lrb_sign_grads(ctypes.byref(layer.struct), _ptr(x), _ptr(ybar), M, _ptr(gU),
+                                                       gU.stride(0), _ptr(gV), gV.stride(0), _ptr(ws), ws.numel(),
+                                                       _stream_ptr(stream)))
+    return gU, gV
 
 
 def lrb_from_latent(Uh: torch.Tensor, Vh: torch.Tensor, r: int | None = None, ld_align_words: int = 4,

@@ -98,6 +98,31 @@ def test_scale_grads_argument_errors(nq):
     assert call(_layer(nq), ws_bytes=16) == NQ["WORKSPACE"]
 
 
+def test_sign_grads_argument_errors(nq):
+    lib = nq.raw_lib()
+
+    def call(L, x=0x50000, ybar=0x60000, M=1, gU=0x80000, ldgu=64, gV=0x90000, ldgv=64, ws=0x70000, ws_bytes=1 << 30):
+        return lib.nq_lrb_sign_grads(ctypes.byref(L) if L is not None else None, x, ybar, M, gU, ldgu, gV, ldgv, ws,
+                                     ws_bytes, None)
+
+    assert call(None) == NQ["NULL"]
+    assert call(_layer(nq, U=0)) == NQ["NULL"]
+    assert call(_layer(nq), x=0) == NQ["NULL"]
+    assert call(_layer(nq), gU=0) == NQ["NULL"]
+    assert call(_layer(nq), gV=0) == NQ["NULL"]
+    assert call(_layer(nq, r=48)) == NQ["SHAPE"]
+    assert call(_layer(nq), M=0) == NQ["SHAPE"]
+    assert call(_layer(nq), ldgu=32) == NQ["SHAPE"]  # below r
+    assert call(_layer(nq), ldgv=60) == NQ["SHAPE"]
+    assert call(_layer(nq), ldgu=66) == NQ["ALIGN"]  # row stride not a multiple of 16 bytes
+    assert call(_layer(nq), gV=0x90008) == NQ["ALIGN"]
+    assert call(_layer(nq), ws_bytes=16) == NQ["WORKSPACE"]
+    for M in (1, 8, 9, 2048):
+        assert lib.nq_sign_grads_workspace_bytes(ctypes.byref(_layer(nq, d_out=28672, d_in=8192, r=3520)), M) > 0
+    assert lib.nq_sign_grads_workspace_bytes(ctypes.byref(_layer(nq)), 0) == 0
+    assert lib.nq_sign_grads_workspace_bytes(ctypes.byref(_layer(nq, r=48)), 1) == 0
+
+
 def test_workspace_covers_both_directions(nq):
     """One workspace serves the forward product, the transpose and the scale gradients: the
     size is the same for a layer and for the layer with its two sides exchanged."""
