@@ -66,6 +66,11 @@ struct PrefillArgs {
     const uint16_t* cot;   // [M][ldcot] bf16
     int64_t ldcot;
     double* gpart;         // [n_tiles_n][rows_w]
+    // split over K (mode V with bits_tma only): every tile's k blocks are divided among ksplit
+    // work units, each writing its fp32 partial product to partial[split][M][ldo]; a reduction
+    // kernel then adds the splits in order and rounds to fp16
+    int ksplit;
+    float* partial;
 };
 
 // fp16 +1 = 0x3C00, -1 = 0xBC00; two elements per 32-bit word, element 2i in the low half.
@@ -144,6 +149,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int n_tiles = args.n_tiles_w * args.n_tiles_n;
     const int nkb = args.n_kblocks;
     unsigned int* err = args.err;
+    // work unit u: tile u / ksplit, k blocks [kb_lo, kb_hi) of split u % ksplit
+    const int ksplit = (MODE == kModeV) ? args.ksplit : 1;
+    const int n_units = n_tiles * ksplit;
+    auto unit_kb = [&](int u, int& kb_lo, int& kb_hi) {
+        const int sp = u % ksplit;
+        kb_lo = sp * nkb / ksplit;
+        kb_hi = (sp + 1) * nkb / ksplit;
+    };
 
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA producer (B)
@@ -152,15 +165,18 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             // waiting for the activations (the stage's barrier also waits for its B tile)
             uint32_t pre = 0;
             if (args.bits_tma) {
-                int tile = blockIdx.x, kb = 0;
-                while (tile < n_tiles && pre < static_cast<uint32_t>(stages)) {
-                    const int tw = tile % args.n_tiles_w;
+                int u = blockIdx.x, kb = 0, kb_lo = 0, kb_hi = nkb;
+                if (u < n_units) unit_kb(u, kb_lo, kb_hi);
+                kb = kb_lo;
+                while (u < n_units && pre < static_cast<uint32_t>(stages)) {
+                    const int tw = (u / ksplit) % args.n_tiles_w;
                     tc::mbar_expect_tx(full_b(pre), bits_bytes);
                     tc::tma_load_2d(bits_tile(pre), &tmap_bits, bits_x(tw, kb), bits_y(tw, kb), full_b(pre));
                     ++pre;
-                    if (++kb == nkb) {
-                        kb = 0;
-                        tile += gridDim.x;
+                    if (++kb == kb_hi) {
+                        u += gridDim.x;
+                        if (u < n_units) unit_kb(u, kb_lo, kb_hi);
+                        kb = kb_lo;
                     }
                 }
             }
@@ -168,10 +184,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             uint32_t it = 0, ph = 0;
             int s = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+            for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+                const int tile = u / ksplit;
                 const int tn = tile / args.n_tiles_w;
                 const int tw = tile - tn * args.n_tiles_w;
-                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                int kb_lo, kb_hi;
+                unit_kb(u, kb_lo, kb_hi);
+                for (int kb = kb_lo; kb < kb_hi; ++kb, ++it) {
                     if (!(ok = tc::mbar_wait(empty(s), ph ^ 1u, err))) break;
                     if (args.bits_tma && it >= pre) {
                         tc::mbar_expect_tx(full_b(s), bits_bytes);
@@ -197,13 +216,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             uint32_t tc_count = 0, ph = 0;
             int s = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++tc_count) {
+            for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++tc_count) {
                 const int acc = tc_count & 1;
                 const uint32_t aph = (tc_count >> 1) & 1u;
                 if (!(ok = tc::mbar_wait(acc_empty(acc), aph ^ 1u, err))) break;
                 tc::tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * 256);
-                for (int kb = 0; kb < nkb; ++kb) {
+                int kb_lo, kb_hi;
+                unit_kb(u, kb_lo, kb_hi);
+                for (int kb = kb_lo; kb < kb_hi; ++kb) {
                     if (!(ok = tc::mbar_wait(full_a(s), ph, err))) break;
                     if (!(ok = tc::mbar_wait(full_b(s), ph, err))) break;
                     tc::tc_fence_after();
@@ -218,7 +239,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                             adesc = tc::smem_desc_sw128(a_tile(s) + kk * 32u, 16u, 1024u);
                         }
                         const uint64_t bdesc = tc::smem_desc_sw128(b_tile(s) + kk * 32u, 16u, 1024u);
-                        tc::mma_f16_ss(d_tmem, adesc, bdesc, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+                        tc::mma_f16_ss(d_tmem, adesc, bdesc, idesc, (kb > kb_lo || kk > 0) ? 1u : 0u);
                     }
                     tc::mma_commit(empty(s));
                     if (++s == stages) {
@@ -294,7 +315,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         constexpr int kPrefetch = 8;
         uint2 ring[kPrefetch];
         const int my_tiles = (n_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x);
-        const uint32_t total_it = static_cast<uint32_t>(my_tiles > 0 ? my_tiles : 0) * static_cast<uint32_t>(nkb);
+        uint32_t total_it = static_cast<uint32_t>(my_tiles > 0 ? my_tiles : 0) * static_cast<uint32_t>(nkb);
+        if (ksplit > 1) {  // the k blocks of this CTA's work units
+            total_it = 0;
+            for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+                int kb_lo, kb_hi;
+                unit_kb(u, kb_lo, kb_hi);
+                total_it += static_cast<uint32_t>(kb_hi - kb_lo);
+            }
+        }
         // this thread's 128-byte smem row within a stage's A tile, and its swizzle
         const uint32_t row_off_b = (MODE == kModeU) ? (tg >> 3) * 1024u + (tg & 7) * 128u
                                                     : ((jl >> 3) * 2 + hgrp) * 1024u + (jl & 7) * 128u;
@@ -357,9 +386,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const int rl = q * 32 + lane;  // accumulator row (TMEM lane)
         uint32_t tc_count = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++tc_count) {
+        for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++tc_count) {
+            const int tile = u / ksplit;
             const int tw = tile % args.n_tiles_w;
             const int tn = tile / args.n_tiles_w;
+            float* part = (ksplit > 1) ? args.partial + static_cast<int64_t>(u % ksplit) * args.M * args.ldo : nullptr;
             const int acc = tc_count & 1;
             const uint32_t aph = (tc_count >> 1) & 1u;
             if (!(ok = tc::mbar_wait(acc_full(acc), aph, err))) break;
@@ -384,6 +415,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                                 g += static_cast<double>(bf16_bits_to_float(args.cot[tok * args.ldcot + wrow])) * f;
                             } else if (MODE == kModeU) {
                                 static_cast<uint16_t*>(args.out)[tok * args.ldo + wrow] = float_to_bf16_bits(scale * f);
+                            } else if (part) {
+                                part[tok * args.ldo + wrow] = f;
                             } else {
                                 static_cast<uint16_t*>(args.out)[tok * args.ldo + wrow] =
                                     __half_as_ushort(__float2half_rn(f));
@@ -443,6 +476,33 @@ __global__ void __launch_bounds__(256) scale_convert_kernel(const uint16_t* __re
     }
 }
 
+// T[m][k] = fp16( sum over splits s = 0 .. S-1, in order, of partial[s][m][k] ) for k < r;
+// four k per thread (r % 32 == 0 and ldt % 8 == 0: 16-byte loads, 8-byte stores).
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restrict__ partial, int S, int64_t M,
+                                                           int64_t r, int64_t ldt, uint16_t* __restrict__ t) {
+    pdl_wait();
+    const int64_t per_row = r / 4;
+    const int64_t n = M * per_row;
+    for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < n;
+         e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t m = e / per_row, k = (e - m * per_row) * 4;
+        float4 acc = *reinterpret_cast<const float4*>(partial + m * ldt + k);
+        for (int sp = 1; sp < S; ++sp) {
+            const float4 v = *reinterpret_cast<const float4*>(partial + (static_cast<int64_t>(sp) * M + m) * ldt + k);
+            acc.x += v.x;
+            acc.y += v.y;
+            acc.z += v.z;
+            acc.w += v.w;
+        }
+        uint2 o;
+        o.x = static_cast<uint32_t>(__half_as_ushort(__float2half_rn(acc.x))) |
+              (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(acc.y))) << 16);
+        o.y = static_cast<uint32_t>(__half_as_ushort(__float2half_rn(acc.z))) |
+              (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(acc.w))) << 16);
+        *reinterpret_cast<uint2*>(t + m * ldt + k) = o;
+    }
+}
+
 // grad[i] = sum over token tiles tn (in order) of gpart[tn][i], fp64, rounded to fp32.
 __global__ void __launch_bounds__(256) grad_reduce_kernel(const double* __restrict__ gpart, int64_t n_tiles,
                                                          int64_t rows, float* __restrict__ grad) {
@@ -466,8 +526,30 @@ int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
 struct PrefillPlan {
     int64_t ldz, ldt;
     int tile_n1, tile_n2;  // token tiles of GEMM 1 and GEMM 2
-    size_t off_z, off_t, off_g, total;
+    int ksplit1;           // K splits of GEMM 1 (when its packed signs arrive by TMA)
+    size_t off_z, off_t, off_p, off_g, total;
 };
+
+// K splits for a GEMM of `tiles` output tiles over nkb k blocks: the fewest k-block steps on
+// the busiest SM, counted as waves x (k blocks per unit + 2 for the unit's pipeline fill and
+// drain), plus the fp32 partials' extra traffic (written once, read once; about 2.25 MB per
+// k-block step of time).  Every unit keeps at least 4 k blocks.
+int choose_ksplit(int64_t tiles, int64_t nkb, int64_t M, int64_t r, int sms) {
+    int best = 1;
+    double best_cost = -1.0;
+    const int64_t top = std::min<int64_t>(16, nkb / 4);
+    for (int64_t S = 1; S <= std::max<int64_t>(1, top); ++S) {
+        const int64_t waves = (tiles * S + sms - 1) / sms;
+        const int64_t per = (nkb + S - 1) / S;
+        const double extra = (S > 1) ? static_cast<double>(S) * M * r * 8 / 2.25e6 : 0.0;
+        const double cost = static_cast<double>(waves * (per + 2)) + extra;
+        if (best_cost < 0.0 || cost < best_cost) {
+            best_cost = cost;
+            best = static_cast<int>(S);
+        }
+    }
+    return best;
+}
 
 // Tokens per tile (MMA N, a multiple of 16 up to 256) for a GEMM with n_tiles_w weight tiles:
 // the fewest waves of persistent tiles over the SMs, each wave costing about max(N, 192) + 64
@@ -498,7 +580,10 @@ PrefillPlan plan_prefill(const nq_lrb_layer* L, int64_t M) {
     p.ldt = round_up(L->r, 8);
     p.off_z = NQ_WS_HEADER_BYTES;  // past the reserved workspace header
     p.off_t = p.off_z + align256(static_cast<size_t>(M * p.ldz) * 2);
-    p.off_g = p.off_t + align256(static_cast<size_t>(M * p.ldt) * 2);
+    p.off_p = p.off_t + align256(static_cast<size_t>(M * p.ldt) * 2);
+    const int64_t tiles1 = ((L->r + nq::kTileW - 1) / nq::kTileW) * ((M + p.tile_n1 - 1) / p.tile_n1);
+    p.ksplit1 = choose_ksplit(tiles1, (L->d_in + nq::kTileK - 1) / nq::kTileK, M, L->r, sms);
+    p.off_g = p.off_p + (p.ksplit1 > 1 ? align256(static_cast<size_t>(p.ksplit1) * M * p.ldt * 4) : 0);
     // gradient mode: fp64 partial per (token tile of GEMM 2, row)
     const int64_t n_tn2 = (M + p.tile_n2 - 1) / p.tile_n2;
     p.total = p.off_g + align256(static_cast<size_t>(n_tn2 * L->d_out) * sizeof(double));
@@ -576,9 +661,9 @@ nq_status launch_umma(const nq::PrefillArgs& a, const CUtensorMap& map, const CU
             return NQ_ERR_LAUNCH;
         attr_done[dev] = true;
     }
-    const int tiles = a.n_tiles_w * a.n_tiles_n;
+    const int units = a.n_tiles_w * a.n_tiles_n * ((MODE == nq::kModeV && a.ksplit > 1) ? a.ksplit : 1);
     int grid = nq_host::sm_count();
-    if (grid > tiles) grid = tiles;
+    if (grid > units) grid = units;
     nq::PrefillArgs args = a;
     args.stages = umma_stages(a.tile_n);
     CUtensorMap tm = map, tb = bits_map;
@@ -639,7 +724,21 @@ nq_status launch_stage1(const nq_lrb_layer* L, const uint16_t* x, int64_t M, voi
         CUtensorMap bmap;
         std::memset(&bmap, 0, sizeof(bmap));
         a.bits_tma = make_tmap_bits(&bmap, L->V, L->d_in, L->r / 32, L->ldv, nq::kTileK) ? 1 : 0;
-        return launch_umma<nq::kModeV>(a, map, bmap, stream, pdl);
+        a.ksplit = a.bits_tma ? p.ksplit1 : 1;
+        a.partial = a.ksplit > 1 ? reinterpret_cast<float*>(static_cast<char*>(ws) + p.off_p) : nullptr;
+        nq_status st = launch_umma<nq::kModeV>(a, map, bmap, stream, pdl);
+        if (st != NQ_OK || a.ksplit == 1) return st;
+        // T = fp16 of the splits' sum, in split order
+        const float* part = a.partial;
+        int S = a.ksplit;
+        int64_t r = L->r, ldt = p.ldt;
+        const int64_t items = M * (r / 4);
+        const unsigned blocks = static_cast<unsigned>(std::min<int64_t>((items + 255) / 256, 8LL * nq_host::sm_count()));
+        void* args[] = {&part, &S, &M, &r, &ldt, &t};
+        return nq_host::launch_pdl(reinterpret_cast<const void*>(nq::splitk_reduce_kernel), dim3(blocks), dim3(256), 0,
+                                   stream, args, pdl) == cudaSuccess
+                   ? NQ_OK
+                   : NQ_ERR_LAUNCH;
     }
 }
 
