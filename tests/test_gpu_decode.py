@@ -20,8 +20,8 @@ from tests.gpu_util import (check_tolerance, download_bf16_bits, need_gpu, nq, u
 pytestmark = pytest.mark.gpu
 
 
-def gpu_forward(p, xb, fn="lrb_matvec"):
-    L = upload_projection(p)
+def gpu_forward(p, xb, fn="lrb_matvec", ld_align_words=4):
+    L = upload_projection(p, ld_align_words=ld_align_words)
     x = upload_bf16(xb)
     y = getattr(nq(), fn)(L, x)
     nq().sync_status()
@@ -46,11 +46,12 @@ def test_tiny_all_batches(M):
     (300, 2049, 320, 10, 10, 2),
     (5, 4097, 32, 4, 4, 6),
 ])
-def test_ragged_and_padded(d_out, d_in, r, ldu, ldv, M):
+@pytest.mark.parametrize("align", [1, 4])  # rows kept at ldu (plain copies) or padded to 16 bytes (bulk copies)
+def test_ragged_and_padded(d_out, d_in, r, ldu, ldv, M, align):
     need_gpu()
     p = synth.make_projection("ragged", d_out, d_in, r, seed=202, key=d_out * 7 + d_in, ldu=ldu, ldv=ldv)
     xb = synth.acts_bf16(synth.rng_for(203, d_in), (M, d_in))
-    y = gpu_forward(p, xb)
+    y = gpu_forward(p, xb, ld_align_words=align)
     y_ref, S = oracle.dense_packed(p.U, p.V, p.s1, p.s2, p.r, xb)
     check_tolerance(y, y_ref, S, "ragged %r" % ((d_out, d_in, r, ldu, ldv, M),))
 
