@@ -48,7 +48,7 @@ def parse_args():
     ap.add_argument("--headline-only", action="store_true", help="skip the other workloads")
     ap.add_argument("--only", default=None,
                     help="run just these extra sections (comma list of attn7b_b8, mlp7b, layer70b, prefill, pack, "
-                         "calib, model70b) "
+                         "calib, signgrad, model70b) "
                          "after the headline; implies no CPU baseline")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU oracle sample budget")
     return ap.parse_args()
@@ -370,6 +370,8 @@ def extras(torch, nq, stream, args, hbm_gbs, bf16_tf, bf16_tf_sus, peak_src):
         out["pack_70b_gate_U"] = _extra_pack(torch, nq, stream, steps, warm, hbm_gbs)
     if on("calib"):
         out.update(_extra_calib(torch, nq, stream, steps, warm, hbm_gbs, bf16_tf))
+    if on("signgrad"):
+        out.update(_extra_sign_grads(torch, nq, stream, steps, warm, hbm_gbs, bf16_tf))
     if on("model70b"):
         out["model70b_decode_b1"] = _extra_model70b(torch, nq, stream, hbm_gbs)
     nq.sync_status(stream)
@@ -498,7 +500,6 @@ def _extra_calib(torch, nq, stream, steps, warm, hbm_gbs, bf16_tf):
     out["scale_grads_prefill70b_gate_M2048"] = {"us": round(us, 2), "TFLOP_s": round(flops / us / 1e6, 2),
                                                 "frac_bf16": round(flops / us / 1e6 / bf16_tf, 4)}
     del g
-    out.update(_extra_sign_grads(torch, nq, stream, steps, warm, hbm_gbs, bf16_tf, L, p))
     # latent factors -> packed layer (balancing, scales, signs) for the 70B gate projection
     Uh = torch.randn((do, r), dtype=torch.float32, device="cuda")
     Vh = torch.randn((di, r), dtype=torch.float32, device="cuda")
@@ -512,7 +513,7 @@ def _extra_calib(torch, nq, stream, steps, warm, hbm_gbs, bf16_tf):
     return out
 
 
-def _extra_sign_grads(torch, nq, stream, steps, warm, hbm_gbs, bf16_tf, L70, p70):
+def _extra_sign_grads(torch, nq, stream, steps, warm, hbm_gbs, bf16_tf):
     """Gradients with respect to the sign factors (the refinement step's straight-through
     backward): the 7B attention shape at batch 1 (distinct layer instances, one fp32 gradient
     pair of 2 x 4096 x 2048 written per call) and the 70B gate at M = 64 and 2048."""
@@ -536,6 +537,8 @@ def _extra_sign_grads(torch, nq, stream, steps, warm, hbm_gbs, bf16_tf, L70, p70
                                    "note": "16 distinct layers; output 2 x 32 MB fp32 per call"}
     del g, ch
     (_, do, di, r), = synth.WORKLOADS["prefill70b"]
+    p70 = synth.make_projection("gate", do, di, r, seed=synth.workload_seed("prefill70b"))
+    L70 = nq.Layer.from_host(p70.U, p70.V, p70.s1, p70.s2, r)
     gU = torch.empty((do, r), dtype=torch.float32, device="cuda")
     gV = torch.empty((di, r), dtype=torch.float32, device="cuda")
     for M in (64, 2048):
@@ -549,7 +552,8 @@ def _extra_sign_grads(torch, nq, stream, steps, warm, hbm_gbs, bf16_tf, L70, p70
         wbytes = 4 * r * (do + di)
         out["sign_grads_prefill70b_gate_M%d" % M] = {
             "us": round(us, 2), "TFLOP_s": round(flops / us / 1e6, 2), "frac_bf16": round(flops / us / 1e6 / bf16_tf, 4),
-            "out_GB_s": round(wbytes / us / 1e3, 1), "out_frac_hbm": round(wbytes / us / 1e3 / hbm_gbs, 4)}
+            "out_GB_s": round(wbytes / us / 1e3, 1), "out_frac_hbm": round(wbytes / us / 1e3 / hbm_gbs, 4),
+            "traffic": profile_traffic("sign_grads_umma_gate70b_m%d" % M)}
         del g
     return out
 

@@ -818,11 +818,13 @@ int chunks_of(int64_t r) { return static_cast<int>((r / 32 + nq::kS1Words - 1) /
 // Stage-1 shape for a grid of `total_chunks` word chunks over d_in rows: the cluster size CS
 // (row slices per chunk) shrinks as the chunk count grows, so that the grid stays near one
 // block per SM; rows per slice and the staging pass follow.
-S1Plan plan_stage1(int64_t d_in, int total_chunks, int64_t M) {
+// A given cluster size (force_cs > 0) replaces the choice, for members of one grid.
+S1Plan plan_stage1(int64_t d_in, int total_chunks, int64_t M, int force_cs = 0) {
     S1Plan p{};
     p.n_chunks = total_chunks;
     int cs = total_chunks <= 8 ? 16 : (total_chunks <= 18 ? 8 : (total_chunks <= 37 ? 4 : 2));
     while (cs > 1 && static_cast<int64_t>(cs) * 32 > d_in) cs >>= 1;
+    if (force_cs > 0) cs = force_cs;
     p.CS = cs;
     p.rows_per_slice = static_cast<int>(((d_in + cs - 1) / cs + 31) / 32 * 32);
     const int nt = ntiles_for(M);
@@ -974,6 +976,54 @@ nq_status launch_decode_group_nt(const nq_lrb_layer* const* Ls, int n, const uin
     return NQ_OK;
 }
 
+// Stage 1 alone for two layers with their own inputs and d_in (a layer and its exchanged form,
+// say), as one grid: t0 = V0^T (s2_0 . x0), t1 = V1^T (s2_1 . x1).  The members share the
+// cluster size (the smaller of their own choices); each keeps its own row slices.
+template <int NT>
+nq_status launch_stage1_pair_nt(const nq_lrb_layer* L0, const uint16_t* x0, float* t0, const nq_lrb_layer* L1,
+                                const uint16_t* x1, float* t1, int M, cudaStream_t stream, bool pdl) {
+    const nq_lrb_layer* Ls[2] = {L0, L1};
+    const uint16_t* xs[2] = {x0, x1};
+    float* ts[2] = {t0, t1};
+    const int total = chunks_of(L0->r) + chunks_of(L1->r);
+    const int cs = std::min(plan_stage1(L0->d_in, total, M).CS, plan_stage1(L1->d_in, total, M).CS);
+    S1Plan sp[2] = {plan_stage1(L0->d_in, total, M, cs), plan_stage1(L1->d_in, total, M, cs)};
+    nq::S1Group g{};
+    g.n = 2;
+    int acc = 0;
+    for (int l = 0; l < 2; ++l) {
+        const nq_lrb_layer* L = Ls[l];
+        nq::S1Params& q = g.p[l];
+        q.V = L->V;
+        q.ldv = L->ldv;
+        q.s2 = L->s2;
+        q.x = xs[l];
+        q.t = ts[l];
+        q.M = M;
+        q.d_in = L->d_in;
+        q.r = static_cast<int>(L->r);
+        q.nw = static_cast<int>(L->r / 32);
+        q.rows_per_slice = sp[l].rows_per_slice;
+        q.jc_rows = sp[l].jc_rows;
+        q.zstage = sp[l].zstage;
+        q.upf = L->U;
+        q.upf_bytes = 0;
+        g.chunk_off[l] = acc;
+        acc += chunks_of(L->r);
+    }
+    g.chunk_off[2] = acc;
+    void* args[] = {&g};
+    const size_t smem = std::max(sp[0].smem, sp[1].smem);
+    const bool wide = (NT <= 2) && std::max(sp[0].rows_per_slice, sp[1].rows_per_slice) >= 1024;
+    const void* fn = wide ? reinterpret_cast<const void*>(nq::decode_stage1_kernel<NT, (NT <= 2 ? 512 : 256), nq::kMaxGroup>)
+                          : reinterpret_cast<const void*>(nq::decode_stage1_kernel<NT, 256, nq::kMaxGroup>);
+    if (wide) set_attrs_once<NT, (NT <= 2 ? 512 : 256), 256, nq::kMaxGroup>();
+    else set_attrs_once<NT, 256, 256, nq::kMaxGroup>();
+    return nq_host::launch_ex(fn, dim3(acc, cs), dim3(wide ? 512 : 256), smem, stream, args, pdl, cs) == cudaSuccess
+               ? NQ_OK
+               : NQ_ERR_LAUNCH;
+}
+
 }  // namespace
 
 size_t nq_decode_workspace_bytes(int64_t d_in, int64_t r, int64_t M) {
@@ -1022,6 +1072,16 @@ nq_status nq_launch_decode_stage1(const nq_lrb_layer* L, const uint16_t* x, int6
         case 1: return launch_decode_group_nt<1, 1>(&L, 1, x, nullptr, m, nullptr, nullptr, nullptr, stream, pdl, t);
         case 2: return launch_decode_group_nt<2, 1>(&L, 1, x, nullptr, m, nullptr, nullptr, nullptr, stream, pdl, t);
         default: return launch_decode_group_nt<3, 1>(&L, 1, x, nullptr, m, nullptr, nullptr, nullptr, stream, pdl, t);
+    }
+}
+
+nq_status nq_launch_decode_stage1_pair(const nq_lrb_layer* L0, const uint16_t* x0, float* t0, const nq_lrb_layer* L1,
+                                       const uint16_t* x1, float* t1, int64_t M, cudaStream_t stream, bool pdl) {
+    const int m = static_cast<int>(M);
+    switch (ntiles_for(M)) {
+        case 1: return launch_stage1_pair_nt<1>(L0, x0, t0, L1, x1, t1, m, stream, pdl);
+        case 2: return launch_stage1_pair_nt<2>(L0, x0, t0, L1, x1, t1, m, stream, pdl);
+        default: return launch_stage1_pair_nt<3>(L0, x0, t0, L1, x1, t1, m, stream, pdl);
     }
 }
 

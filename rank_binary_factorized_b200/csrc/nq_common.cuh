@@ -88,3 +88,6 @@ nq_status nq_launch_prefill_stage1(const nq_lrb_layer* L, const uint16_t* x, int
 // Stage 1 alone (decode.cu): t = V^T (s2 . x) [M][r] fp32 into t, M <= NQ_MATVEC_MAX_M.
 nq_status nq_launch_decode_stage1(const nq_lrb_layer* L, const uint16_t* x, int64_t M, float* t, cudaStream_t stream,
                                   bool pdl);
+// Stage 1 alone for two layers with their own inputs, one launch (decode.cu).
+nq_status nq_launch_decode_stage1_pair(const nq_lrb_layer* L0, const uint16_t* x0, float* t0, const nq_lrb_layer* L1,
+                                       const uint16_t* x1, float* t1, int64_t M, cudaStream_t stream, bool pdl);

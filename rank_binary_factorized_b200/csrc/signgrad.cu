@@ -395,8 +395,7 @@ nq_status nq_launch_sign_grads(const nq_lrb_layer* L, const nq_lrb_layer* X, con
     if (M <= NQ_MATVEC_MAX_M) {
         float* t = reinterpret_cast<float*>(w + NQ_WS_HEADER_BYTES);
         float* p = reinterpret_cast<float*>(w + NQ_WS_HEADER_BYTES + align256(static_cast<size_t>(M * L->r) * 4));
-        if ((st = nq_launch_decode_stage1(L, x, M, t, stream, pdl)) != NQ_OK) return st;
-        if ((st = nq_launch_decode_stage1(X, ybar, M, p, stream, pdl)) != NQ_OK) return st;
+        if ((st = nq_launch_decode_stage1_pair(L, x, t, X, ybar, p, M, stream, pdl)) != NQ_OK) return st;
         nq::SignGradSmallArgs a{};
         a.t = t;
         a.p = p;
