@@ -214,12 +214,22 @@ def timed_replays(torch, g, stream, steps, warmup, dist=None, sampler=None):
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
-    ms = start.elapsed_time(end)
-    if dist is not None:
-        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    return ms
+    return max_over_ranks(torch, start.elapsed_time(end), dist, "cuda")
+
+
+def max_over_ranks(torch, ms, dist, device):
+    """The slowest rank's time: every rank gets the maximum of the ranks' values."""
+    if dist is None:
+        return ms
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_us_per_layer(ms, steps, layers_per_step, world):
+    """Whole-job time per layer: every rank runs `layers_per_step` layers per step, so the job
+    processes steps x layers_per_step x world layers in the slowest rank's time."""
+    return ms * 1e3 / (steps * layers_per_step * world)
 
 
 class _null:
@@ -264,8 +274,7 @@ def gpu_arm(args, rank, world, local):
                            int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local]))
     ms = timed_replays(torch, g, stream, args.steps, args.warmup, dist, sampler)
     nq.sync_status(stream)
-    layers_total = args.steps * n * world
-    us_per_layer_job = ms * 1e3 / layers_total  # whole job: all ranks' layers in the max time
+    us_per_layer_job = job_us_per_layer(ms, args.steps, n, world)  # all ranks' layers in the max time
     us_per_layer_gpu = ms * 1e3 / (args.steps * n)  # one GPU's layer forward
     achieved = lbytes / (us_per_layer_gpu * 1e-6) / 1e9
     del g

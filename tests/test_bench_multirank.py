@@ -1,0 +1,63 @@
+"""The N > 1 host path of bench.py on CPU: two gloo ranks take the slowest rank's time and
+report whole-job throughput; under torchrun the reference arm prints one line from rank 0
+only.  No GPU is used."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.distributed as tdist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    sys.path.insert(0, ROOT)
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    tdist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        ms = [3.0, 5.0][rank]
+        got = bench.max_over_ranks(torch, ms, tdist, "cpu")
+        out[rank] = (got, bench.job_us_per_layer(got, steps=4, layers_per_step=10, world=world))
+    finally:
+        tdist.destroy_process_group()
+
+
+def test_two_gloo_ranks_take_the_slowest_time():
+    world, port = 2, _free_port()
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_rank_main, args=(world, port, out), nprocs=world, start_method="spawn", join=True)
+    assert out[0] == out[1] == (5.0, 5.0 * 1e3 / (4 * 10 * 2))
+
+
+def test_single_process_needs_no_collective():
+    import bench
+    assert bench.max_over_ranks(torch, 2.5, None, "cpu") == 2.5
+    assert bench.job_us_per_layer(2.0, 2, 5, 1) == 200.0
+
+
+def test_reference_arm_under_torchrun_prints_once_from_rank_0():
+    port = _free_port()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2", "--master-addr",
+           "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus",
+           "2", "--steps", "2", "--warmup", "1", "--cpu-seconds", "1"]
+    env = dict(os.environ, OMP_NUM_THREADS="1")
+    proc = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert proc.returncode == 0, proc.stderr[-2000:]
+    lines = [ln for ln in proc.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["unit"] == "us/layer"
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
