@@ -39,6 +39,9 @@ __device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
 __device__ __forceinline__ void cp_async8(uint32_t dst, const void* src) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
 }
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 // Asks the memory system to bring [src, src + bytes) into L2 (no data returns to the SM);
 // src and bytes are multiples of 16.
@@ -68,6 +71,18 @@ __device__ __forceinline__ uint32_t digit_byte(int v, int q) {
     return static_cast<uint32_t>((v1 - d1) >> 8) & 255u;
 }
 
+
+// Stage 2's B table (t's digits), which stage 1 writes.
+// B table layout: the two B-fragment words of lane (gid, tig) for bit offset s, word group g
+// (8 words) and column tile nt sit next to each other, lanes in order, so one 64-bit load per
+// lane and MMA reads 256 contiguous bytes:
+//   word ((((s * ng + g) * NT + nt) * 32 + 4 * gid + tig) * 2 + half)
+// holds the digits of column 8 nt + gid for word 8 g + tig + 4 half.
+template <int NT>
+__device__ __forceinline__ int s2_bidx(int s_, int w, int col, int ng) {
+    const int g = w >> 3, tg = w & 3, half = (w >> 2) & 1;
+    return ((((s_ * ng + g) * NT + (col >> 3)) * 32 + 4 * (col & 7) + tg) * 2 + half);
+}
 
 // ------------------------------------------------------------------ stage 1 (integer MMA)
 //
@@ -107,6 +122,14 @@ struct S1Params {
     int zstage;          // z of the slice (M x rows_per_slice fp32) is kept in shared memory
     const uint32_t* upf;  // U of the same layer: its first upf_bytes (a multiple of 16) are
     int64_t upf_bytes;    // prefetched into L2 for stage 2, 1/grid of them per block
+    // Stage 2's input, when tab != nullptr (otherwise t is written in fp32): t quantised with
+    // one shift per batch row taken from a bound on |t| (sum over the slices of 2^-shift
+    // sum_j |z_q|, the same in every cluster), as the digit table in s2_bidx layout; the
+    // owner blocks' sums of t_q, tsum[(chunk * CS + rank) * M + m]; the shift, tsh[m].
+    uint32_t* tab;
+    long long* tsum;
+    int* tsh;
+    int nwp;  // words per row padded to a multiple of 8 (the table's geometry)
 };
 
 // Up to kMaxGroup projections that share their input x are launched as one grid: block
@@ -160,6 +183,8 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const __grid_const
     __shared__ float s_mul[NQ_MATVEC_MAX_M];
     __shared__ double s_dinv[NQ_MATVEC_MAX_M];  // 2^-shift: turns the exact integers into values
     __shared__ unsigned long long s_zsum[NQ_MATVEC_MAX_M];
+    __shared__ unsigned long long s_zabs[NQ_MATVEC_MAX_M];  // sum_j |z_q| of the slice
+    __shared__ long long s_tqsum[NQ_MATVEC_MAX_M];          // owner's sum of t_q
     __shared__ float s_wmax[kS1Threads / 32][NQ_MATVEC_MAX_M];
 
     cg::cluster_group cluster = cg::this_cluster();
@@ -294,7 +319,11 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const __grid_const
         }
         if (kKSplit > 1)  // several warps add into one output; otherwise each stores its own
             for (int e = tid; e < kS1Outs * NT * 8; e += kS1Threads) red[e] = 0;
-        if (tid < NQ_MATVEC_MAX_M) s_zsum[tid] = 0ull;
+        if (tid < NQ_MATVEC_MAX_M) {
+            s_zsum[tid] = 0ull;
+            s_zabs[tid] = 0ull;
+            s_tqsum[tid] = 0ll;
+        }
         __syncthreads();
         if (tid < p.M) {
             float v = 0.0f;
@@ -309,9 +338,9 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const __grid_const
     }
     // per-thread partial sums of the quantised z, per batch row (column group of the z table)
     constexpr int MG = (NT * 8 + 2) / 3;
-    long long zacc[MG];
+    long long zacc[MG], zabs[MG];
 #pragma unroll
-    for (int m = 0; m < MG; ++m) zacc[m] = 0;
+    for (int m = 0; m < MG; ++m) zacc[m] = zabs[m] = 0;
 
     // ---- passes over the slice: z table, then MMAs; integer accumulators live in registers
     // two accumulator sets, even and odd K steps, for two independent MMA chains per tile
@@ -356,12 +385,13 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const __grid_const
                                              : f16_bits_to_float(p.s2[j]) * bf16_bits_to_float(xm[j]);
                         }
                     }
-                    int qsum = 0;
+                    int qsum = 0, qabs = 0;
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         uint32_t a0, a1, a2;
                         const int qv = __float2int_rn(zv[i] * mul);
                         qsum += qv;
+                        qabs += abs(qv);
                         digits3(qv, a0, a1, a2);
                         d0 |= a0 << (8 * i);
                         d1 |= a1 << (8 * i);
@@ -369,7 +399,10 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const __grid_const
                     }
 #pragma unroll
                     for (int mm = 0; mm < MG; ++mm)
-                        if (mm == m) zacc[mm] += qsum;
+                        if (mm == m) {
+                            zacc[mm] += qsum;
+                            zabs[mm] += qabs;
+                        }
                 }
                 uint32_t* dst = zq + jq * SWZ + 3 * m;
                 if (m < p.M) {  // rows >= M: their D columns are never read
@@ -412,9 +445,15 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const __grid_const
 #pragma unroll
     for (int m = 0; m < MG; ++m) {
         if (m < p.M) {
-            long long v = zacc[m];
-            for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-            if (lane == 0) atomicAdd(&s_zsum[m], static_cast<unsigned long long>(v));
+            long long v = zacc[m], va = zabs[m];
+            for (int off = 16; off > 0; off >>= 1) {
+                v += __shfl_xor_sync(0xffffffffu, v, off);
+                va += __shfl_xor_sync(0xffffffffu, va, off);
+            }
+            if (lane == 0) {
+                atomicAdd(&s_zsum[m], static_cast<unsigned long long>(v));
+                atomicAdd(&s_zabs[m], static_cast<unsigned long long>(va));
+            }
         }
     }
 
@@ -453,14 +492,36 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const __grid_const
         double* dst = cluster.map_shared_rank(part, owner);
         dst[(m * per + ko) * CS + q] = static_cast<double>(val) * s_dinv[m];
     }
+    // the slice's bound on its share of |t| (exact), into every owner's inbox after the partials
+    double* bound = part + p.M * kS1Outs;  // [M][CS]
+    if (p.tab)
+        for (int e = tid; e < p.M * CS; e += kS1Threads) {
+            const int m = e / CS, owner = e - m * CS;
+            cluster.map_shared_rank(bound, owner)[m * CS + q] = static_cast<double>(s_zabs[m]) * s_dinv[m];
+        }
     cluster.sync();
+    // one shift per batch row for t: |t| <= L = sum over the slices, in rank order (the same
+    // value in every thread, block and cluster), so |t_q| <= 2^22
+    auto t_shift = [&](int m) {
+        double L = 0.0;
+        for (int rank = 0; rank < CS; ++rank) L += bound[m * CS + rank];
+        int e = 0;
+        frexp(L, &e);  // L < 2^e
+        return (L > 0.0) ? min(max(22 - e, -126), 126) : 0;
+    };
+    if (p.tab && chunk == 0 && q == 0 && tid < p.M) p.tsh[tid] = t_shift(tid);
     {
         // owner q: its `per` outputs, each the sum of the CS slices' partials in a fixed order
         // (four interleaved accumulators, then pairwise): a short dependent chain, few registers
         const int k_lo = q * per;
+        const int ngp = p.nwp / 8;
+        long long tqacc[MG];  // this thread's sum of t_q per batch row
+#pragma unroll
+        for (int m = 0; m < MG; ++m) tqacc[m] = 0;
         for (int e = tid; e < p.M * per; e += kS1Threads) {
             const int m = e >> lg_per, ko = e & (per - 1);
             const int64_t k = static_cast<int64_t>(wglob0) * 32 + k_lo + ko;
+            double sum = 0.0;
             if (k < p.r) {
                 const double* src = part + (m * per + ko) * CS;
                 double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
@@ -470,8 +531,39 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const __grid_const
                     if (rank + 2 < CS) a2 += src[rank + 2];
                     if (rank + 3 < CS) a3 += src[rank + 3];
                 }
-                p.t[static_cast<int64_t>(m) * p.r + k] = static_cast<float>((a0 + a1) + (a2 + a3));
+                sum = (a0 + a1) + (a2 + a3);
             }
+            if (p.tab) {
+                // t_q's three digits, byte (k / 8) % 4 of the table words for (k % 8, k / 32);
+                // outputs past r (up to the padded word count) get zero digits
+                const int tq = (k < p.r) ? __double2int_rn(sum * ldexp(1.0, t_shift(m))) : 0;
+#pragma unroll
+                for (int mm = 0; mm < MG; ++mm)
+                    if (mm == m) tqacc[mm] += tq;
+                uint32_t d0, d1, d2;
+                digits3(tq, d0, d1, d2);
+                const int w = static_cast<int>(k >> 5), s_ = static_cast<int>(k & 7), b = static_cast<int>((k >> 3) & 3);
+                uint8_t* tb = reinterpret_cast<uint8_t*>(p.tab);
+                tb[4 * s2_bidx<NT>(s_, w, 3 * m, ngp) + b] = static_cast<uint8_t>(d0);
+                tb[4 * s2_bidx<NT>(s_, w, 3 * m + 1, ngp) + b] = static_cast<uint8_t>(d1);
+                tb[4 * s2_bidx<NT>(s_, w, 3 * m + 2, ngp) + b] = static_cast<uint8_t>(d2);
+            } else if (k < p.r) {
+                p.t[static_cast<int64_t>(m) * p.r + k] = static_cast<float>(sum);
+            }
+        }
+        if (p.tab) {
+            // the block's sum of t_q per batch row: warp sums, then one shared add per warp
+#pragma unroll
+            for (int m = 0; m < MG; ++m) {
+                if (m < p.M) {
+                    long long v = tqacc[m];
+                    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+                    if (lane == 0 && v != 0)
+                        atomicAdd(reinterpret_cast<unsigned long long*>(&s_tqsum[m]), static_cast<unsigned long long>(v));
+                }
+            }
+            __syncthreads();
+            if (tid < p.M) p.tsum[(static_cast<int64_t>(chunk) * CS + q) * p.M + tid] = s_tqsum[tid];
         }
     }
 }
@@ -495,7 +587,12 @@ struct S2Params {
     const uint32_t* U;
     int64_t ldu;
     const uint16_t* s1;
-    const float* t;
+    // t as stage 1 leaves it: the digit table (s2_bidx layout, 8 nwp NT 8 words), the owner
+    // blocks' sums of t_q (tsum_n per batch row, [i][M]) and the shift per batch row
+    const uint32_t* tab;
+    const long long* tsum;
+    int tsum_n;
+    const int* tsh;
     uint16_t* y;
     int M;
     int64_t d_out;
@@ -503,7 +600,6 @@ struct S2Params {
     int su;              // shared-memory row stride of U (words), = 4 (mod 32)
     int mt_total;        // 16-row M-tiles of U
     int chunk_mt;        // M-tiles staged in shared memory at a time
-    int tstage;          // t (M x r fp32) is copied into shared memory for the table build
     // gradient mode (grad != nullptr): instead of y, grad[i] = sum_m cot[m][i] (U t_m)_i, the
     // derivative of sum_m <cot_m, y_m> with respect to s1_i; cot [M][d_out] bf16, grad fp32
     const uint16_t* cot;
@@ -516,17 +612,6 @@ struct S2Group {
     int cta_off[kMaxGroup + 1];
     int n;
 };
-
-// B table layout: the two B-fragment words of lane (gid, tig) for bit offset s, word group g
-// (8 words) and column tile nt sit next to each other, lanes in order, so one 64-bit load per
-// lane and MMA reads 256 contiguous bytes:
-//   word ((((s * ng + g) * NT + nt) * 32 + 4 * gid + tig) * 2 + half)
-// holds the digits of column 8 nt + gid for word 8 g + tig + 4 half.
-template <int NT>
-__device__ __forceinline__ int s2_bidx(int s_, int w, int col, int ng) {
-    const int g = w >> 3, tg = w & 3, half = (w >> 2) & 1;
-    return ((((s_ * ng + g) * NT + (col >> 3)) * 32 + 4 * (col & 7) + tg) * 2 + half);
-}
 
 template <int NT, int TH, int GN>
 __global__ void __launch_bounds__(TH, 1) decode_stage2_kernel(const __grid_constant__ S2Group grp) {
@@ -543,13 +628,12 @@ __global__ void __launch_bounds__(TH, 1) decode_stage2_kernel(const __grid_const
     uint32_t* ublk = bt + 8 * p.nwp * NT * 8;              // [chunk_mt*16][su]
     int* red = reinterpret_cast<int*>(ublk + p.chunk_mt * 16 * p.su);  // [chunk_mt*16][NT*8]
     float* s1_s = reinterpret_cast<float*>(red + p.chunk_mt * 16 * NT * 8);  // [chunk_mt*16]
-    float* ts_s = s1_s + p.chunk_mt * 16;                                   // [M][r] when p.tstage
-    __shared__ float s_mul[NQ_MATVEC_MAX_M];
     __shared__ double s_dinv[NQ_MATVEC_MAX_M];  // 2^-shift: turns the exact integers into values
     __shared__ unsigned long long s_tsum[NQ_MATVEC_MAX_M];
-    __shared__ float s_wmax[kS2Warps][NQ_MATVEC_MAX_M];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid < NQ_MATVEC_MAX_M) s_tsum[tid] = 0ull;
+    __syncthreads();
 
     const int mt0 = static_cast<int>((static_cast<int64_t>(bid) * p.mt_total) / G);
     const int mt1 = static_cast<int>((static_cast<int64_t>(bid + 1) * p.mt_total) / G);
@@ -588,107 +672,23 @@ __global__ void __launch_bounds__(TH, 1) decode_stage2_kernel(const __grid_const
     pdl_launch_dependents();
     pdl_wait();  // t comes from stage 1 of this call
 
-    // ---- per-batch-row scale: |t_q| < 2^22 with t_q = rint(t * 2^shift).  The batch rows are
-    // the inner, unrolled loop, so every row's loads of t are in flight together.
-    constexpr int MGS = (NT * 8 + 2) / 3;  // batch rows the B columns can hold (>= M)
+    // ---- t as stage 1 left it: the digit table goes to shared memory as it is (the chunk
+    // loop's wait and barrier publish it), the shift and the sum of t_q come from the owners
     {
-        float vmax[MGS];
-#pragma unroll
-        for (int m = 0; m < MGS; ++m) vmax[m] = 0.0f;
-        if (p.M == 1) {
-#pragma unroll 8
-            for (int k = tid; k < p.r; k += kS2Threads) {
-                const float tv = p.t[k];
-                if (p.tstage) ts_s[k + (k >> 5)] = tv;
-                vmax[0] = fmaxf(vmax[0], fabsf(tv));
-            }
-        } else {
-#pragma unroll 4
-            for (int k = tid; k < p.r; k += kS2Threads) {
-#pragma unroll
-                for (int m = 0; m < MGS; ++m) {
-                    if (m < p.M) {
-                        const float tv = p.t[static_cast<int64_t>(m) * p.r + k];
-                        if (p.tstage) ts_s[m * (p.r + p.r / 32) + k + (k >> 5)] = tv;
-                        vmax[m] = fmaxf(vmax[m], fabsf(tv));
-                    }
-                }
+        const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(bt));
+        const int pieces = 2 * p.nwp * NT * 8;  // 16-byte pieces of 8 nwp NT 8 words
+        for (int c = tid; c < pieces; c += kS2Threads) cp_async16(dst + 16u * c, p.tab + 4 * c);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        // warp m adds row m's owner sums (exact integers), lane 0 keeps the result
+        for (int m = warp; m < p.M; m += kS2Warps) {
+            long long v = 0;
+            for (int i = lane; i < p.tsum_n; i += 32) v += p.tsum[static_cast<int64_t>(i) * p.M + m];
+            for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+            if (lane == 0) {
+                s_tsum[m] = static_cast<unsigned long long>(v);
+                s_dinv[m] = ldexp(1.0, -p.tsh[m]);
             }
         }
-#pragma unroll
-        for (int m = 0; m < MGS; ++m) {
-            if (m < p.M) {
-                float v = vmax[m];
-                for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
-                if (lane == 0) s_wmax[warp][m] = v;
-            }
-        }
-        if (tid < NQ_MATVEC_MAX_M) s_tsum[tid] = 0ull;
-        __syncthreads();
-        if (tid < p.M) {
-            float v = 0.0f;
-            for (int w = 0; w < kS2Warps; ++w) v = fmaxf(v, s_wmax[w][tid]);
-            int e = 0;
-            frexpf(v, &e);  // v < 2^e
-            const int sh = (v > 0.0f) ? min(max(22 - e, -126), 126) : 0;
-            s_mul[tid] = ldexpf(1.0f, sh);
-            s_dinv[tid] = ldexp(1.0, -sh);
-        }
-        __syncthreads();
-        // t staged with one pad word after every 32 values, so that the table build's
-        // stride-32 reads fall in different banks
-        const int tld = p.tstage ? p.r + p.r / 32 : p.r;
-        auto t_at = [&](int m, int k) -> float {
-            return p.tstage ? ts_s[m * tld + k + (k >> 5)] : p.t[static_cast<int64_t>(m) * p.r + k];
-        };
-        // B table: the word for (s, w, column 3m + q) holds digit q of t_q(m, 32w + s + 8b) in
-        // byte b; one thread builds the digit words of one (s, w) for every batch row.  Every k
-        // < r lies in exactly one entry, so the entries' integers also give sum_k t_q(m, k).
-        const int ngp = p.nwp / 8;
-        constexpr int MG = (NT * 8 + 2) / 3;  // column groups of three
-        long long tacc[MG];
-#pragma unroll
-        for (int m = 0; m < MG; ++m) tacc[m] = 0;
-        for (int sw = tid; sw < 8 * p.nwp; sw += kS2Threads) {
-            const int s_ = sw / p.nwp, w = sw - s_ * p.nwp;
-#pragma unroll
-            for (int m = 0; m < MG; ++m) {
-                uint32_t d0 = 0u, d1 = 0u, d2 = 0u;
-                if (m < p.M && w < p.nw) {
-                    const float mul = s_mul[m];
-                    float tv[4];
-#pragma unroll
-                    for (int b = 0; b < 4; ++b) tv[b] = t_at(m, 32 * w + s_ + 8 * b);
-                    int qsum = 0;
-#pragma unroll
-                    for (int b = 0; b < 4; ++b) {
-                        uint32_t a0, a1, a2;
-                        const int qv = __float2int_rn(tv[b] * mul);
-                        qsum += qv;
-                        digits3(qv, a0, a1, a2);
-                        d0 |= a0 << (8 * b);
-                        d1 |= a1 << (8 * b);
-                        d2 |= a2 << (8 * b);
-                    }
-                    tacc[m] += qsum;
-                }
-                if (m < p.M) {  // rows >= M: their D columns are never read
-                    bt[s2_bidx<NT>(s_, w, 3 * m, ngp)] = d0;
-                    bt[s2_bidx<NT>(s_, w, 3 * m + 1, ngp)] = d1;
-                    bt[s2_bidx<NT>(s_, w, 3 * m + 2, ngp)] = d2;
-                }
-            }
-        }
-        // per-warp partial sums into s_tsum; read by the epilogue, after the barriers below
-#pragma unroll
-        for (int m = 0; m < MG; ++m) {
-            if (m < p.M) {
-                long long v = tacc[m];
-                for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-                if (lane == 0) atomicAdd(&s_tsum[m], static_cast<unsigned long long>(v));
-            }
-        }
-        // (the barrier before the MMAs publishes the table)
     }
 
     const int gid = lane >> 2, tig = lane & 3;
@@ -824,6 +824,10 @@ S1Plan plan_stage1(int64_t d_in, int total_chunks, int64_t M, int force_cs = 0) 
     p.n_chunks = total_chunks;
     int cs = total_chunks <= 8 ? 16 : (total_chunks <= 18 ? 8 : (total_chunks <= 37 ? 4 : 2));
     while (cs > 1 && static_cast<int64_t>(cs) * 32 > d_in) cs >>= 1;
+    // more than 8 output columns (M > 2): blocks too register-heavy to share an SM with the
+    // previous grid's, so a cluster waits for that many free SMs of one GPC; 8 keeps the wait
+    // short (7B attention, M = 8: 30.8 -> 19.1 us per layer against 16)
+    if (ntiles_for(M) >= 2 && cs > 8) cs = 8;
     if (force_cs > 0) cs = force_cs;
     p.CS = cs;
     p.rows_per_slice = static_cast<int>(((d_in + cs - 1) / cs + 31) / 32 * 32);
@@ -842,7 +846,23 @@ S1Plan plan_stage1(int64_t d_in, int total_chunks, int64_t M, int force_cs = 0) 
     return p;
 }
 
-size_t decode_ws_bytes(int64_t r, int64_t M) { return kWsHeader + align256(static_cast<size_t>(M * r) * sizeof(float)); }
+// One layer's share of the workspace: stage 2's digit table of t, the owner blocks' sums of
+// t_q (room for the largest cluster, 16) and the shifts.
+struct TLayout {
+    size_t tab, tsum, tsh, total;
+};
+TLayout t_layout(int64_t r, int64_t M) {
+    TLayout o{};
+    const int64_t nwp = (r / 32 + 7) / 8 * 8;
+    const int nt = ntiles_for(M);
+    o.tab = 0;
+    o.tsum = align256(static_cast<size_t>(8 * nwp * nt * 8) * 4);
+    o.tsh = o.tsum + align256(static_cast<size_t>(chunks_of(r)) * 16 * M * 8);
+    o.total = o.tsh + align256(static_cast<size_t>(M) * 4);
+    return o;
+}
+
+size_t decode_ws_bytes(int64_t r, int64_t M) { return kWsHeader + t_layout(r, M).total; }
 
 template <int NT, int TH1, int TH2, int GN>
 void set_attrs_once() {
@@ -863,19 +883,22 @@ template <int NT, int GN>
 nq_status launch_decode_group_nt(const nq_lrb_layer* const* Ls, int n, const uint16_t* x, uint16_t* const* ys, int M,
                                  void* ws, const uint16_t* cot, float* grad, cudaStream_t stream, bool pdl,
                                  float* t_only = nullptr) {
-    // t of member l follows the earlier members' t in the workspace; with t_only (one layer),
-    // stage 1 alone runs and writes t there
-    float* t[nq::kMaxGroup];
+    // member l's share of the workspace (t's digit table, owner sums, shifts) follows the
+    // earlier members'; with t_only (one layer), stage 1 alone runs and writes t in fp32 there
+    char* base[nq::kMaxGroup];
+    TLayout tl[nq::kMaxGroup];
     size_t off = kWsHeader;
     for (int l = 0; l < n; ++l) {
-        t[l] = ws ? reinterpret_cast<float*>(static_cast<char*>(ws) + off) : nullptr;
-        off += align256(static_cast<size_t>(M) * Ls[l]->r * sizeof(float));
+        tl[l] = t_layout(Ls[l]->r, M);
+        base[l] = ws ? static_cast<char*>(ws) + off : nullptr;
+        off += tl[l].total;
     }
-    if (t_only) t[0] = t_only;
+    int cs1 = 1;  // stage 1's cluster size: owner blocks per word chunk
     {
         int total = 0;
         for (int l = 0; l < n; ++l) total += chunks_of(Ls[l]->r);
         const S1Plan sp = plan_stage1(Ls[0]->d_in, total, M);
+        cs1 = sp.CS;
         nq::S1Group g{};
         g.n = n;
         int acc = 0;
@@ -886,7 +909,13 @@ nq_status launch_decode_group_nt(const nq_lrb_layer* const* Ls, int n, const uin
             q.ldv = L->ldv;
             q.s2 = L->s2;
             q.x = x;
-            q.t = t[l];
+            q.t = t_only;
+            if (!t_only) {
+                q.tab = reinterpret_cast<uint32_t*>(base[l] + tl[l].tab);
+                q.tsum = reinterpret_cast<long long*>(base[l] + tl[l].tsum);
+                q.tsh = reinterpret_cast<int*>(base[l] + tl[l].tsh);
+            }
+            q.nwp = static_cast<int>((L->r / 32 + 7) / 8 * 8);
             q.M = M;
             q.d_in = L->d_in;
             q.r = static_cast<int>(L->r);
@@ -935,7 +964,10 @@ nq_status launch_decode_group_nt(const nq_lrb_layer* const* Ls, int n, const uin
             q.U = L->U;
             q.ldu = L->ldu;
             q.s1 = L->s1;
-            q.t = t[l];
+            q.tab = reinterpret_cast<const uint32_t*>(base[l] + tl[l].tab);
+            q.tsum = reinterpret_cast<const long long*>(base[l] + tl[l].tsum);
+            q.tsum_n = chunks_of(L->r) * cs1;
+            q.tsh = reinterpret_cast<const int*>(base[l] + tl[l].tsh);
             q.y = ys ? ys[l] : nullptr;
             q.cot = cot;
             q.grad = grad;
@@ -955,10 +987,7 @@ nq_status launch_decode_group_nt(const nq_lrb_layer* const* Ls, int n, const uin
                 chunk = static_cast<int>((kStage2SmemBudget - bt_bytes) / per_mt);
             if (chunk < 1) return NQ_ERR_SHAPE;
             q.chunk_mt = chunk;
-            size_t smem2 = bt_bytes + chunk * per_mt;
-            const size_t t_bytes = static_cast<size_t>(M) * (L->r + L->r / 32) * sizeof(float);
-            q.tstage = (smem2 + t_bytes <= kStage2SmemBudget) ? 1 : 0;
-            if (q.tstage) smem2 += t_bytes;
+            const size_t smem2 = bt_bytes + chunk * per_mt;
             smem = std::max(smem, smem2);
             g.cta_off[l] = acc;
             acc += gl;
@@ -1087,6 +1116,6 @@ nq_status nq_launch_decode_stage1_pair(const nq_lrb_layer* L0, const uint16_t* x
 
 size_t nq_decode_group_workspace_bytes(const nq_lrb_layer* const* Ls, int n, int64_t M) {
     size_t off = kWsHeader;
-    for (int l = 0; l < n; ++l) off += align256(static_cast<size_t>(M) * Ls[l]->r * sizeof(float));
+    for (int l = 0; l < n; ++l) off += t_layout(Ls[l]->r, M).total;
     return off;
 }

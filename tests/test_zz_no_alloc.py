@@ -66,10 +66,11 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     need_gpu()
     mod = nq()
     fn = noalloc_fn()
-    # M = 8 at r = 65536: t alone is 8 x 65536 fp32 = 2 MiB, plus the 4 KiB counter header,
-    # more than NQ_NOALLOC_SCRATCH_BYTES; the call must refuse before launching anything
+    # M = 8 at r = 131072: stage 2's digit table of t alone is 8 bit offsets x 4096 words x 24
+    # columns x 4 B = 3 MiB, more than NQ_NOALLOC_SCRATCH_BYTES; the call must refuse before
+    # launching anything
     M = 8
-    p = synth.make_projection("big", 64, 64, 65536, seed=501)
+    p = synth.make_projection("big", 64, 64, 131072, seed=501)
     L = upload_projection(p)
     x = upload_bf16(synth.acts_bf16(synth.rng_for(502), (M, p.d_in)))
     y = upload_bf16(np.zeros((M, p.d_out), dtype=np.uint16))
