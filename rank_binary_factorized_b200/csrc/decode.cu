@@ -43,11 +43,6 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-// Asks the memory system to bring [src, src + bytes) into L2 (no data returns to the SM);
-// src and bytes are multiples of 16.
-__device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
 
 // The three balanced base-256 digits of a 23-bit signed integer v = a0 + 2^8 a1 + 2^16 a2,
 // each in [-128, 127], returned as s8 bytes.
@@ -120,8 +115,6 @@ struct S1Params {
     int rows_per_slice;  // rows of V per block (multiple of 32)
     int jc_rows;         // rows staged per pass (multiple of 32)
     int zstage;          // z of the slice (M x rows_per_slice fp32) is kept in shared memory
-    const uint32_t* upf;  // U of the same layer: its first upf_bytes (a multiple of 16) are
-    int64_t upf_bytes;    // prefetched into L2 for stage 2, 1/grid of them per block
     // Stage 2's input, when tab != nullptr (otherwise t is written in fp32): t quantised with
     // one shift per batch row taken from a bound on |t| (sum over the slices of 2^-shift
     // sum_j |z_q|, the same in every cluster), as the digit table in s2_bidx layout; the
@@ -231,15 +224,6 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const __grid_const
         }
     };
 
-    // stage 2's weights: start their way from HBM into L2 now, so that stage 2 reads them there
-    if (tid == 0 && p.upf_bytes > 0) {
-        const int G = n_chunks * gridDim.y, b = blockIdx.y * n_chunks + chunk;
-        const int64_t share = ((p.upf_bytes + G - 1) / G + 15) & ~static_cast<int64_t>(15);
-        const int64_t beg = static_cast<int64_t>(b) * share, end = min(beg + share, p.upf_bytes);
-        for (int64_t off = beg; off < end; off += 32768)
-            prefetch_l2_bulk(reinterpret_cast<const char*>(p.upf) + off,
-                             static_cast<uint32_t>(min(static_cast<int64_t>(32768), end - off)));
-    }
     // s2 of the slice (a weight) is read before the wait, into registers when the slice has
     // at most kS2Reg rows per thread
     constexpr int kS2Reg = 8;
@@ -923,9 +907,6 @@ nq_status launch_decode_group_nt(const nq_lrb_layer* const* Ls, int n, const uin
             q.rows_per_slice = sp.rows_per_slice;
             q.jc_rows = sp.jc_rows;
             q.zstage = sp.zstage;
-            q.upf = L->U;
-            // U up to the last valid word of its last row, rounded down to 16 bytes
-            q.upf_bytes = t_only ? 0 : (((L->d_out - 1) * L->ldu + L->r / 32) * 4) & ~static_cast<int64_t>(15);
             g.chunk_off[l] = acc;
             acc += chunks_of(L->r);
         }
@@ -1035,8 +1016,6 @@ nq_status launch_stage1_pair_nt(const nq_lrb_layer* L0, const uint16_t* x0, floa
         q.rows_per_slice = sp[l].rows_per_slice;
         q.jc_rows = sp[l].jc_rows;
         q.zstage = sp[l].zstage;
-        q.upf = L->U;
-        q.upf_bytes = 0;
         g.chunk_off[l] = acc;
         acc += chunks_of(L->r);
     }
