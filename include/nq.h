@@ -103,22 +103,23 @@ NQ_API nq_status nq_pack_signs(const float* latent, int64_t rows, int64_t r, int
 /*
  * nq_workspace_bytes -- device scratch a call with M activation rows needs (for
  * nq_lrb_matvec, nq_lrb_matmul, nq_layer_forward, nq_lrb_transposed and
- * nq_lrb_scale_grads alike).  Returns 0 for an invalid
- * layer or M.  The workspace must stay untouched by other work while the call runs.  Its
- * first 4096 bytes hold counters that read zero between calls (the library restores them
- * before each call ends); the rest is scratch.  So one workspace can be reused by
- * consecutive calls of any shape on the same stream, provided it was zero-filled once
- * before its first use (and again after a call reported NQ_ERR_TIMEOUT).
+ * nq_lrb_scale_grads alike).  Returns 0 for an invalid layer or M.  The workspace must stay
+ * untouched by other work while the call runs.  Its first 4096 bytes are a reserved header
+ * that the kernels neither read nor write; the rest is per-call scratch, fully written
+ * before it is read.  So one workspace can be reused by consecutive calls of any shape on
+ * the same stream, with no initialisation.
  */
 NQ_API size_t nq_workspace_bytes(const nq_lrb_layer* L, int64_t M);
 
 /*
  * nq_lrb_matvec -- decode path, 1 <= M <= NQ_MATVEC_MAX_M.
  * Section 2 factorisation equation, evaluated as two streaming stages over the packed
- * words: t[m][k] = sum_j V_jk s2_j x[m][j] (fp32), then y[m][i] = bf16(s1_i sum_k U_ik t[m][k]).
+ * words: t[m][k] = sum_j V_jk s2_j x[m][j], then y[m][i] = bf16(s1_i sum_k U_ik t[m][k]).
  *   x [M][d_in] bf16, y [M][d_out] bf16 (round to nearest even), ws = workspace of at
- *   least nq_workspace_bytes(L, M) bytes (16-byte aligned, zero-filled before first use).
- * Accumulation is fp32; results are run-to-run deterministic.
+ *   least nq_workspace_bytes(L, M) bytes (16-byte aligned).
+ * Both stages sum exact integers: s2 x is quantised to 23-bit fixed point per row slice of V,
+ * t to 23-bit fixed point per batch row (the shift from an exact bound on |t|), and the
+ * partial sums are combined in fp64 in a fixed order.  Results are run-to-run deterministic.
  */
 NQ_API nq_status nq_lrb_matvec(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y, int64_t M, void* ws,
                         size_t ws_bytes, void* stream);
@@ -248,13 +249,13 @@ NQ_API nq_status nq_sync_status(void* stream);
  * (cudaMalloc is not a stream operation and may synchronise the device), latency-critical
  * loops that cannot take an allocator round trip, plain C callers without an allocator.
  * Same operation, arguments and numerics as nq_lrb_matvec, minus the workspace: the
- * scratch (stage-1 tickets, t and the per-slice partials) lives in one statically sized
+ * scratch (t's digit table and its sums) lives in one statically sized
  * array of NQ_NOALLOC_SCRATCH_BYTES inside libnq.so, which every GPU that loads the library
  * holds until the process exits.  A call whose scratch need (nq_workspace_bytes for the same
  * layer and M <= 8) exceeds that size returns NQ_ERR_SCRATCH_LIMIT without launching.
  * The first call on a device looks up the array's device address (set-up, once per
  * device, on the calling thread with that device current); make that first call before
- * any stream capture.  Every call clears the ticket header on `stream` before launching.
+ * any stream capture.
  * All calls on a device share the one array: calls that can overlap on the GPU (different
  * streams, or the same stream without ordering) race and must be serialised by the caller.
  * Never calls cudaMalloc, cudaFree or any allocating routine.

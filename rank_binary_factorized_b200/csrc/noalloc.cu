@@ -64,8 +64,5 @@ extern "C" NQ_API nq_status nq_lrb_matvec_noalloc(const nq_lrb_layer* L, const u
     void* scratch = scratch_address(dev);
     if (!scratch) return NQ_ERR_LAUNCH;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // The stage-1 tickets at the head of the scratch must read zero when a call starts; the
-    // previous call may have been cut short, so clear them on the stream first.
-    if (cudaMemsetAsync(scratch, 0, NQ_WS_HEADER_BYTES, s) != cudaSuccess) return NQ_ERR_LAUNCH;
     return nq_launch_decode(L, x, y, M, scratch, s, true);
 }

@@ -12,11 +12,10 @@
 #error "libnq is written for sm_100a (B200) only"
 #endif
 
-// Every workspace starts with this many bytes of counters owned by the decode path (zero
-// between calls); the rest is per-call scratch.  Bounds the word-chunk count of stage 1.
+// Every workspace starts with this many reserved bytes, which the kernels neither read nor
+// write; the per-call scratch follows.
 #define NQ_WS_HEADER_BYTES 4096
-#define NQ_MAX_RANK (NQ_WS_HEADER_BYTES / 4 * 8 * 32)
-static_assert(NQ_MAX_RANK == NQ_MAX_RANK_LIMIT, "rank limit of nq.h and the ticket header disagree");
+#define NQ_MAX_RANK NQ_MAX_RANK_LIMIT
 
 namespace nq {
 

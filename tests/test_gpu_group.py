@@ -46,6 +46,23 @@ def test_group_ragged_members(M):
     _check_group(projs, M, 1320 + M)
 
 
+def test_group_70b_gate_up():
+    """The 70B MLP's gate and up as the benchmark launches them: one grid of 28 word chunks in
+    clusters of 4, 512-thread blocks."""
+    need_gpu()
+    projs = synth.make_workload("layer70b")[4:6]
+    assert [p.name for p in projs] == ["gate", "up"]
+    _check_group(projs, 1, 1350, sample_rows=48)
+
+
+@pytest.mark.parametrize("M", [1, 8])
+def test_70b_o_projection(M):
+    need_gpu()
+    p = synth.make_workload("layer70b")[3]
+    assert p.name == "o"
+    _check_group([p], M, 1360 + M, sample_rows=48)
+
+
 def test_group_mlp_gate_up():
     need_gpu()
     projs = synth.make_workload("mlp7b")[:2]
