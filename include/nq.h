@@ -242,6 +242,16 @@ NQ_API nq_status nq_silu_mul(const uint16_t* g, const uint16_t* u, uint16_t* h, 
 NQ_API nq_status nq_sync_status(void* stream);
 
 /*
+ * nq_selftest_bounded_wait -- exercises the failure path of the library's bounded device waits
+ * (diagnostic; never needed in normal use).  Launches one block on `stream` whose thread waits,
+ * for limit_us microseconds (1000 .. 2000000, NQ_ERR_SHAPE otherwise), on an mbarrier that
+ * nothing completes.  The wait gives up, records the timeout in the device error word and the
+ * kernel exits normally, so the context stays usable; the next nq_sync_status returns
+ * NQ_ERR_TIMEOUT and clears the word.  NQ_ERR_DEVICE on a device that is not sm_100.
+ */
+NQ_API nq_status nq_selftest_bounded_wait(int64_t limit_us, void* stream);
+
+/*
  * nq_lrb_matvec_noalloc -- nq_lrb_matvec for callers that cannot allocate device memory.
  * The pages have no counterpart to this entry point; it exists for deployment.  Callers
  * that cannot hand over a workspace: plug-ins that an inference engine gives only their

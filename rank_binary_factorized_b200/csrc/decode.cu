@@ -164,7 +164,6 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const __grid_const
         while (li + 1 < grp.n && static_cast<int>(blockIdx.x) >= grp.chunk_off[li + 1]) ++li;
     const S1Params& p = grp.p[li];
     const int chunk = blockIdx.x - grp.chunk_off[li];
-    const int n_chunks = grp.chunk_off[li + 1] - grp.chunk_off[li];
     const int nq_rows = p.jc_rows / 4;  // quads per pass
     const int nkb = p.jc_rows / 32;     // K steps per pass
     uint32_t* aws = smem1;                          // [8 words][nkb][2][4][4]

@@ -55,16 +55,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // kWaitLimitNs of wall time, records NQ timeout in the error word and returns false.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned int* err) {
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, unsigned int* err, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 255u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) {
+        if ((i & 255u) == 0u && globaltimer_ns() - t0 > limit_ns) {
             flag_error(err, kErrTimeout);
             return false;
         }
     }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned int* err) {
+    return mbar_wait_for(bar, parity, err, kWaitLimitNs);
 }
 
 // ------------------------------------------------------------------ TMA (tile mode, no multicast)

@@ -69,6 +69,8 @@ _lib.nq_sign_grads_workspace_bytes.argtypes = [ctypes.POINTER(nq_lrb_layer), _i6
 _lib.nq_lrb_sign_grads.restype = ctypes.c_int
 _lib.nq_lrb_sign_grads.argtypes = [ctypes.POINTER(nq_lrb_layer), _p, _p, _i64, _p, _i64, _p, _i64, _p, ctypes.c_size_t,
                                    _p]
+_lib.nq_selftest_bounded_wait.restype = ctypes.c_int
+_lib.nq_selftest_bounded_wait.argtypes = [_i64, _p]
 _lib.nq_sync_status.argtypes = [_p]
 _lib.nq_status_string.restype = ctypes.c_char_p
 _lib.nq_status_string.argtypes = [ctypes.c_int]
@@ -306,6 +308,12 @@ def silu_mul(g: torch.Tensor, u: torch.Tensor, h=None, stream=None) -> torch.Ten
         h = torch.empty_like(g)
     _check("nq_silu_mul", _lib.nq_silu_mul(_ptr(g), _ptr(u), _ptr(h), g.numel(), _stream_ptr(stream)))
     return h
+
+
+def selftest_bounded_wait(limit_us: int = 20000, stream=None) -> None:
+    """Launch the diagnostic kernel whose bounded wait runs out (see nq.h); the next
+    sync_status raises NQError with NQ_ERR_TIMEOUT."""
+    _check("nq_selftest_bounded_wait", _lib.nq_selftest_bounded_wait(int(limit_us), _stream_ptr(stream)))
 
 
 def sync_status(stream=None) -> None:

@@ -123,6 +123,12 @@ def test_sign_grads_argument_errors(nq):
     assert lib.nq_sign_grads_workspace_bytes(ctypes.byref(_layer(nq, r=48)), 1) == 0
 
 
+def test_selftest_argument_errors(nq):
+    lib = nq.raw_lib()
+    assert lib.nq_selftest_bounded_wait(999, None) == NQ["SHAPE"]
+    assert lib.nq_selftest_bounded_wait(2000001, None) == NQ["SHAPE"]
+
+
 def test_workspace_covers_both_directions(nq):
     """One workspace serves the forward product, the transpose and the scale gradients: the
     size is the same for a layer and for the layer with its two sides exchanged."""
