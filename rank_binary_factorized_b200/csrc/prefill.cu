@@ -440,8 +440,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     }
 }
 
-// Z[m][j] = fp16(bf16 x[m][j] * fp16 s2[j]) for j < d_in; row stride ldz.  Rows m by grid y,
-// 8 elements (16 bytes) per thread when d_in is a multiple of 8 (rows 16-byte aligned).
+// Z[m][j] = fp16(bf16 x[m][j] * fp16 s2[j]) for j < d_in; row stride ldz.  Rows m by grid y;
+// when d_in is a multiple of 8 (rows 16-byte aligned), up to VPT 16-byte vectors per thread,
+// otherwise one element per thread.
 __device__ __forceinline__ uint32_t scale2_f16(uint32_t xb2, uint32_t sh2) {
     const float a = bf16_bits_to_float(static_cast<uint16_t>(xb2 & 0xFFFFu)) * f16_bits_to_float(static_cast<uint16_t>(sh2 & 0xFFFFu));
     const float b = bf16_bits_to_float(static_cast<uint16_t>(xb2 >> 16)) * f16_bits_to_float(static_cast<uint16_t>(sh2 >> 16));
@@ -449,29 +450,51 @@ __device__ __forceinline__ uint32_t scale2_f16(uint32_t xb2, uint32_t sh2) {
            (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(b))) << 16);
 }
 
+template <int VPT>
 __global__ void __launch_bounds__(256) scale_convert_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ s2,
                                                            uint16_t* __restrict__ z, int64_t M, int64_t d_in, int64_t ldz) {
     pdl_wait();
+    if ((d_in & 7) == 0) {
+        // rows by grid y; each thread up to VPT 16-byte vectors of a row, loads issued together
+        const int64_t per_row = d_in / 8;
+        const int64_t step = static_cast<int64_t>(blockDim.x) * VPT;
+        for (int64_t m = blockIdx.y; m < M; m += gridDim.y) {
+            const uint4* xr = reinterpret_cast<const uint4*>(x + m * d_in);
+            uint4* zr = reinterpret_cast<uint4*>(z + m * ldz);
+            for (int64_t c0 = static_cast<int64_t>(blockIdx.x) * step + threadIdx.x; c0 < per_row;
+                 c0 += static_cast<int64_t>(gridDim.x) * step) {
+                uint4 xv[VPT], sv[VPT];
+#pragma unroll
+                for (int u = 0; u < VPT; ++u) {
+                    const int64_t c = c0 + static_cast<int64_t>(u) * blockDim.x;
+                    if (c < per_row) {
+                        xv[u] = __ldcs(xr + c);
+                        sv[u] = __ldg(reinterpret_cast<const uint4*>(s2) + c);
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < VPT; ++u) {
+                    const int64_t c = c0 + static_cast<int64_t>(u) * blockDim.x;
+                    if (c < per_row) {
+                        uint4 o;
+                        o.x = scale2_f16(xv[u].x, sv[u].x);
+                        o.y = scale2_f16(xv[u].y, sv[u].y);
+                        o.z = scale2_f16(xv[u].z, sv[u].z);
+                        o.w = scale2_f16(xv[u].w, sv[u].w);
+                        zr[c] = o;
+                    }
+                }
+            }
+        }
+        return;
+    }
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     for (int64_t m = blockIdx.y; m < M; m += gridDim.y) {
         const uint16_t* xr = x + m * d_in;
         uint16_t* zr = z + m * ldz;
-        if ((d_in & 7) == 0) {
-            for (int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; v < d_in / 8; v += stride) {
-                const uint4 xv = __ldg(reinterpret_cast<const uint4*>(xr) + v);
-                const uint4 sv = __ldg(reinterpret_cast<const uint4*>(s2) + v);
-                uint4 o;
-                o.x = scale2_f16(xv.x, sv.x);
-                o.y = scale2_f16(xv.y, sv.y);
-                o.z = scale2_f16(xv.z, sv.z);
-                o.w = scale2_f16(xv.w, sv.w);
-                reinterpret_cast<uint4*>(zr)[v] = o;
-            }
-        } else {
-            for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < d_in; j += stride) {
-                const float v = bf16_bits_to_float(xr[j]) * f16_bits_to_float(s2[j]);
-                zr[j] = __half_as_ushort(__float2half_rn(v));
-            }
+        for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < d_in; j += stride) {
+            const float v = bf16_bits_to_float(xr[j]) * f16_bits_to_float(s2[j]);
+            zr[j] = __half_as_ushort(__float2half_rn(v));
         }
     }
 }
@@ -692,13 +715,19 @@ nq_status launch_stage1(const nq_lrb_layer* L, const uint16_t* x, int64_t M, voi
     uint16_t* t = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + p.off_t);
     unsigned int* err = nq_host::error_word();
     {  // Z = fp16(x * s2)
+        // four vectors per thread once the job has enough of them for 2 blocks per SM at that
+        // depth; one otherwise (more, smaller blocks for few rows)
         const int64_t per_row = (L->d_in % 8 == 0) ? L->d_in / 8 : L->d_in;  // work items per row
-        const unsigned gx = static_cast<unsigned>(std::min<int64_t>((per_row + 255) / 256, 64));
+        const bool deep = (L->d_in % 8 == 0) && M * per_row >= 2LL * 1024 * nq_host::sm_count();
+        const int64_t per_block = deep ? 1024 : 256;
+        const unsigned gx = static_cast<unsigned>(std::min<int64_t>((per_row + per_block - 1) / per_block, 64));
         const unsigned gy = static_cast<unsigned>(std::min<int64_t>(M, 65535));
         const uint16_t* s2 = L->s2;
         int64_t d_in = L->d_in, ldz = p.ldz;
         void* args[] = {&x, &s2, &z, &M, &d_in, &ldz};
-        if (nq_host::launch_pdl(reinterpret_cast<const void*>(nq::scale_convert_kernel), dim3(gx, gy), dim3(256), 0, stream,
+        const void* fn = deep ? reinterpret_cast<const void*>(nq::scale_convert_kernel<4>)
+                              : reinterpret_cast<const void*>(nq::scale_convert_kernel<1>);
+        if (nq_host::launch_pdl(fn, dim3(gx, gy), dim3(256), 0, stream,
                                 args, pdl) != cudaSuccess)
             return NQ_ERR_LAUNCH;
     }
