@@ -74,12 +74,19 @@ def measured_peaks():
 HOST_SIDE_MARKER = "// ------------------------------------------------------------------------------ host side"
 
 
-def device_source_sha(path: str) -> str:
-    """Hash of a kernel file's device part (everything before its host-side marker), so that
-    host-only edits keep a capture valid and any kernel edit invalidates it."""
+def device_source_sha(path: str, text: str = None) -> str:
+    """Hash of a kernel file's device part (everything before its host-side marker) with
+    comments and whitespace removed, so that host-only or comment edits keep a capture valid and
+    any code edit of a kernel invalidates it."""
     import hashlib
-    text = open(path).read()
-    return hashlib.sha256(text.split(HOST_SIDE_MARKER)[0].encode()).hexdigest()[:16]
+    import re
+    if text is None:
+        text = open(path).read()
+    code = text.split(HOST_SIDE_MARKER)[0]
+    code = re.sub(r"/\*.*?\*/", "", code, flags=re.S)
+    code = re.sub(r"//[^\n]*", "", code)
+    code = re.sub(r"\s+", "", code)
+    return hashlib.sha256(code.encode()).hexdigest()[:16]
 
 
 def profile_traffic(kernel_key: str):

@@ -13,9 +13,10 @@
 // quantised to 23-bit fixed point and split into three base-256 digits, are the B operand.
 // Stage 1 is a split-d_in reduction over thread-block clusters (one cluster per chunk of 256
 // outputs, one block per row slice of V) that sum their exact partials in distributed
-// shared memory; stage 2 gives every block a run of 16-row tiles of U with t's digit table in
-// shared memory.  The two kernels chain by programmatic dependent launch: each reads its
-// weights before it waits for the previous grid.
+// shared memory; its owner blocks hand t over already quantised, as stage 2's digit table.
+// Stage 2 gives every block a run of 16-row tiles of U and copies that table into shared
+// memory.  The two kernels chain by programmatic dependent launch: each reads its weights
+// before it waits for the previous grid.
 #include <cooperative_groups.h>
 
 #include <algorithm>
@@ -554,8 +555,9 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const __grid_const
 // ------------------------------------------------------------------ stage 2 (integer MMA)
 //
 // y[m][i] = s1_i * sum_k (2 u_ik - 1) t[m][k] with u in {0, 1} the packed bits of U.
-// t is quantised per batch row to a 23-bit fixed-point integer t_q = rint(t * 2^sh) (|t_q| <
-// 2^22) and split into three signed base-256 digits (planes) t_q = d0 + 2^8 d1 + 2^16 d2.
+// Stage 1 quantises t per batch row to a 23-bit fixed-point integer t_q = rint(t * 2^sh)
+// (|t_q| <= 2^22, sh from a bound on |t|), split into three signed base-256 digits (planes)
+// t_q = d0 + 2^8 d1 + 2^16 d2, and writes them as this kernel's B table.
 // The packed words feed mma.sync m16n8k32 (A u8, B s8, D s32) directly: for a bit offset
 // s in 0..7 the register  word & (0x01010101 << s)  holds, in its four bytes, the bits
 // s, s+8, s+16, s+24 of the word as the values {0, 2^s} -- four K elements for one AND.
