@@ -91,7 +91,9 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
                  : "memory");
 }
 
-template <int MODE>
+// SPLIT: the launch splits tiles over K (mode V); without it the unit of work is the tile and
+// the unit bookkeeping folds away at compile time.
+template <int MODE, bool SPLIT>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     lrb_umma_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant__ CUtensorMap tmap_bits,
                     const PrefillArgs args) {
@@ -150,7 +152,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int nkb = args.n_kblocks;
     unsigned int* err = args.err;
     // work unit u: tile u / ksplit, k blocks [kb_lo, kb_hi) of split u % ksplit
-    const int ksplit = (MODE == kModeV) ? args.ksplit : 1;
+    const int ksplit = (MODE == kModeV && SPLIT) ? args.ksplit : 1;
     const int n_units = n_tiles * ksplit;
     auto unit_kb = [&](int u, int& kb_lo, int& kb_hi) {
         const int sp = u % ksplit;
@@ -671,15 +673,15 @@ int umma_stages(int tile_n) {
     return st;
 }
 
-template <int MODE>
-nq_status launch_umma(const nq::PrefillArgs& a, const CUtensorMap& map, const CUtensorMap& bits_map, cudaStream_t stream,
-                      bool pdl) {
+template <int MODE, bool SPLIT>
+nq_status launch_umma_t(const nq::PrefillArgs& a, const CUtensorMap& map, const CUtensorMap& bits_map,
+                        cudaStream_t stream, bool pdl) {
     static bool attr_done[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     const size_t smem = kUmmaSmemBudget;
     if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-        if (cudaFuncSetAttribute(nq::lrb_umma_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(nq::lrb_umma_kernel<MODE, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(smem)) != cudaSuccess)
             return NQ_ERR_LAUNCH;
         attr_done[dev] = true;
@@ -691,11 +693,20 @@ nq_status launch_umma(const nq::PrefillArgs& a, const CUtensorMap& map, const CU
     args.stages = umma_stages(a.tile_n);
     CUtensorMap tm = map, tb = bits_map;
     void* kargs[] = {&tm, &tb, &args};
-    return nq_host::launch_pdl(reinterpret_cast<const void*>(nq::lrb_umma_kernel<MODE>), dim3(grid),
+    return nq_host::launch_pdl(reinterpret_cast<const void*>(nq::lrb_umma_kernel<MODE, SPLIT>), dim3(grid),
                                dim3(nq::kPrefillThreads), umma_smem_bytes(a.tile_n, args.stages), stream, kargs,
                                pdl) == cudaSuccess
                ? NQ_OK
                : NQ_ERR_LAUNCH;
+}
+
+template <int MODE>
+nq_status launch_umma(const nq::PrefillArgs& a, const CUtensorMap& map, const CUtensorMap& bits_map, cudaStream_t stream,
+                      bool pdl) {
+    if constexpr (MODE == nq::kModeV) {
+        if (a.ksplit > 1) return launch_umma_t<MODE, true>(a, map, bits_map, stream, pdl);
+    }
+    return launch_umma_t<MODE, false>(a, map, bits_map, stream, pdl);
 }
 
 }  // namespace

@@ -97,9 +97,12 @@ def test_full_size_70b_gate_sampled(M):
     p = synth.make_workload("prefill70b")[0]
     xb = synth.make_input("prefill70b", p.d_in, M, key=M)
     y = gpu_matmul(p, xb)
-    rows = np.unique(np.concatenate([[0, 127, 128, p.d_out - 1], np.linspace(0, p.d_out - 1, 40).astype(np.int64)]))
+    # rows of the last weight tiles too
+    tail = [p.d_out - 512, p.d_out - 300, p.d_out - 129, p.d_out - 128, p.d_out - 1]
+    rows = np.unique(np.concatenate([[0, 127, 128], tail, np.linspace(0, p.d_out - 1, 40).astype(np.int64)]))
     y_ref, S = oracle.dense_packed(p.U, p.V, p.s1, p.s2, p.r, xb, rows=rows)
     check_tolerance(y[:, rows], y_ref, S, "prefill 70B gate M=%d" % M)
+
 
 
 def test_layer_forward_dispatches_to_matmul_and_is_deterministic():
