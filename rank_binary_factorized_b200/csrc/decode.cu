@@ -152,6 +152,18 @@ __device__ __forceinline__ void byte_transpose4(uint32_t w0, uint32_t w1, uint32
     o[3] = __byte_perm(t1, t3, 0x7632);
 }
 
+// 2^e as a double, written into the exponent field (|e| <= 1022)
+__device__ __forceinline__ double pow2_d(int e) { return __longlong_as_double(static_cast<long long>(1023 + e) << 52); }
+
+// Shift for a bound L >= 0 on |t|: with L < 2^e, |t * 2^(22 - e)| < 2^22.  The exponent comes
+// from the bits of L, which is a normal double here (a positive L is at least 2^-126).
+__device__ __forceinline__ int shift_for_bound(double L) {
+    if (!(L > 0.0)) return 0;
+    const int biased = static_cast<int>((__double_as_longlong(L) >> 52) & 0x7ff);
+    const int e = biased - 1022;  // L = f 2^e with 0.5 <= f < 1
+    return min(max(22 - e, -126), 126);
+}
+
 // GN: 1 for a single layer (member 0, resolved at compile time), kMaxGroup for a group.
 template <int NT, int TH, int GN>
 __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const __grid_constant__ S1Group grp) {
@@ -484,14 +496,18 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const __grid_const
             cluster.map_shared_rank(bound, owner)[m * CS + q] = static_cast<double>(s_zabs[m]) * s_dinv[m];
         }
     cluster.sync();
-    // one shift per batch row for t: |t| <= L = sum over the slices, in rank order (the same
-    // value in every thread, block and cluster), so |t_q| <= 2^22
+    // one shift per batch row for t: |t| <= L = the sum over the slices, taken as a fixed
+    // pairwise tree over 16 leaves (ranks past CS are zeros, which add exactly), so L is the
+    // same value in every thread, block and cluster, and |t_q| <= 2^22
     auto t_shift = [&](int m) {
-        double L = 0.0;
-        for (int rank = 0; rank < CS; ++rank) L += bound[m * CS + rank];
-        int e = 0;
-        frexp(L, &e);  // L < 2^e
-        return (L > 0.0) ? min(max(22 - e, -126), 126) : 0;
+        double v[16];
+#pragma unroll
+        for (int rank = 0; rank < 16; ++rank) v[rank] = (rank < CS) ? bound[m * CS + rank] : 0.0;
+#pragma unroll
+        for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+            for (int i = 0; i < w; ++i) v[i] = v[i] + v[i + w];
+        return shift_for_bound(v[0]);
     };
     if (p.tab && chunk == 0 && q == 0 && tid < p.M) p.tsh[tid] = t_shift(tid);
     {
@@ -520,7 +536,7 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const __grid_const
             if (p.tab) {
                 // t_q's three digits, byte (k / 8) % 4 of the table words for (k % 8, k / 32);
                 // outputs past r (up to the padded word count) get zero digits
-                const int tq = (k < p.r) ? __double2int_rn(sum * ldexp(1.0, t_shift(m))) : 0;
+                const int tq = (k < p.r) ? __double2int_rn(sum * pow2_d(t_shift(m))) : 0;
 #pragma unroll
                 for (int mm = 0; mm < MG; ++mm)
                     if (mm == m) tqacc[mm] += tq;
@@ -664,14 +680,24 @@ __global__ void __launch_bounds__(TH, 1) decode_stage2_kernel(const __grid_const
         const int pieces = 2 * p.nwp * NT * 8;  // 16-byte pieces of 8 nwp NT 8 words
         for (int c = tid; c < pieces; c += kS2Threads) cp_async16(dst + 16u * c, p.tab + 4 * c);
         asm volatile("cp.async.commit_group;" ::: "memory");
-        // warp m adds row m's owner sums (exact integers), lane 0 keeps the result
+        // warp m adds row m's owner sums (exact integers), lane 0 keeps the result; each lane
+        // issues its loads four at a time, so the sums cost one round trip to L2
         for (int m = warp; m < p.M; m += kS2Warps) {
+            const int sh = p.tsh[m];
             long long v = 0;
-            for (int i = lane; i < p.tsum_n; i += 32) v += p.tsum[static_cast<int64_t>(i) * p.M + m];
+            for (int i0 = lane; i0 < p.tsum_n; i0 += 4 * 32) {
+                long long a[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int i = i0 + 32 * u;
+                    a[u] = (i < p.tsum_n) ? p.tsum[static_cast<int64_t>(i) * p.M + m] : 0ll;
+                }
+                v += (a[0] + a[1]) + (a[2] + a[3]);
+            }
             for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
             if (lane == 0) {
                 s_tsum[m] = static_cast<unsigned long long>(v);
-                s_dinv[m] = ldexp(1.0, -p.tsh[m]);
+                s_dinv[m] = pow2_d(-sh);
             }
         }
     }
