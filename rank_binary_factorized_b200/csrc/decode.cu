@@ -94,7 +94,7 @@ __device__ __forceinline__ int s2_bidx(int s_, int w, int col, int ng) {
 // Blocks form a thread-block cluster along d_in: block (c, q) owns word chunk c (8 words =
 // 256 outputs k) and row slice q of V.  Each block turns its exact integer partial into an
 // fp64 value with its own scale; after a cluster barrier, block q sums a 1/CS share of the
-// chunk's outputs over the CS blocks' shared memory (distributed shared memory) in rank
+// chunk's outputs over the CS blocks' shared memory (distributed shared memory) in a fixed
 // order and writes t.  No atomics, no global partials: deterministic.
 
 // Threads per stage-1 block: 256 (one warp per word column) or 512 (two warps per word column,
@@ -473,7 +473,7 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const __grid_const
     // ---- cluster reduction over the CS row slices.  Output k of the chunk belongs to the
     // block of rank k / per; every block stores its fp64 partial for k into slot [rank of
     // the sender] of the owner's inbox (distributed shared memory), one cluster barrier
-    // publishes the stores, and each owner sums its slots in rank order.
+    // publishes the stores, and each owner sums its slots in a fixed order.
     // CS is a power of two (1 .. 16), so is the share per owner; the exact integer times the
     // power of two 2^-shift is exact in fp64
     const int lg_per = 8 - (31 - __clz(CS));  // log2(kS1Outs / CS)
