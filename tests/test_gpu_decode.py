@@ -15,7 +15,8 @@ import torch
 
 import oracle
 from rank_binary_factorized_b200 import synth
-from tests.gpu_util import (check_tolerance, download_bf16_bits, need_gpu, nq, upload_bf16, upload_projection)
+from tests.gpu_util import (bf16_bits_to_f64, check_tolerance, download_bf16_bits, need_gpu, nq, upload_bf16,
+                            upload_projection)
 
 pytestmark = pytest.mark.gpu
 
@@ -72,6 +73,21 @@ def test_integer_exact_bitwise(d_out, d_in, r, M):
     rows = np.arange(d_out) if d_out <= 1024 else np.linspace(0, d_out - 1, 257).astype(np.int64)
     y_ref, _ = oracle.dense_packed(p.U, p.V, p.s1, p.s2, p.r, xb, rows=rows)
     np.testing.assert_array_equal(y[:, rows], oracle.round_bf16(y_ref))
+
+
+def test_per_row_magnitudes_and_zero_row():
+    """Each batch row gets its own fixed-point shifts (for z and for t): rows scaled by 2^-40,
+    2^-8, 1 and 2^20 (exact power-of-two scalings in bf16) and an all-zero row, in one call,
+    each within its own tolerance; the zero row comes out exactly zero."""
+    need_gpu()
+    p = synth.make_workload("tiny")[0]
+    xf = synth.rng_for(211, 5).standard_normal((5, p.d_in)).astype(np.float32)
+    xf *= np.array([2.0 ** -40, 2.0 ** -8, 1.0, 2.0 ** 20, 0.0], dtype=np.float32)[:, None]
+    xb = synth.f32_to_bf16_bits(xf)
+    y = gpu_forward(p, xb)
+    y_ref, S = oracle.dense_packed(p.U, p.V, p.s1, p.s2, p.r, xb)
+    check_tolerance(y, y_ref, S, "per-row magnitudes")
+    assert np.all(bf16_bits_to_f64(y[4]) == 0.0)
 
 
 def test_every_sign_pattern_4x2_bitwise():
