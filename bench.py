@@ -297,12 +297,14 @@ def gpu_arm(args, rank, world, local):
         "higher_is_better": False,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "f32",
+        "dtype": "int32",
         "data": "synthetic (seeded iid +-1 signs, fp16 0.02|N(0,1)| scales, bf16 N(0,1) activations)",
         "config": {
             "workload": "Llama-2-7B attention projection d_out=d_in=4096 r=2048 (1.0 bit/weight), decode batch %d" % M,
             "batch": M,
-            "operands": "1-bit packed U, V (uint32 words); fp16 s1, s2; bf16 x, y; fp32 accumulate",
+            "operands": "1-bit packed U, V (uint32 words); fp16 s1, s2; bf16 x, y",
+            "arithmetic": "s2 x in fp32, fixed-point per batch row (23-bit integers); sign products on u8 x s8 "
+                          "MMAs with exact int32 accumulation; fp64 sums across row slices; fp32 scale by s1, bf16 out",
             "layers_per_step": n,
             "chain": "y of each layer is x of the next (distinct weights per layer)",
             "l2": "no flush: %d distinct layers = %.0f MB of weights per step > 3x L2" % (n, chain.weight_bytes / 1e6),
