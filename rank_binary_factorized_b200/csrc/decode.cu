@@ -17,11 +17,11 @@
 // Stage 2 gives every block a run of 16-row tiles of U and copies that table into shared
 // memory.  The two kernels chain by programmatic dependent launch: each reads its weights
 // before it waits for the previous grid.
+#include <cooperative_groups.h>
 
 #include <algorithm>
 
 #include "nq_common.cuh"
-#include "tc_common.cuh"
 
 namespace nq {
 
@@ -133,11 +133,7 @@ struct S1Group {
     S1Params p[kMaxGroup];
     int chunk_off[kMaxGroup + 1];
     int n;
-    unsigned int* err;  // the library's error word (a bounded wait that gives up sets a bit)
 };
-
-// Longest wait of a stage-1 block for its inbox (the other slices' partials).
-constexpr uint64_t kInboxWaitNs = 200000000ull;  // 0.2 s
 
 template <int NT>
 struct S1Layout {
@@ -173,6 +169,7 @@ template <int NT, int TH, int GN>
 __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const __grid_constant__ S1Group grp) {
     constexpr int kS1Threads = TH;
     constexpr int kKSplit = kS1Threads / (32 * kS1Words);  // warps per word column
+    namespace cg = cooperative_groups;
     constexpr int SWZ = S1Layout<NT>::SWZ;
     extern __shared__ __align__(16) uint32_t smem1[];
     int li = 0;  // the member of the group this block works for
@@ -195,28 +192,12 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const __grid_const
     __shared__ long long s_tqsum[NQ_MATVEC_MAX_M];          // owner's sum of t_q
     __shared__ float s_wmax[kS1Threads / 32][NQ_MATVEC_MAX_M];
 
+    cg::cluster_group cluster = cg::this_cluster();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int gid = lane >> 2, tig = lane & 3;
 
     const int q = blockIdx.y;  // slice index == rank in the cluster
     const int CS = gridDim.y;
-    const int lg_per = 8 - (31 - __clz(CS));  // log2(kS1Outs / CS): outputs each block owns
-    const int per = 1 << lg_per;
-
-    // The inbox barrier completes once every other slice's partials (and bounds) for this
-    // block's outputs have landed in `part`: the senders' st.async stores count their bytes
-    // against it.  Initialised and armed before the cluster barrier's arrive, which the
-    // senders wait for before their first store.
-    __shared__ __align__(8) unsigned long long s_inbox;
-    const uint32_t inbox = tc::smem_u32(&s_inbox);
-    if (tid == 0) {
-        const uint32_t incoming = 8u * static_cast<uint32_t>(p.M) * static_cast<uint32_t>(CS - 1) *
-                                  static_cast<uint32_t>(per + (p.tab ? 1 : 0));
-        tc::mbar_init(inbox, 1);
-        tc::mbar_arrive_expect_tx(inbox, incoming);
-        tc::mbar_fence_init();
-    }
-    tc::cluster_arrive_relaxed();
     const int64_t j0 = static_cast<int64_t>(q) * p.rows_per_slice;
     const int64_t j1 = min(p.d_in, j0 + p.rows_per_slice);
     const int wglob0 = chunk * kS1Words;
@@ -491,12 +472,12 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const __grid_const
     __syncthreads();
     // ---- cluster reduction over the CS row slices.  Output k of the chunk belongs to the
     // block of rank k / per; every block stores its fp64 partial for k into slot [rank of
-    // the sender] of the owner's inbox (distributed shared memory, st.async stores whose bytes
-    // the owner's inbox barrier counts), and each owner, once its inbox is complete, sums its
-    // slots in a fixed order.
+    // the sender] of the owner's inbox (distributed shared memory), one cluster barrier
+    // publishes the stores, and each owner sums its slots in a fixed order.
     // CS is a power of two (1 .. 16), so is the share per owner; the exact integer times the
     // power of two 2^-shift is exact in fp64
-    tc::cluster_wait_acquire();  // every block of the cluster has armed its inbox
+    const int lg_per = 8 - (31 - __clz(CS));  // log2(kS1Outs / CS)
+    const int per = 1 << lg_per;
     for (int e = tid; e < p.M * kS1Outs; e += kS1Threads) {
         const int m = e / kS1Outs, kl = e - m * kS1Outs;
         const int* rr = red + kl * (NT * 8) + 3 * m;
@@ -504,29 +485,17 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const __grid_const
                             (static_cast<long long>(rr[2]) << 16);
         const long long val = 2 * P - static_cast<long long>(s_zsum[m]);
         const int owner = kl >> lg_per, ko = kl & (per - 1);
-        const double v = static_cast<double>(val) * s_dinv[m];
-        double* slot = part + (m * per + ko) * CS + q;
-        if (owner == q) *slot = v;
-        else tc::st_async_b64(tc::map_to_rank(tc::smem_u32(slot), owner), static_cast<uint64_t>(__double_as_longlong(v)),
-                              tc::map_to_rank(inbox, owner));
+        double* dst = cluster.map_shared_rank(part, owner);
+        dst[(m * per + ko) * CS + q] = static_cast<double>(val) * s_dinv[m];
     }
     // the slice's bound on its share of |t| (exact), into every owner's inbox after the partials
     double* bound = part + p.M * kS1Outs;  // [M][CS]
     if (p.tab)
         for (int e = tid; e < p.M * CS; e += kS1Threads) {
             const int m = e / CS, owner = e - m * CS;
-            const double v = static_cast<double>(s_zabs[m]) * s_dinv[m];
-            double* slot = bound + m * CS + q;
-            if (owner == q) *slot = v;
-            else tc::st_async_b64(tc::map_to_rank(tc::smem_u32(slot), owner),
-                                  static_cast<uint64_t>(__double_as_longlong(v)), tc::map_to_rank(inbox, owner));
+            cluster.map_shared_rank(bound, owner)[m * CS + q] = static_cast<double>(s_zabs[m]) * s_dinv[m];
         }
-    __syncthreads();  // this block's own slots
-    tc::mbar_wait_cluster_for(inbox, 0u, grp.err, kInboxWaitNs);  // the other slices' slots
-    __syncthreads();
-    // no block leaves before every inbox of the cluster is complete, so no store is still in
-    // flight to or from it; the wait half is at the end of the kernel
-    tc::cluster_arrive_release();
+    cluster.sync();
     // one shift per batch row for t: |t| <= L = the sum over the slices, taken as a fixed
     // pairwise tree over 16 leaves (ranks past CS are zeros, which add exactly), so L is the
     // same value in every thread, block and cluster, and |t_q| <= 2^22
@@ -597,7 +566,6 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const __grid_const
             if (tid < p.M) p.tsum[(static_cast<int64_t>(chunk) * CS + q) * p.M + tid] = s_tqsum[tid];
         }
     }
-    tc::cluster_wait_acquire();
 }
 
 // ------------------------------------------------------------------ stage 2 (integer MMA)
@@ -944,7 +912,6 @@ nq_status launch_decode_group_nt(const nq_lrb_layer* const* Ls, int n, const uin
         cs1 = sp.CS;
         nq::S1Group g{};
         g.n = n;
-        g.err = nq_host::error_word();
         int acc = 0;
         for (int l = 0; l < n; ++l) {
             const nq_lrb_layer* L = Ls[l];
@@ -1060,7 +1027,6 @@ nq_status launch_stage1_pair_nt(const nq_lrb_layer* L0, const uint16_t* x0, floa
     S1Plan sp[2] = {plan_stage1(L0->d_in, total, M, cs), plan_stage1(L1->d_in, total, M, cs)};
     nq::S1Group g{};
     g.n = 2;
-    g.err = nq_host::error_word();
     int acc = 0;
     for (int l = 0; l < 2; ++l) {
         const nq_lrb_layer* L = Ls[l];

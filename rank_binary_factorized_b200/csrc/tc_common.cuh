@@ -1,6 +1,5 @@
-// tc_common.cuh -- thin inline-PTX wrappers for the sm_100a machinery used by the kernels:
-// mbarriers, cluster barrier halves and remote shared-memory stores (decode), TMA tile loads
-// (no multicast), tcgen05 MMA / TMEM (prefill).
+// tc_common.cuh -- thin inline-PTX wrappers for the sm_100a tensor-core machinery used by
+// the prefill kernels: mbarriers, TMA tile loads (no multicast), tcgen05 MMA / TMEM.
 // Written from the public PTX ISA descriptions of these instructions.
 #pragma once
 
@@ -69,58 +68,6 @@ __device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, uns
 }
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned int* err) {
     return mbar_wait_for(bar, parity, err, kWaitLimitNs);
-}
-
-// The same bounded wait with acquire semantics at cluster scope, for a barrier whose
-// transactions are stores from other CTAs of the cluster (st.async).
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-__device__ __forceinline__ bool mbar_wait_cluster_for(uint32_t bar, uint32_t parity, unsigned int* err, uint64_t limit_ns) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
-    for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait_cluster(bar, parity)) return true;
-        if ((i & 255u) == 0u && globaltimer_ns() - t0 > limit_ns) {
-            if (err != nullptr) flag_error(err, kErrTimeout);
-            return false;
-        }
-    }
-}
-
-// ------------------------------------------------------------------ cluster: barrier halves, remote stores
-// barrier.cluster split into its arrive and wait halves (every thread of every CTA of the
-// cluster executes each once per use).  The relaxed arrive orders nothing; it pairs with
-// fence.mbarrier_init to publish mbarrier initialisation to the cluster.
-__device__ __forceinline__ void cluster_arrive_relaxed() {
-    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_arrive_release() {
-    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait_acquire() {
-    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// The shared::cluster address of the same shared-memory offset in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t map_to_rank(uint32_t local_smem, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_smem), "r"(rank));
-    return r;
-}
-// 8-byte store into another CTA's shared memory; its completion counts 8 bytes against the
-// transaction count of the mbarrier `remote_bar` in that same CTA.
-__device__ __forceinline__ void st_async_b64(uint32_t remote_addr, uint64_t v, uint32_t remote_bar) {
-    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b64 [%0], %1, [%2];" ::"r"(remote_addr),
-                 "l"(v), "r"(remote_bar)
-                 : "memory");
 }
 
 // ------------------------------------------------------------------ TMA (tile mode, no multicast)
