@@ -810,6 +810,8 @@ __global__ void __launch_bounds__(TH, 1) decode_stage2_kernel(const __grid_const
 }  // namespace nq
 
 // ------------------------------------------------------------------------------ host side
+#include <atomic>
+
 namespace {
 
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
@@ -877,16 +879,16 @@ size_t decode_ws_bytes(int64_t r, int64_t M) { return kWsHeader + t_layout(r, M)
 
 template <int NT, int TH1, int TH2, int GN>
 void set_attrs_once() {
-    static bool done[64] = {};
+    static std::atomic<bool> done[64];  // per device; setting an attribute twice is harmless
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64 || done[dev]) return;
+    if (dev < 0 || dev >= 64 || done[dev].load(std::memory_order_acquire)) return;
     cudaFuncSetAttribute(nq::decode_stage1_kernel<NT, TH1, GN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(kStage1SmemBudget));
     cudaFuncSetAttribute(nq::decode_stage1_kernel<NT, TH1, GN>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     cudaFuncSetAttribute(nq::decode_stage2_kernel<NT, TH2, GN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(kStage2SmemBudget));
-    done[dev] = true;
+    done[dev].store(true, std::memory_order_release);
 }
 
 // One launch of each stage for n projections that share x (n = 1: a single layer).

@@ -543,6 +543,8 @@ __global__ void __launch_bounds__(256) grad_reduce_kernel(const double* __restri
 }  // namespace nq
 
 // ------------------------------------------------------------------------------ host side
+#include <atomic>
+
 namespace {
 
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
@@ -676,15 +678,15 @@ int umma_stages(int tile_n) {
 template <int MODE, bool SPLIT>
 nq_status launch_umma_t(const nq::PrefillArgs& a, const CUtensorMap& map, const CUtensorMap& bits_map,
                         cudaStream_t stream, bool pdl) {
-    static bool attr_done[64] = {};
+    static std::atomic<bool> attr_done[64];  // per device; setting an attribute twice is harmless
     int dev = 0;
     cudaGetDevice(&dev);
     const size_t smem = kUmmaSmemBudget;
-    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+    if (dev >= 0 && dev < 64 && !attr_done[dev].load(std::memory_order_acquire)) {
         if (cudaFuncSetAttribute(nq::lrb_umma_kernel<MODE, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(smem)) != cudaSuccess)
             return NQ_ERR_LAUNCH;
-        attr_done[dev] = true;
+        attr_done[dev].store(true, std::memory_order_release);
     }
     const int units = a.n_tiles_w * a.n_tiles_n * ((MODE == nq::kModeV && a.ksplit > 1) ? a.ksplit : 1);
     int grid = nq_host::sm_count();

@@ -325,6 +325,8 @@ __global__ void __launch_bounds__(kSgThreads, 1)
 }  // namespace nq
 
 // ------------------------------------------------------------------------------ host side
+#include <atomic>
+
 namespace {
 
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
@@ -457,14 +459,14 @@ nq_status nq_launch_sign_grads(const nq_lrb_layer* L, const nq_lrb_layer* X, con
     a.stages = stages;
     const size_t smem = sg_smem_bytes(a.tile_n, stages);
 
-    static bool attr_done[64] = {};
+    static std::atomic<bool> attr_done[64];  // per device; setting an attribute twice is harmless
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+    if (dev >= 0 && dev < 64 && !attr_done[dev].load(std::memory_order_acquire)) {
         if (cudaFuncSetAttribute(nq::sign_grads_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(kSgSmemMax)) != cudaSuccess)
             return NQ_ERR_LAUNCH;
-        attr_done[dev] = true;
+        attr_done[dev].store(true, std::memory_order_release);
     }
     int grid = nq_host::sm_count();
     if (grid > a.n_tiles) grid = a.n_tiles;
