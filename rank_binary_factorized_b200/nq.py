@@ -1,6 +1,7 @@
 """Thin Python binding of libnq.so (include/nq.h) -- argument marshalling only.
 
-Every step of the LRB path runs in the CUDA library; this module turns torch tensors into
+Every step of the LRB path runs in the CUDA library; this module checks tensor arguments
+(CUDA device, dtype, shape, layout: the C ABI cannot see a tensor's extent), turns them into
 device pointers and the current torch stream into a ``cudaStream_t``.  PyTorch provides
 device memory and streams, nothing else.  If ``libnq.so`` is missing the import fails: there
 is no other implementation to fall back to.
@@ -107,10 +108,49 @@ def _ptr(t) -> int:
     return 0 if t is None else int(t.data_ptr())
 
 
+def _need(t, name: str, dtype, shape=None, device=None, contiguous: bool = True) -> None:
+    """Checks a tensor argument before its address reaches the library, which reads device
+    memory only and at the layout nq.h states: a CUDA tensor of the given dtype (and shape and
+    device), contiguous unless the call takes a row stride."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s: expected a torch.Tensor, got %s" % (name, type(t).__name__))
+    if not t.is_cuda:
+        raise ValueError("%s: expected a CUDA tensor, got one on %s" % (name, t.device))
+    if t.dtype != dtype:
+        raise ValueError("%s: expected dtype %s, got %s" % (name, dtype, t.dtype))
+    if shape is not None and tuple(t.shape) != tuple(int(d) for d in shape):
+        raise ValueError("%s: expected shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+    if device is not None and t.device != device:
+        raise ValueError("%s: on %s, the layer's tensors on %s" % (name, t.device, device))
+    if contiguous and not t.is_contiguous():
+        raise ValueError("%s: expected a contiguous tensor" % name)
+
+
+def _need_rows(t, name: str, dtype, rows: int, min_cols: int, device=None) -> None:
+    """A 2-D CUDA tensor with `rows` rows of at least `min_cols` columns and unit column stride
+    (the call takes its row stride)."""
+    _need(t, name, dtype, device=device, contiguous=False)
+    if t.dim() != 2 or int(t.shape[0]) != rows or int(t.shape[1]) < min_cols or t.stride(1) != 1:
+        raise ValueError("%s: expected [%d][>= %d] with unit column stride, got shape %s strides %s" %
+                         (name, rows, min_cols, tuple(t.shape), tuple(t.stride())))
+
+
+def _need_ws(ws, layer_device) -> None:
+    _need(ws, "ws", torch.uint8, device=layer_device)
+
+
 class Layer:
     """A device-resident LRB layer: packed U, V (int32 words), fp16 s1, s2."""
 
     def __init__(self, U: torch.Tensor, V: torch.Tensor, s1: torch.Tensor, s2: torch.Tensor, r: int):
+        _need(U, "U", torch.int32)
+        if U.dim() != 2:
+            raise ValueError("U: expected [d_out][ldu] words, got shape %s" % (tuple(U.shape),))
+        _need(V, "V", torch.int32, device=U.device)
+        if V.dim() != 2:
+            raise ValueError("V: expected [d_in][ldv] words, got shape %s" % (tuple(V.shape),))
+        _need(s1, "s1", torch.float16, shape=(U.shape[0],), device=U.device)
+        _need(s2, "s2", torch.float16, shape=(V.shape[0],), device=U.device)
         self.U, self.V, self.s1, self.s2 = U, V, s1, s2
         self.d_out, self.ldu = int(U.shape[0]), int(U.shape[1])
         self.d_in, self.ldv = int(V.shape[0]), int(V.shape[1])
@@ -163,24 +203,33 @@ class Layer:
 def pack_signs(latent: torch.Tensor, r: int | None = None, ld_words: int | None = None, out=None,
                stream=None) -> torch.Tensor:
     """sign(latent) >= 0 packed 32 per word along r (bit k%32 of word k/32)."""
-    if latent.dim() != 2 or latent.stride(1) != 1 or latent.dtype != torch.float32:
+    _need(latent, "latent", torch.float32, contiguous=False)
+    if latent.dim() != 2 or latent.stride(1) != 1:
         raise ValueError("latent must be a 2-D float32 tensor with unit column stride")
     rows, ld_latent = int(latent.shape[0]), int(latent.stride(0))
     r = int(latent.shape[1]) if r is None else int(r)
+    if r > int(latent.shape[1]):
+        raise ValueError("r = %d exceeds the latent's %d columns" % (r, int(latent.shape[1])))
     ld_words = r // 32 if ld_words is None else int(ld_words)
     if out is None:
         out = torch.empty((rows, ld_words), dtype=torch.int32, device=latent.device)
+    _need(out, "out", torch.int32, shape=(rows, ld_words), device=latent.device)
     _check("nq_pack_signs", _lib.nq_pack_signs(_ptr(latent), rows, r, ld_latent, _ptr(out), ld_words,
                                                _stream_ptr(stream)))
     return out
 
 
 def _forward(fn_name: str, layer: Layer, x: torch.Tensor, y=None, ws=None, stream=None) -> torch.Tensor:
+    dev = layer.U.device
+    _need(x, "x", torch.bfloat16, device=dev)
     M = int(x.shape[0])
+    _need(x, "x", torch.bfloat16, shape=(M, layer.d_in))
     if y is None:
         y = torch.empty((M, layer.d_out), dtype=torch.bfloat16, device=x.device)
+    _need(y, "y", torch.bfloat16, shape=(M, layer.d_out), device=dev)
     if ws is None:
         ws = layer.workspace(M)
+    _need_ws(ws, dev)
     fn = getattr(_lib, fn_name)
     _check(fn_name, fn(ctypes.byref(layer.struct), _ptr(x), _ptr(y), M, _ptr(ws), ws.numel(), _stream_ptr(stream)))
     return y
@@ -200,11 +249,16 @@ def layer_forward(layer: Layer, x: torch.Tensor, y=None, ws=None, stream=None) -
 
 def lrb_transposed(layer: Layer, ybar: torch.Tensor, xbar=None, ws=None, stream=None) -> torch.Tensor:
     """xbar = the layer's transpose applied to ybar ([M][d_out] bf16 -> [M][d_in] bf16)."""
+    dev = layer.U.device
+    _need(ybar, "ybar", torch.bfloat16, device=dev)
     M = int(ybar.shape[0])
+    _need(ybar, "ybar", torch.bfloat16, shape=(M, layer.d_out))
     if xbar is None:
         xbar = torch.empty((M, layer.d_in), dtype=torch.bfloat16, device=ybar.device)
+    _need(xbar, "xbar", torch.bfloat16, shape=(M, layer.d_in), device=dev)
     if ws is None:
         ws = layer.workspace(M)
+    _need_ws(ws, dev)
     _check("nq_lrb_transposed", _lib.nq_lrb_transposed(ctypes.byref(layer.struct), _ptr(ybar), _ptr(xbar), M,
                                                        _ptr(ws), ws.numel(), _stream_ptr(stream)))
     return xbar
@@ -212,11 +266,16 @@ def lrb_transposed(layer: Layer, ybar: torch.Tensor, xbar=None, ws=None, stream=
 
 def lrb_scale_grads(layer: Layer, x: torch.Tensor, ybar: torch.Tensor, ws=None, stream=None):
     """(dL/ds1 [d_out], dL/ds2 [d_in]) fp32 for L = sum <ybar, layer(x)>."""
+    dev = layer.U.device
+    _need(x, "x", torch.bfloat16, device=dev)
     M = int(x.shape[0])
+    _need(x, "x", torch.bfloat16, shape=(M, layer.d_in))
+    _need(ybar, "ybar", torch.bfloat16, shape=(M, layer.d_out), device=dev)
     g1 = torch.empty(layer.d_out, dtype=torch.float32, device=x.device)
     g2 = torch.empty(layer.d_in, dtype=torch.float32, device=x.device)
     if ws is None:
         ws = layer.workspace(M)
+    _need_ws(ws, dev)
     _check("nq_lrb_scale_grads", _lib.nq_lrb_scale_grads(ctypes.byref(layer.struct), _ptr(x), _ptr(ybar), M,
                                                          _ptr(g1), _ptr(g2), _ptr(ws), ws.numel(),
                                                          _stream_ptr(stream)))
@@ -234,17 +293,21 @@ def lrb_sign_grads(layer: Layer, x: torch.Tensor, ybar: torch.Tensor, gU=None, g
     """(dL/dU [d_out][r], dL/dV [d_in][r]) fp32 for L = sum <ybar, layer(x)>: the gradients the
     identity straight-through estimator passes to the latent factors.  gU, gV may be given
     ([rows][ld] fp32 with ld >= r a multiple of 4); only their first r columns are written."""
+    dev = layer.U.device
+    _need(x, "x", torch.bfloat16, device=dev)
     M = int(x.shape[0])
+    _need(x, "x", torch.bfloat16, shape=(M, layer.d_in))
+    _need(ybar, "ybar", torch.bfloat16, shape=(M, layer.d_out), device=dev)
     r = layer.r
     if gU is None:
         gU = torch.empty((layer.d_out, r), dtype=torch.float32, device=x.device)
     if gV is None:
         gV = torch.empty((layer.d_in, r), dtype=torch.float32, device=x.device)
-    for g in (gU, gV):
-        if g.dtype != torch.float32 or g.dim() != 2 or g.stride(1) != 1:
-            raise ValueError("gradients must be 2-D float32 with unit column stride")
+    _need_rows(gU, "gU", torch.float32, layer.d_out, r, device=dev)
+    _need_rows(gV, "gV", torch.float32, layer.d_in, r, device=dev)
     if ws is None:
         ws = torch.empty(sign_grads_workspace_bytes(layer, M), dtype=torch.uint8, device=x.device)
+    _need_ws(ws, dev)
     _check("nq_lrb_sign_grads", _lib.nq_lrb_sign_grads(ctypes.byref(layer.struct), _ptr(x), _ptr(ybar), M, _ptr(gU),
                                                        gU.stride(0), _ptr(gV), gV.stride(0), _ptr(ws), ws.numel(),
                                                        _stream_ptr(stream)))
@@ -255,9 +318,9 @@ def lrb_from_latent(Uh: torch.Tensor, Vh: torch.Tensor, r: int | None = None, ld
                     stream=None):
     """A device Layer from fp32 latent proxies Uh [d_out][r], Vh [d_in][r]: magnitude balancing,
     mean-absolute-value scales, packed signs.  Returns (Layer, eta as a 0-d fp64 tensor)."""
-    if Uh.dtype != torch.float32 or Vh.dtype != torch.float32 or Uh.stride(1) != 1 or Vh.stride(1) != 1:
-        raise ValueError("latents must be float32 with unit column stride")
     r = int(Uh.shape[1]) if r is None else int(r)
+    _need_rows(Uh, "Uh", torch.float32, int(Uh.shape[0]), r)
+    _need_rows(Vh, "Vh", torch.float32, int(Vh.shape[0]), r, device=Uh.device)
     d_out, d_in = int(Uh.shape[0]), int(Vh.shape[0])
     ld = -(-(r // 32) // ld_align_words) * ld_align_words
     dev = Uh.device
@@ -289,14 +352,27 @@ def group_workspace_bytes(layers, M: int) -> int:
 
 def layer_forward_group(layers, x: torch.Tensor, ys=None, ws=None, stream=None):
     """y_l = layers[l](x) for projections sharing x (one decode launch per stage for M <= 8)."""
+    if len(layers) == 0:
+        raise ValueError("layers: expected at least one layer")
+    dev = layers[0].U.device
+    _need(x, "x", torch.bfloat16, device=dev)
     M = int(x.shape[0])
+    for L in layers:
+        if L.U.device != dev:
+            raise ValueError("layers: all on one device")
+        _need(x, "x", torch.bfloat16, shape=(M, L.d_in))
     if ys is None:
         ys = [torch.empty((M, L.d_out), dtype=torch.bfloat16, device=x.device) for L in layers]
+    if len(ys) != len(layers):
+        raise ValueError("ys: expected one output per layer")
+    for i, (L, y) in enumerate(zip(layers, ys)):
+        _need(y, "ys[%d]" % i, torch.bfloat16, shape=(M, L.d_out), device=dev)
     if ws is None:
         need = group_workspace_bytes(layers, M)
         if need == 0:
             raise NQError("nq_group_workspace_bytes", 2)
         ws = torch.zeros(need, dtype=torch.uint8, device=x.device)
+    _need_ws(ws, dev)
     yp = (_p * len(ys))(*[_ptr(y) for y in ys])
     _check("nq_layer_forward_group", _lib.nq_layer_forward_group(_layer_array(layers), len(layers), _ptr(x), yp, M,
                                                                  _ptr(ws), ws.numel(), _stream_ptr(stream)))
@@ -304,8 +380,11 @@ def layer_forward_group(layers, x: torch.Tensor, ys=None, ws=None, stream=None):
 
 
 def silu_mul(g: torch.Tensor, u: torch.Tensor, h=None, stream=None) -> torch.Tensor:
+    _need(g, "g", torch.bfloat16)
+    _need(u, "u", torch.bfloat16, shape=tuple(g.shape), device=g.device)
     if h is None:
         h = torch.empty_like(g)
+    _need(h, "h", torch.bfloat16, shape=tuple(g.shape), device=g.device)
     _check("nq_silu_mul", _lib.nq_silu_mul(_ptr(g), _ptr(u), _ptr(h), g.numel(), _stream_ptr(stream)))
     return h
 

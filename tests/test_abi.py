@@ -214,3 +214,21 @@ def test_no_gpu_gives_device_error(nq):
     # valid arguments, no device: the call must refuse, not fall back to anything
     assert _call(nq, "nq_lrb_matvec", _layer(nq)) == NQ["DEVICE"]
     assert nq.raw_lib().nq_pack_signs(0x1000, 4, 64, 64, 0x2000, 2, None) == NQ["DEVICE"]
+
+
+def test_binding_refuses_host_tensors_before_any_call(nq):
+    """The binding checks tensor arguments before their addresses reach the library (which
+    reads device memory only): host tensors and wrong types raise, nothing is launched."""
+    import torch
+    U, V = torch.zeros((64, 2), dtype=torch.int32), torch.zeros((96, 2), dtype=torch.int32)
+    s1, s2 = torch.zeros(64, dtype=torch.float16), torch.zeros(96, dtype=torch.float16)
+    with pytest.raises(ValueError, match="CUDA"):
+        nq.Layer(U, V, s1, s2, 64)
+    with pytest.raises(TypeError):
+        nq.Layer(None, V, s1, s2, 64)
+    with pytest.raises(ValueError, match="CUDA"):
+        nq.pack_signs(torch.zeros((4, 64)))
+    with pytest.raises(ValueError, match="CUDA"):
+        nq.silu_mul(torch.zeros(8, dtype=torch.bfloat16), torch.zeros(8, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="CUDA"):
+        nq.lrb_from_latent(torch.zeros((8, 64)), torch.zeros((8, 64)))

@@ -198,3 +198,22 @@ def test_layer_forward_dispatch_small_batch():
     y1 = gpu_forward(p, xb, fn="layer_forward")
     y2 = gpu_forward(p, xb, fn="lrb_matvec")
     np.testing.assert_array_equal(y1, y2)
+
+
+def test_binding_rejects_mismatched_tensors():
+    """Wrong widths, dtypes, devices or layouts raise in the binding before the library is
+    called (the C ABI cannot see a tensor's extent)."""
+    need_gpu()
+    p = synth.make_workload("tiny")[0]
+    L = upload_projection(p)
+    x = upload_bf16(synth.make_input("tiny", p.d_in, 2))
+    for bad in (x[:, :-8].contiguous(), x.float(), x.cpu(), x.t().contiguous().t()):
+        with pytest.raises(ValueError):
+            nq().layer_forward(L, bad)
+    with pytest.raises(ValueError):
+        nq().layer_forward(L, x, y=torch.empty((2, p.d_out - 1), dtype=torch.bfloat16, device="cuda"))
+    with pytest.raises(ValueError):
+        nq().layer_forward(L, x, ws=torch.zeros(1 << 20, dtype=torch.int32, device="cuda"))
+    y = nq().layer_forward(L, x)  # the same call with valid arguments runs
+    nq().sync_status()
+    assert tuple(y.shape) == (2, p.d_out)
