@@ -185,7 +185,9 @@ class Layer:
         return int(_lib.nq_workspace_bytes(ctypes.byref(self.struct), M))
 
     def workspace(self, M: int) -> torch.Tensor:
-        """A zero-filled workspace large enough for M rows (cached per size)."""
+        """A zero-filled workspace large enough for M rows, cached on the layer and grown on
+        demand.  Every call on this layer that passes no ``ws`` uses it, so calls that may run
+        at the same time on the GPU (on different streams) must each pass their own ``ws``."""
         need = self.workspace_bytes(M)
         if need == 0:
             raise NQError("nq_workspace_bytes", 2)
