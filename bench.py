@@ -106,6 +106,28 @@ def profile_traffic(kernel_key: str):
     return None
 
 
+def nvml_index(local: int) -> int:
+    """NVML index of this rank's GPU.  CUDA_VISIBLE_DEVICES maps the local ordinal to the
+    physical one; a UUID entry is looked up through NVML, and anything unreadable falls back to
+    the local ordinal (the clock record then names that GPU)."""
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").strip()
+    if not vis:
+        return local
+    entries = [e.strip() for e in vis.split(",") if e.strip()]
+    if local >= len(entries):
+        return local
+    try:
+        return int(entries[local])
+    except ValueError:
+        pass
+    try:
+        import pynvml
+        pynvml.nvmlInit()
+        return int(pynvml.nvmlDeviceGetIndex(pynvml.nvmlDeviceGetHandleByUUID(entries[local])))
+    except Exception:
+        return local
+
+
 class ClockSampler:
     """Samples SM clock and throttle reasons through NVML while the timed region runs."""
 
@@ -277,8 +299,7 @@ def gpu_arm(args, rank, world, local):
     n = n_instances(lbytes)
     chain = Chain(torch, nq, d_out, d_in, r, M, n, seed=synth.workload_seed(HEADLINE))
     g = graph_of(torch, lambda: chain.run(nq, stream), stream)
-    sampler = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else
-                           int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local]))
+    sampler = ClockSampler(nvml_index(local))
     ms = timed_replays(torch, g, stream, args.steps, args.warmup, dist, sampler)
     nq.sync_status(stream)
     us_per_layer_job = job_us_per_layer(ms, args.steps, n, world)  # all ranks' layers in the max time

@@ -67,3 +67,13 @@ def test_committed_traffic_lines_parse_and_name_kernel_sources():
                 assert os.path.exists(os.path.join(here, m.group(3))), m.group(3)
                 found += 1
     assert found >= 1
+
+
+def test_nvml_index_follows_visible_devices(monkeypatch):
+    monkeypatch.delenv("CUDA_VISIBLE_DEVICES", raising=False)
+    assert bench.nvml_index(3) == 3
+    monkeypatch.setenv("CUDA_VISIBLE_DEVICES", "4,6")
+    assert bench.nvml_index(0) == 4 and bench.nvml_index(1) == 6
+    assert bench.nvml_index(5) == 5  # beyond the list: the ordinal
+    monkeypatch.setenv("CUDA_VISIBLE_DEVICES", "GPU-00000000-0000-0000-0000-000000000000")
+    assert bench.nvml_index(0) == 0  # a UUID NVML cannot resolve here: the ordinal
