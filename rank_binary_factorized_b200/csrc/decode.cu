@@ -955,7 +955,7 @@ nq_status launch_decode_group_nt(const nq_lrb_layer* const* Ls, int n, const uin
         // the SMs are shared among the members in proportion to their weight words
         const int sms = nq_host::sm_count();
         double wsum = 0.0;
-        int mt[nq::kMaxGroup], nwp[nq::kMaxGroup], grid[nq::kMaxGroup];
+        int mt[nq::kMaxGroup], nwp[nq::kMaxGroup];
         for (int l = 0; l < n; ++l) {
             mt[l] = static_cast<int>((Ls[l]->d_out + 15) / 16);
             nwp[l] = static_cast<int>((Ls[l]->r / 32 + 7) / 8 * 8);
@@ -969,7 +969,6 @@ nq_status launch_decode_group_nt(const nq_lrb_layer* const* Ls, int n, const uin
             const nq_lrb_layer* L = Ls[l];
             int gl = static_cast<int>(sms * (static_cast<double>(mt[l]) * nwp[l]) / wsum + 0.5);
             gl = std::max(1, std::min(gl, mt[l]));
-            grid[l] = gl;
             nq::S2Params& q = g.p[l];
             q.U = L->U;
             q.ldu = L->ldu;
