@@ -2,12 +2,10 @@
 the nq_silu_mul kernel, against the CPU oracle."""
 import numpy as np
 import pytest
-import torch
 
 import oracle
 from rank_binary_factorized_b200 import synth
-from tests.gpu_util import (bf16_bits_to_f64, check_tolerance, download_bf16_bits, need_gpu, nq, upload_bf16,
-                            upload_projection)
+from tests.gpu_util import check_tolerance, download_bf16_bits, need_gpu, nq, upload_bf16, upload_projection
 
 pytestmark = pytest.mark.gpu
 
