@@ -358,15 +358,28 @@ def silu_mul(g, u) -> np.ndarray:
     return h
 
 
-def mlp(gate, up, down, x_bf16, rows=None):
+def mlp(gate, up, down, x_bf16, rows=None, order="dense"):
     """Llama MLP block from three LRB projections, each given as (Uw, Vw, s1, s2, r).
 
-    gate and up are evaluated exactly (fp64) and rounded to bf16 (the activation dtype),
-    h = bf16(silu(g) * u), then the down projection is evaluated exactly on h.  Returns
-    (y, S) of the down projection ([B][n_rows]) and h (bf16 bits, [B][d_ff]).
+    Not on the pages: the block that the 7B and 70B MLP workloads compose from three LRB
+    layers (section 2 factorisation equation for each).  The gate and up projections are
+    evaluated in fp64 and rounded to bf16 (the activation dtype), h = bf16(silu(g) * u), then
+    the down projection is evaluated exactly on h.  ``order`` picks how gate and up are
+    evaluated: "dense" is the definition (materialised W, exact up to the final fp64 sum);
+    "factored" is s1 (.) (U (V^T (s2 (.) x))) in fp64, which is much faster at the 70B shapes
+    and differs from the definition only by fp64 rounding (a bf16 rounding of g or u could
+    differ only for a value within about 1e-15 of a midpoint).  ``rows`` selects output rows
+    of the down projection.  Returns (y, S) of the down projection ([B][n_rows]) and h (bf16
+    bits, [B][d_ff]).
     """
-    g, _ = dense_packed(*gate[:4], gate[4], x_bf16)
-    u, _ = dense_packed(*up[:4], up[4], x_bf16)
+    if order == "dense":
+        g, _ = dense_packed(*gate[:4], gate[4], x_bf16)
+        u, _ = dense_packed(*up[:4], up[4], x_bf16)
+    elif order == "factored":
+        g = factored_packed(*gate[:4], gate[4], x_bf16)
+        u = factored_packed(*up[:4], up[4], x_bf16)
+    else:
+        raise ValueError("order must be 'dense' or 'factored'")
     g16 = bf16_to_double(round_bf16(g))
     u16 = bf16_to_double(round_bf16(u))
     h = silu_mul(g16, u16)

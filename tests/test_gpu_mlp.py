@@ -43,11 +43,8 @@ def test_mlp_block_decode(workload):
     h = nq().silu_mul(g, u)
     y = nq().layer_forward(Ld, h)
     nq().sync_status()
-    # oracle: exact gate/up (factored fp64 order), rounded to bf16, h, then exact down
-    g_ref = oracle.factored_packed(gate.U, gate.V, gate.s1, gate.s2, gate.r, xb)
-    u_ref = oracle.factored_packed(up.U, up.V, up.s1, up.s2, up.r, xb)
-    h_ref = oracle.silu_mul(oracle.bf16_to_double(oracle.round_bf16(g_ref)),
-                            oracle.bf16_to_double(oracle.round_bf16(u_ref)))
+    # oracle: gate/up in the factored fp64 order, rounded to bf16, h, then the exact down
     rows = np.unique(np.concatenate([[0, down.d_out - 1], np.linspace(0, down.d_out - 1, 96).astype(np.int64)]))
-    y_ref, S = oracle.dense_packed(down.U, down.V, down.s1, down.s2, down.r, h_ref, rows=rows)
+    as_tuple = lambda p: (p.U, p.V, p.s1, p.s2, p.r)  # noqa: E731
+    y_ref, S, _ = oracle.mlp(as_tuple(gate), as_tuple(up), as_tuple(down), xb, rows=rows, order="factored")
     check_tolerance(download_bf16_bits(y)[:, rows], y_ref, S, workload + " MLP")
