@@ -27,10 +27,11 @@
 //  - Stage 2 reads the whole accumulator, takes its maximum and re-quantises t to 23 bits
 //    (round to nearest even), so y = s1 (2 P - sum t_q) 2^(d - Q) up to the final bf16 rounding.
 //
-// Workspace.  The accumulator and two counters live in the workspace's leading region, which
-// must be zero before a call and which every call leaves zero: the grid-barrier counter and the
-// "t read" counter only grow (a launch of G CTAs moves each by G), and after every CTA has read
-// t, each CTA clears its share of the accumulator.
+// Workspace.  The grid-barrier counter, the bounds on |t| and the accumulators live in the
+// workspace's leading region, which must be zero before the first call.  The counter only grows
+// (each launch of G CTAs adds G), so counter / G numbers the launches; the accumulators and
+// bounds come in two halves, launch k uses half k & 1 and clears the other one, which launch
+// k - 1 read and launch k + 1 will use.
 #include "tc_common.cuh"
 
 namespace nq {
@@ -43,7 +44,8 @@ constexpr int kMaxM = 2;                 // batch rows: three digit columns each
 constexpr int kMaxMem = NQ_MAX_GROUP;
 constexpr int kMaxSlots = 16;
 constexpr int kMaxTiles1 = 64;           // stage-1 tiles per CTA (runs are at most as many)
-constexpr int kTPer = 24;                // accumulator values per consumer thread in stage 2's prologue
+constexpr int kTPer = 16;                // accumulator values a consumer thread loads at once (stage 2's prologue)
+constexpr int kZoneHalf = NQ_WS_ZONE_BYTES / 16;  // int64 elements per zone half
 
 struct Member {
     CUtensorMap tmV;  // V words [d_in][nw] (row stride ldv), box {16, H1}, 64-byte swizzle
@@ -51,7 +53,7 @@ struct Member {
     const uint16_t* s1;
     const uint16_t* s2;
     uint16_t* y;       // [M][d_out]
-    long long* tacc;   // [M][rp] exact accumulator of t in units of 2^-Q
+    int tacc;          // [M][rp] exact accumulator of t (units of 2^-Q): element offset in a zone half
     int d_out, r, nw, ng;  // ng = 8-word groups of a U row
     int BW, R2;        // stage-2 box: BW words (= 8 or 24 mod 32) by R2 rows
     int rp;            // r rounded up to a chunk (512)
@@ -69,7 +71,8 @@ struct Params {
     int t1_off[kMaxMem + 1];   // first stage-1 tile of each member (tiles: member, chunk, row block)
     int t2_off[kMaxMem + 1];   // first stage-2 block of each member
     long long b2_cum[kMaxMem + 1];  // bytes of the stage-2 blocks before each member
-    int zero_elems;            // int64 accumulator elements of this launch (cleared at the end)
+    long long* zone;           // two halves of kZoneHalf int64: launch k accumulates into half k & 1
+    int off_tq;                // t_q of the members, int32 [M][r], while the digit tables are built
     int n1max, n2max, R2max;   // per-CTA table sizes
     int off_ztab, off_zs, off_s2s, off_s1s, off_dw;  // dynamic shared memory carve-up
 };
@@ -104,14 +107,6 @@ __device__ __forceinline__ void digits3(int v, uint32_t& d0, uint32_t& d1, uint3
     d0 = static_cast<uint32_t>(a0) & 255u;
     d1 = static_cast<uint32_t>(a1) & 255u;
     d2 = static_cast<uint32_t>(a2) & 255u;
-}
-
-// Shift that puts a maximum v into [2^21, 2^22): |z 2^shift| < 2^22.  v == 0 gives `none`.
-__device__ __forceinline__ int shift_for_max(float v, int none) {
-    if (!(v > 0.0f)) return none;
-    int e = 0;
-    frexpf(v, &e);  // v = f 2^e, 0.5 <= f < 1
-    return 22 - e;
 }
 
 // 4x4 byte transpose of four rows given in the order (w0, w1, w2, w3): o[b] holds byte b of the
@@ -200,10 +195,25 @@ __device__ __forceinline__ void combine_cols(int c_lo, int c_hi, int tig, long l
 
 __device__ __forceinline__ double pow2_d(int e) { return __longlong_as_double(static_cast<long long>(1023 + e) << 52); }
 
+// Exponent e of a positive float v = f 2^e with 0.5 <= f < 1, from its bits (frexp for
+// subnormals, which stage 1 meets only for values below 2^-126).
+__device__ __forceinline__ int exp_of(float v) {
+    const int biased = static_cast<int>((__float_as_uint(v) >> 23) & 0xffu);
+    if (biased != 0) return biased - 126;
+    int e = 0;
+    frexpf(v, &e);
+    return e;
+}
+
 // End of a stage-1 run (member mb, chunk c): this warp's exact partials of t for its 64
 // outputs, (2 P - sum z_q) 2^(Q - shift), into the accumulator; the warp's sums restart at 0.
-__device__ __forceinline__ void flush_run(const Member& mb, int c, int cw, int gid, int tig, int M,
-                                          const long long* zsum, const int* sh, const int* Q, int (&acc)[2][2][4]) {
+// The digit columns are combined into P in registers and parked in the warp's buffer pbuf
+// ([64 outputs][2 batch rows]); a short rolled loop then adds them to the accumulator, two
+// outputs per lane.
+__device__ __forceinline__ void flush_run(const Member& mb, long long* half, int c, int cw, int lane, int M,
+                                          long long zsum0, long long zsum1, const int* sh, const int* Q,
+                                          int (&acc)[2][2][4], long long* pbuf) {
+    const int gid = lane >> 2, tig = lane & 3;
 #pragma unroll
     for (int wi = 0; wi < 2; ++wi)
 #pragma unroll
@@ -212,16 +222,22 @@ __device__ __forceinline__ void flush_run(const Member& mb, int c, int cw, int g
             for (int rh = 0; rh < 2; ++rh) {
                 long long P0, P1;
                 combine_cols(acc[wi][h][2 * rh] >> gid, acc[wi][h][2 * rh + 1] >> gid, tig, P0, P1);
-                const int k = 512 * c + 32 * (2 * cw + wi) + 16 * h + 8 * rh + gid;
-                if (tig == 0 && k < mb.r) {
-                    for (int m = 0; m < M; ++m) {
-                        const long long Pm = (m == 0) ? P0 : P1;
-                        const long long v = (2 * Pm - zsum[m]) << (Q[m] - sh[m]);
-                        atomicAdd(reinterpret_cast<unsigned long long*>(mb.tacc + static_cast<int64_t>(m) * mb.rp + k),
-                                  static_cast<unsigned long long>(v));
-                    }
-                }
+                const int kl = 32 * wi + 16 * h + 8 * rh + gid;
+                if (tig == 0) pbuf[2 * kl] = P0;
+                if (tig == 1) pbuf[2 * kl + 1] = P1;
             }
+    __syncwarp();
+#pragma unroll 1
+    for (int e = lane; e < 64 * M; e += 32) {
+        const int m = e >> 6, kl = e & 63;
+        const int k = 512 * c + 64 * cw + kl;
+        if (k < mb.r) {
+            const long long v = (2 * pbuf[2 * kl + m] - (m ? zsum1 : zsum0)) << (Q[m] - sh[m]);
+            atomicAdd(reinterpret_cast<unsigned long long*>(half + mb.tacc + static_cast<int64_t>(m) * mb.rp + k),
+                      static_cast<unsigned long long>(v));
+        }
+    }
+    __syncwarp();
 #pragma unroll
     for (int a = 0; a < 2; ++a)
 #pragma unroll
@@ -230,25 +246,32 @@ __device__ __forceinline__ void flush_run(const Member& mb, int c, int cw, int g
             for (int e = 0; e < 4; ++e) acc[a][b][e] = 0;
 }
 
+// Sum over the lanes of aligned groups of `width` lanes (a power of two <= 32).
+__device__ __forceinline__ long long group_sum(long long v, int width) {
+    for (int off = 1; off < width; off <<= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    return v;
+}
+
 // ------------------------------------------------------------------ the kernel
 __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(const __grid_constant__ Params P) {
     extern __shared__ unsigned char smem_raw[];
     __shared__ __align__(8) uint64_t full_bar[kMaxSlots];
     __shared__ __align__(8) uint64_t empty_bar[kMaxSlots];
-    __shared__ unsigned int s_s2max[kMaxMem];          // max |s2| per member (float bits)
-    __shared__ unsigned int s_xmax[kMaxM];             // max |x| per batch row (float bits)
-    __shared__ int s_Q[kMaxMem][kMaxM];                // common exponent of t's accumulator
-    __shared__ unsigned int s_runmax[kMaxTiles1][kMaxM];  // max |z| per run (float bits)
-    __shared__ int s_runsh[kMaxTiles1][kMaxM];
-    __shared__ long long s_runzsum[kMaxTiles1][kMaxM];
-    __shared__ unsigned long long s_tmax[kMaxMem][kMaxM];
-    __shared__ int s_td[kMaxMem][kMaxM];               // right shift of t's accumulator
-    __shared__ long long s_tsum[kMaxMem][kMaxM];       // sum over k of t_q
-    __shared__ unsigned char s_tl[kMaxTiles1], s_trun[kMaxTiles1];  // member and run of each stage-1 tile
-    __shared__ short s_tc[kMaxTiles1], s_trb[kMaxTiles1];            // chunk and row block
+    __shared__ unsigned int s_s2max[kMaxMem];              // max |s2| per member (float bits)
+    __shared__ unsigned int s_xmax[kMaxM];                 // max |x| per batch row (float bits)
+    __shared__ int s_Q[kMaxMem][kMaxM];                    // common exponent of t's accumulator
+    __shared__ unsigned int s_tilemax[kMaxTiles1][kMaxM];  // max |z| per stage-1 tile (float bits)
+    __shared__ int s_tilesh[kMaxTiles1][kMaxM];            // shift of the tile's run
+    __shared__ long long s_tilezsum[kMaxTiles1][kMaxM];    // sum of z_q over the tile's rows
+    __shared__ long long s_tilezabs[kMaxTiles1][kMaxM];    // sum of |z_q|
+    __shared__ int s_td[kMaxMem][kMaxM];                   // right shift of t's accumulator
+    __shared__ long long s_tsum[kMaxMem][kMaxM];           // sum over k of t_q
+    __shared__ unsigned char s_tl[kMaxTiles1];             // member of each stage-1 tile
+    __shared__ short s_tc[kMaxTiles1], s_trb[kMaxTiles1];  // chunk and row block
+    __shared__ unsigned char s_rfirst[kMaxTiles1], s_rlast[kMaxTiles1];  // first / last tile of its run
     __shared__ volatile int s_abort;
     __shared__ int s_issued;
-    __shared__ unsigned long long s_target2;
+    __shared__ unsigned long long s_launch;  // index of this launch on the workspace
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int gid = lane >> 2, tig = lane & 3;
@@ -260,6 +283,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(const __grid
     const int a2 = stage2_start(P, cta, G);
     const int n2 = stage2_start(P, cta + 1, G) - a2;
     const int KS = P.H1 / 32;  // K steps (32 rows) per stage-1 tile
+    // per zone half: [member][m] sums |z_q| 2^(Q - shift), exact bounds on |t| at scale 2^-Q
+    long long* const bounds_base = reinterpret_cast<long long*>(P.sync + 8);
 
     // 1024-byte aligned base (the swizzled TMA boxes need it)
     const uint32_t raw_base = tc::smem_u32(smem_raw);
@@ -277,44 +302,50 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(const __grid
         tc::mbar_fence_init();
         s_abort = 0;
         s_issued = 0;
-        // stage-1 tiles of this CTA: member, chunk, row block, run (a run = consecutive tiles
-        // of one member and chunk)
-        int run = -1, pl = -1, pc = -1;
-        for (int t = 0; t < n1; ++t) {
-            const int g = a1 + t;
-            const int l = member_of(P.t1_off, P.nmem, g);
+    }
+    // stage-1 tiles of this CTA: member, chunk, row block, and the run (consecutive tiles of
+    // one member and chunk) each belongs to
+    if (tid < n1) {
+        const int t = tid;
+        auto key = [&](int u, int& l, int& c, int& rb) {
+            const int g = a1 + u;
+            l = member_of(P.t1_off, P.nmem, g);
             const int loc = g - P.t1_off[l];
-            const int c = loc / P.nrb;
-            if (l != pl || c != pc) {
-                ++run;
-                pl = l;
-                pc = c;
-            }
-            s_tl[t] = static_cast<unsigned char>(l);
-            s_tc[t] = static_cast<short>(c);
-            s_trb[t] = static_cast<short>(loc - c * P.nrb);
-            s_trun[t] = static_cast<unsigned char>(run);
+            c = loc / P.nrb;
+            rb = loc - c * P.nrb;
+        };
+        int l, c, rb;
+        key(t, l, c, rb);
+        s_tl[t] = static_cast<unsigned char>(l);
+        s_tc[t] = static_cast<short>(c);
+        s_trb[t] = static_cast<short>(rb);
+        int f = t, e = t;
+        while (f > 0) {
+            int l2, c2, rb2;
+            key(f - 1, l2, c2, rb2);
+            if (l2 != l || c2 != c) break;
+            --f;
         }
+        while (e + 1 < n1) {
+            int l2, c2, rb2;
+            key(e + 1, l2, c2, rb2);
+            if (l2 != l || c2 != c) break;
+            ++e;
+        }
+        s_rfirst[t] = static_cast<unsigned char>(f);
+        s_rlast[t] = static_cast<unsigned char>(e);
     }
     if (tid < kMaxMem) s_s2max[tid] = 0u;
     if (tid < kMaxM) s_xmax[tid] = 0u;
     for (int e = tid; e < kMaxTiles1 * kMaxM; e += kThreads) {
-        (&s_runmax[0][0])[e] = 0u;
-        (&s_runzsum[0][0])[e] = 0;
+        (&s_tilemax[0][0])[e] = 0u;
+        (&s_tilezsum[0][0])[e] = 0;
+        (&s_tilezabs[0][0])[e] = 0;
     }
-    if (tid < kMaxMem * kMaxM) {
-        (&s_tmax[0][0])[tid] = 0ull;
-        (&s_tsum[0][0])[tid] = 0;
-    }
+    if (tid < kMaxMem * kMaxM) (&s_tsum[0][0])[tid] = 0;
     __syncthreads();
     pdl_launch_dependents();
 
-    // stage-1 tile t of this CTA: member, chunk, row block (tables filled above)
-    auto tile_of = [&](int t, int& l, int& c, int& rb) {
-        l = s_tl[t];
-        c = s_tc[t];
-        rb = s_trb[t];
-    };
     auto block_of = [&](int b, int& l, int& rho) {
         const int g = a2 + b;
         l = member_of(P.t2_off, P.nmem, g);
@@ -333,10 +364,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(const __grid
                     break;
                 }
                 if (i < n1) {
-                    int l, c, rb;
-                    tile_of(i, l, c, rb);
                     tc::mbar_arrive_expect_tx(full(s), static_cast<uint32_t>(64 * P.H1));
-                    tc::tma_load_2d(slot_addr(s), &P.mem[l].tmV, kTileWords * c, rb * P.H1, full(s));
+                    tc::tma_load_2d(slot_addr(s), &P.mem[s_tl[i]].tmV, kTileWords * s_tc[i], s_trb[i] * P.H1, full(s));
                 } else {
                     int l, rho;
                     block_of(i - n1, l, rho);
@@ -351,38 +380,40 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(const __grid
         // ================================================================ consumers
         const int cw = warp - 1;      // consumer warp 0..7
         const int ctid = tid - 32;    // consumer thread 0..255
+        constexpr int kCT = 32 * kCW;
         uint2* const ztab = reinterpret_cast<uint2*>(gbase + P.off_ztab);   // [n1][KS][32]
         float* const zs = reinterpret_cast<float*>(gbase + P.off_zs);       // [n1][M][H1]
         uint16_t* const s2s = reinterpret_cast<uint16_t*>(gbase + P.off_s2s);  // [n1][H1]
         uint16_t* const s1s = reinterpret_cast<uint16_t*>(gbase + P.off_s1s);  // [n2][R2max]
+        long long* const pbuf = reinterpret_cast<long long*>(gbase + P.off_dw) + cw * 64 * kMaxM;  // this warp's
 
         // ---- weights first (before the wait for the previous kernel): max |s2| of every member,
         // s2 of this CTA's stage-1 rows, s1 of its stage-2 rows, cleared digit tables
+#pragma unroll 1
         for (int l = 0; l < P.nmem; ++l) {
             const uint16_t* s2 = P.mem[l].s2;
-            float mx = 0.0f;
+            uint32_t mx = 0u;  // max of |s2| as fp16 magnitude bits (order-preserving)
             const int nv = P.d_in / 8;
-            for (int v = ctid; v < nv; v += 32 * kCW) {
+#pragma unroll 1
+            for (int v = ctid; v < nv; v += kCT) {
                 const uint4 q = __ldg(reinterpret_cast<const uint4*>(s2) + v);
                 const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    mx = fmaxf(mx, fabsf(f16_bits_to_float(static_cast<uint16_t>(w[h] & 0xFFFFu))));
-                    mx = fmaxf(mx, fabsf(f16_bits_to_float(static_cast<uint16_t>(w[h] >> 16))));
-                }
+                for (int h = 0; h < 4; ++h) mx = max(mx, max(w[h] & 0x7fffu, (w[h] >> 16) & 0x7fffu));
             }
-            for (int j = nv * 8 + ctid; j < P.d_in; j += 32 * kCW) mx = fmaxf(mx, fabsf(f16_bits_to_float(__ldg(s2 + j))));
-            for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-            if (lane == 0) atomicMax(&s_s2max[l], __float_as_uint(mx));
+#pragma unroll 1
+            for (int j = nv * 8 + ctid; j < P.d_in; j += kCT) mx = max(mx, static_cast<uint32_t>(__ldg(s2 + j)) & 0x7fffu);
+            mx = __reduce_max_sync(0xffffffffu, mx);
+            if (lane == 0) atomicMax(&s_s2max[l], __float_as_uint(f16_bits_to_float(static_cast<uint16_t>(mx))));
         }
-        for (int e = ctid; e < n1 * P.H1; e += 32 * kCW) {
+#pragma unroll 1
+        for (int e = ctid; e < n1 * P.H1; e += kCT) {
             const int t = e / P.H1, i = e - t * P.H1;
-            int l, c, rb;
-            tile_of(t, l, c, rb);
-            const int j = rb * P.H1 + i;
-            s2s[e] = (j < P.d_in) ? __ldg(P.mem[l].s2 + j) : static_cast<uint16_t>(0);
+            const int j = s_trb[t] * P.H1 + i;
+            s2s[e] = (j < P.d_in) ? __ldg(P.mem[s_tl[t]].s2 + j) : static_cast<uint16_t>(0);
         }
-        for (int e = ctid; e < n2 * P.R2max; e += 32 * kCW) {
+#pragma unroll 1
+        for (int e = ctid; e < n2 * P.R2max; e += kCT) {
             const int b = e / P.R2max, i = e - b * P.R2max;
             int l, rho;
             block_of(b, l, rho);
@@ -391,116 +422,172 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(const __grid
             s1s[e] = (i < m.R2 && row < m.d_out) ? __ldg(m.s1 + row) : static_cast<uint16_t>(0);
         }
         {
-            // digit tables of z (all columns past 3M stay zero) and of t
             uint4* z4 = reinterpret_cast<uint4*>(ztab);
-            const int nz = n1 * KS * 32 / 2;
-            for (int e = ctid; e < nz; e += 32 * kCW) z4[e] = make_uint4(0u, 0u, 0u, 0u);
+            const int nz = n1 * KS * 16;
+#pragma unroll 1
+            for (int e = ctid; e < nz; e += kCT) z4[e] = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll 1
             for (int l = 0; l < P.nmem; ++l) {
                 uint4* b4 = reinterpret_cast<uint4*>(gbase + P.mem[l].btab);
-                const int nb = 8 * P.mem[l].ng * 32 / 2;
-                for (int e = ctid; e < nb; e += 32 * kCW) b4[e] = make_uint4(0u, 0u, 0u, 0u);
+                const int nb = 8 * P.mem[l].ng * 16;
+#pragma unroll 1
+                for (int e = ctid; e < nb; e += kCT) b4[e] = make_uint4(0u, 0u, 0u, 0u);
             }
         }
 
         pdl_wait();  // x (and the workspace) may be written by the previous kernel
-
-        // ---- max |x| per batch row over the whole input, and z of this CTA's stage-1 rows
+        // Launches on this workspace run in stream order and each adds G to the barrier counter,
+        // which no CTA of this launch can move past a multiple of G before all have read it:
+        // the launch index k = counter / G.  Launch k accumulates into zone half k & 1 and
+        // clears the other half (last read by launch k - 1, complete) for launch k + 1.
+        if (ctid == 0) s_launch = *reinterpret_cast<volatile unsigned long long*>(P.sync) / G;
+        consumers_sync();
+        const int parity = static_cast<int>(s_launch & 1ull);
+        long long* const half = P.zone + parity * kZoneHalf;
+        long long* const bounds = bounds_base + parity * (kMaxMem * kMaxM);
         {
-            float mx[kMaxM] = {0.0f, 0.0f};
+            long long* other = P.zone + (parity ^ 1) * kZoneHalf;
+            const int e0 = static_cast<int>(static_cast<long long>(kZoneHalf / 2) * cta / G);
+            const int e1 = static_cast<int>(static_cast<long long>(kZoneHalf / 2) * (cta + 1) / G);
+#pragma unroll 1
+            for (int e = e0 + ctid; e < e1; e += kCT) reinterpret_cast<uint4*>(other)[e] = make_uint4(0u, 0u, 0u, 0u);
+            if (cta == 0 && ctid < kMaxMem * kMaxM) bounds_base[(parity ^ 1) * (kMaxMem * kMaxM) + ctid] = 0;
+        }
+
+        // ---- max |x| per batch row over the whole input (bf16 magnitude bits order like the
+        // values), and z of this CTA's stage-1 rows with each tile's maximum.  One pass issues
+        // up to 16 loads of each kind per thread before it uses any.
+        {
+            constexpr int U = 8;
+            const int lgH1 = __ffs(P.H1) - 1, lgM = M - 1;  // H1 a power of two, M 1 or 2
+            uint32_t mx0 = 0u, mx1 = 0u;
             const int total = M * P.d_in;
             const int nv = total / 8;
-            for (int v = ctid; v < nv; v += 32 * kCW) {
-                const uint4 q = *reinterpret_cast<const uint4*>(P.x + 8 * v);
-                const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+            const int nz = n1 * M * P.H1;
+            const int rounds = (max(nv, nz) + U * kCT - 1) / (U * kCT);
+#pragma unroll 1
+            for (int rd = 0; rd < rounds; ++rd) {
+                uint4 xv[U];
+                uint16_t xz[U];
 #pragma unroll
-                for (int h = 0; h < 8; ++h) {
-                    const int e = 8 * v + h;
-                    const float a = fabsf(bf16_bits_to_float(static_cast<uint16_t>((w[h >> 1] >> (16 * (h & 1))) & 0xFFFFu)));
-                    if (e < P.d_in) mx[0] = fmaxf(mx[0], a);
-                    else mx[1] = fmaxf(mx[1], a);
+                for (int u = 0; u < U; ++u) {
+                    const int v = (rd * U + u) * kCT + ctid;
+                    xv[u] = (v < nv) ? *reinterpret_cast<const uint4*>(P.x + 8 * v) : make_uint4(0u, 0u, 0u, 0u);
+                    const int tm = v >> lgH1, t = tm >> lgM, m = tm & lgM;
+                    const int j = s_trb[min(t, kMaxTiles1 - 1)] * P.H1 + (v & (P.H1 - 1));
+                    xz[u] = (v < nz && j < P.d_in) ? P.x[static_cast<int64_t>(m) * P.d_in + j] : static_cast<uint16_t>(0);
                 }
-            }
-            for (int e = nv * 8 + ctid; e < total; e += 32 * kCW) {
-                const float a = fabsf(bf16_bits_to_float(P.x[e]));
-                if (e < P.d_in) mx[0] = fmaxf(mx[0], a);
-                else mx[1] = fmaxf(mx[1], a);
-            }
 #pragma unroll
-            for (int m = 0; m < kMaxM; ++m) {
-                float v = mx[m];
-                for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
-                if (lane == 0 && m < M) atomicMax(&s_xmax[m], __float_as_uint(v));
-            }
-            // z of the stage-1 rows, run maxima
-            for (int t = 0; t < n1; ++t) {
-                int l, c, rb;
-                tile_of(t, l, c, rb);
-                const int run = s_trun[t];
-                for (int m = 0; m < M; ++m) {
-                    float v = 0.0f;
-                    for (int i = ctid; i < P.H1; i += 32 * kCW) {
-                        const int j = rb * P.H1 + i;
-                        float z = 0.0f;
-                        if (j < P.d_in)
-                            z = f16_bits_to_float(s2s[t * P.H1 + i]) * bf16_bits_to_float(P.x[static_cast<int64_t>(m) * P.d_in + j]);
-                        zs[(t * M + m) * P.H1 + i] = z;
-                        v = fmaxf(v, fabsf(z));
+                for (int u = 0; u < U; ++u) {
+                    const int v = (rd * U + u) * kCT + ctid;
+                    // magnitudes of the eight bf16 values, two per word
+                    const uint32_t a = __vmaxu2(__vmaxu2(xv[u].x & 0x7fff7fffu, xv[u].y & 0x7fff7fffu),
+                                                __vmaxu2(xv[u].z & 0x7fff7fffu, xv[u].w & 0x7fff7fffu));
+                    const uint32_t vm = max(a & 0xffffu, a >> 16);
+                    if (8 * v + 8 <= P.d_in) {
+                        mx0 = max(mx0, vm);
+                    } else if (8 * v >= P.d_in) {
+                        mx1 = max(mx1, vm);
+                    } else {  // the vector that holds the end of row 0
+                        const uint32_t w[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
+#pragma unroll
+                        for (int h = 0; h < 8; ++h) {
+                            const uint32_t b = (w[h >> 1] >> (16 * (h & 1))) & 0x7fffu;
+                            if (8 * v + h < P.d_in) mx0 = max(mx0, b);
+                            else mx1 = max(mx1, b);
+                        }
                     }
-                    for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
-                    if (lane == 0) atomicMax(&s_runmax[run][m], __float_as_uint(v));
+                    if (v < nz) {
+                        const int t = (v >> lgH1) >> lgM;
+                        zs[v] = f16_bits_to_float(s2s[(t << lgH1) + (v & (P.H1 - 1))]) * bf16_bits_to_float(xz[u]);
+                    }
                 }
+            }
+#pragma unroll 1
+            for (int e = nv * 8 + ctid; e < total; e += kCT) {
+                const uint32_t a = static_cast<uint32_t>(P.x[e]) & 0x7fffu;
+                if (e < P.d_in) mx0 = max(mx0, a);
+                else mx1 = max(mx1, a);
+            }
+            mx0 = __reduce_max_sync(0xffffffffu, mx0);
+            mx1 = __reduce_max_sync(0xffffffffu, mx1);
+            if (lane == 0) {
+                atomicMax(&s_xmax[0], __float_as_uint(bf16_bits_to_float(static_cast<uint16_t>(mx0))));
+                if (M > 1) atomicMax(&s_xmax[1], __float_as_uint(bf16_bits_to_float(static_cast<uint16_t>(mx1))));
             }
         }
         consumers_sync();
-        // common exponent per member and batch row; shift per run
+        // each tile's maximum |z| (a warp per 32 values; H1 is a multiple of 32)
+#pragma unroll 1
+        for (int e0 = cw * 32; e0 < n1 * M * P.H1; e0 += kCT) {
+            const int tm = e0 / P.H1;
+            const int t = tm / M, m = tm - t * M;
+            const uint32_t v = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(zs[e0 + lane])));
+            if (lane == 0) atomicMax(&s_tilemax[t][m], v);
+        }
+        consumers_sync();
+        // common exponent per member and batch row: Q = 16 + (22 - e(max|s2| max|x|))
         if (ctid < P.nmem * M) {
             const int l = ctid / M, m = ctid - l * M;
             const double bound = static_cast<double>(__uint_as_float(s_s2max[l])) * static_cast<double>(__uint_as_float(s_xmax[m]));
-            int e = 0;
-            if (bound > 0.0) frexp(bound, &e);
+            const int e = static_cast<int>((__double_as_longlong(bound) >> 52) & 0x7ff) - 1022;
             s_Q[l][m] = (bound > 0.0) ? (22 - e) + 16 : 0;
         }
         consumers_sync();
-        for (int t = ctid / kMaxM; t < n1; t += 32 * kCW / kMaxM) {
-            const int m = ctid % kMaxM;
-            if (m < M && (t == 0 || s_trun[t] != s_trun[t - 1])) {
-                const int Q = s_Q[s_tl[t]][m];
-                s_runsh[s_trun[t]][m] = min(shift_for_max(__uint_as_float(s_runmax[s_trun[t]][m]), Q), Q);
-            }
+        // each tile's run shift: from the run's maximum, at most Q
+        if (ctid < n1 * M) {
+            const int t = ctid / M, m = ctid - t * M;
+            float v = 0.0f;
+            for (int u = s_rfirst[t]; u <= s_rlast[t]; ++u) v = fmaxf(v, __uint_as_float(s_tilemax[u][m]));
+            const int Q = s_Q[s_tl[t]][m];
+            s_tilesh[t][m] = (v > 0.0f) ? min(22 - exp_of(v), Q) : Q;
         }
         consumers_sync();
         // ---- z's digit table: for tile t, K step kb and lane (gid, tig), .x holds digit
-        // column gid of rows 32 kb + 4 tig + i (byte i), .y of rows 32 kb + 16 + 4 tig + i
+        // column gid of rows 32 kb + 4 tig + i (byte i), .y of rows 32 kb + 16 + 4 tig + i.
+        // A task is (t, kb, tig, half); the 8 KS tasks of a tile are consecutive, so aligned
+        // lane groups reduce each tile's sums of z_q and |z_q|.
         {
-            const int tasks = n1 * KS * 8 * M;  // (tile, K step, tig, half, m)
-            for (int e = ctid; e < tasks; e += 32 * kCW) {
-                const int m = e % M;
-                const int rest = e / M;
-                const int half = rest & 1, tg = (rest >> 1) & 3;
-                const int kt = rest >> 3;  // t * KS + kb
-                const int t = kt / KS, kb = kt - t * KS;
-                const int run = s_trun[t];
-                const double mul = ldexp(1.0, s_runsh[run][m]);
-                uint32_t d0 = 0u, d1 = 0u, d2 = 0u;
-                int qs = 0;
+            const int tasks = n1 * KS * 8;
+            const int gw = min(32, 8 * KS);
+#pragma unroll 1
+            for (int e0 = cw * 32; e0 < tasks; e0 += kCT) {
+                const int e = e0 + lane;
+                const bool on = e < tasks;
+                const int half = e & 1, tg = (e >> 1) & 3, kt = e >> 3;  // kt = t KS + kb
+                const int t = on ? kt / KS : 0, kb = kt - t * KS;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int jl = 32 * kb + 16 * half + 4 * tg + i;
-                    const int qv = __double2int_rn(static_cast<double>(zs[(t * M + m) * P.H1 + jl]) * mul);
-                    qs += qv;
-                    uint32_t a0, a1, a2;
-                    digits3(qv, a0, a1, a2);
-                    d0 |= a0 << (8 * i);
-                    d1 |= a1 << (8 * i);
-                    d2 |= a2 << (8 * i);
+                for (int m = 0; m < kMaxM; ++m) {
+                    long long qs = 0, qa = 0;
+                    if (on && m < M) {
+                        const double mul = pow2_d(s_tilesh[t][m]);
+                        uint32_t d0 = 0u, d1 = 0u, d2 = 0u;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int jl = 32 * kb + 16 * half + 4 * tg + i;
+                            const int qv = __double2int_rn(static_cast<double>(zs[(t * M + m) * P.H1 + jl]) * mul);
+                            qs += qv;
+                            qa += abs(qv);
+                            uint32_t a0, a1, a2;
+                            digits3(qv, a0, a1, a2);
+                            d0 |= a0 << (8 * i);
+                            d1 |= a1 << (8 * i);
+                            d2 |= a2 << (8 * i);
+                        }
+                        uint32_t* zt = reinterpret_cast<uint32_t*>(ztab + kt * 32);
+                        zt[2 * (4 * (3 * m + 0) + tg) + half] = d0;
+                        zt[2 * (4 * (3 * m + 1) + tg) + half] = d1;
+                        zt[2 * (4 * (3 * m + 2) + tg) + half] = d2;
+                    }
+                    if (m < M) {
+                        qs = group_sum(qs, gw);
+                        qa = group_sum(qa, gw);
+                        if (on && (lane & (gw - 1)) == 0) {
+                            atomicAdd(reinterpret_cast<unsigned long long*>(&s_tilezsum[t][m]), static_cast<unsigned long long>(qs));
+                            atomicAdd(reinterpret_cast<unsigned long long*>(&s_tilezabs[t][m]), static_cast<unsigned long long>(qa));
+                        }
+                    }
                 }
-                uint32_t* zt = reinterpret_cast<uint32_t*>(ztab + kt * 32);
-                zt[2 * (4 * (3 * m + 0) + tg) + half] = d0;
-                zt[2 * (4 * (3 * m + 1) + tg) + half] = d1;
-                zt[2 * (4 * (3 * m + 2) + tg) + half] = d2;
-                // this thread's tasks are few; add each one's sum straight into its run
-                atomicAdd(reinterpret_cast<unsigned long long*>(&s_runzsum[run][m]),
-                          static_cast<unsigned long long>(static_cast<long long>(qs)));
             }
         }
         consumers_sync();
@@ -515,23 +602,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(const __grid
 #pragma unroll
                     for (int e = 0; e < 4; ++e) acc[a][b][e] = 0;
             const uint32_t msk = 0x01010101u << gid;
-            int run = -1, pl = -1, pc = -1;
+#pragma unroll 1
             for (int t = 0; t < n1; ++t) {
-                int l, c, rb;
-                tile_of(t, l, c, rb);
-                if (l != pl || c != pc) {
-                    if (run >= 0) flush_run(P.mem[pl], pc, cw, gid, tig, M, s_runzsum[run], s_runsh[run], s_Q[pl], acc);
-                    ++run;
-                    pl = l;
-                    pc = c;
-                }
+                const int l = s_tl[t], c = s_tc[t];
                 const int s = t % ns;
                 if (!tc::mbar_wait(full(s), (t / ns) & 1, P.err)) s_abort = 1;
                 consumers_sync();
                 if (s_abort) break;
                 const uint32_t slot = slot_addr(s);
                 // in-place transpose: thread (q, p), rows read in a rotated order
-                for (int task = ctid; task < P.H1; task += 32 * kCW) {
+#pragma unroll 1
+                for (int task = ctid; task < P.H1; task += kCT) {
                     const int q = task >> 2, p = task & 3;
                     // instruction i reads row 4q + ((i + (q & 1)) & 3); the transpose's last byte
                     // permutation puts the rows back in order
@@ -556,6 +637,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(const __grid
                 const Member& mb = P.mem[l];
                 if (16 * c + 2 * cw < mb.nw) {
                     const uint2* zt = ztab + t * KS * 32;
+#pragma unroll 1
                     for (int kb = 0; kb < KS; ++kb) {
                         const uint2 bz = zt[kb * 32 + lane];
 #pragma unroll
@@ -570,30 +652,46 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(const __grid
                 }
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(empty(s));
+                if (s_rlast[t] == t) {
+                    // end of the run: its sums of z_q and |z_q|, then this warp's partials
+                    long long zs0 = 0, zs1 = 0, za0 = 0, za1 = 0;
+                    for (int u = s_rfirst[t]; u <= t; ++u) {
+                        zs0 += s_tilezsum[u][0];
+                        zs1 += s_tilezsum[u][1];
+                        za0 += s_tilezabs[u][0];
+                        za1 += s_tilezabs[u][1];
+                    }
+                    if (cw == 0 && lane < M) {
+                        const long long b = (lane == 0 ? za0 : za1) << (s_Q[l][lane] - s_tilesh[t][lane]);
+                        atomicAdd(reinterpret_cast<unsigned long long*>(bounds + l * kMaxM + lane), static_cast<unsigned long long>(b));
+                    }
+                    flush_run(mb, half, c, cw, lane, M, zs0, zs1, s_tilesh[t], s_Q[l], acc, pbuf);
+                }
             }
-            if (run >= 0 && !s_abort) flush_run(P.mem[pl], pc, cw, gid, tig, M, s_runzsum[run], s_runsh[run], s_Q[pl], acc);
         }
 
-        // ---- grid barrier: every CTA's partials are in the accumulator
+        // ---- grid barrier: every CTA's partials are in the accumulator.  The arrival is a
+        // release reduction (it orders this CTA's partials, seen through the CTA barrier, before
+        // it); launch k is complete when the counter reaches (k + 1) G.
         consumers_sync();
         if (ctid == 0) {
-            __threadfence();
-            const unsigned long long old = atomicAdd(P.sync, 1ull);
-            const unsigned long long target = (old / G + 1) * G;
+            asm volatile("red.release.gpu.global.add.u64 [%0], 1;" ::"l"(P.sync) : "memory");
+            const unsigned long long target = (s_launch + 1) * static_cast<unsigned long long>(G);
             const uint64_t t0 = tc::globaltimer_ns();
             while (ld_acquire_u64(P.sync) < target) {
-                __nanosleep(64);
                 if (tc::globaltimer_ns() - t0 > tc::kWaitLimitNs) {
                     flag_error(P.err, kErrTimeout);
                     s_abort = 1;
                     break;
                 }
             }
-            __threadfence();
         }
         consumers_sync();
 
-        // ---- stage 2 prologue: t of the members this CTA's blocks belong to, re-quantised
+        // ---- stage 2 prologue: t of the members this CTA's blocks belong to, as 23-bit digits.
+        // The shift comes from the exact bound sum |z_q| 2^(Q - shift) >= |t|, so one pass
+        // suffices: a task is (word w, bit offset s, batch row m); it reads the four t of k =
+        // 32 w + s + 8 i and writes whole words of the digit table.
         int l_lo = P.nmem, l_hi = -1;
         if (n2 > 0) {
             int rho;
@@ -601,174 +699,160 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(const __grid
             block_of(n2 - 1, l_hi, rho);
         }
         if (!s_abort) {
+            int32_t* const tq = reinterpret_cast<int32_t*>(gbase + P.off_tq);  // [M][r] of the member in hand
+#pragma unroll 1
             for (int l = l_lo; l <= l_hi; ++l) {
                 const Member& mb = P.mem[l];
+                const long long* tl = half + mb.tacc;
+                // the bound and up to kTPer accumulator values per thread in one round of loads
                 const int E = M * mb.r;
-                long long tv[kTPer];
-                unsigned long long mx[kMaxM] = {0ull, 0ull};
+                const long long b0 = bounds[l * kMaxM];
+                const long long b1 = (M > 1) ? bounds[l * kMaxM + 1] : 0ll;
+                const int d0 = max(0, (64 - __clzll(b0)) - 22), d1 = max(0, (64 - __clzll(b1)) - 22);
+                long long ts0 = 0, ts1 = 0;
+#pragma unroll 1
+                for (int e0 = 0; e0 < E; e0 += kTPer * kCT) {
+                    long long v[kTPer];
 #pragma unroll
-                for (int u = 0; u < kTPer; ++u) {
-                    const int e = ctid + u * 32 * kCW;
-                    tv[u] = 0;
-                    if (e < E) {
-                        const int m = e / mb.r, k = e - m * mb.r;
-                        tv[u] = mb.tacc[static_cast<int64_t>(m) * mb.rp + k];
-                        const unsigned long long a = static_cast<unsigned long long>(tv[u] < 0 ? -tv[u] : tv[u]);
-                        if (m == 0) mx[0] = max(mx[0], a);
-                        else mx[1] = max(mx[1], a);
+                    for (int u = 0; u < kTPer; ++u) {
+                        const int e = e0 + u * kCT + ctid;
+                        const int m = (e >= mb.r) ? 1 : 0, k = e - m * mb.r;
+                        v[u] = (e < E) ? tl[static_cast<int64_t>(m) * mb.rp + k] : 0ll;
                     }
-                }
 #pragma unroll
-                for (int m = 0; m < kMaxM; ++m) {
-                    unsigned long long v = mx[m];
-                    for (int off = 16; off > 0; off >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, off));
-                    if (lane == 0 && m < M) atomicMax(&s_tmax[l][m], v);
-                }
-                consumers_sync();
-                if (ctid < M) {
-                    const unsigned long long v = s_tmax[l][ctid];
-                    const int bits = 64 - __clzll(static_cast<long long>(v));
-                    s_td[l][ctid] = max(0, bits - 22);
-                }
-                consumers_sync();
-                long long sum[kMaxM] = {0, 0};
-                unsigned char* bt = gbase + mb.btab;
-#pragma unroll
-                for (int u = 0; u < kTPer; ++u) {
-                    const int e = ctid + u * 32 * kCW;
-                    if (e < E) {
-                        const int m = e / mb.r, k = e - m * mb.r;
-                        const int d = s_td[l][m];
-                        long long q = tv[u];
-                        if (d > 0) {
-                            // round to nearest, ties to even
-                            const long long fl = q >> d;
-                            const long long rem = q - (fl << d);
-                            const long long half = 1ll << (d - 1);
-                            q = fl + ((rem > half || (rem == half && (fl & 1))) ? 1 : 0);
+                    for (int u = 0; u < kTPer; ++u) {
+                        const int e = e0 + u * kCT + ctid;
+                        if (e < E) {
+                            const int m = (e >= mb.r) ? 1 : 0;
+                            const int d = m ? d1 : d0;
+                            long long q = v[u];
+                            if (d > 0) {  // round to nearest, ties to even
+                                const long long fl = q >> d;
+                                const long long rem = q - (fl << d);
+                                const long long hf = 1ll << (d - 1);
+                                q = fl + ((rem > hf || (rem == hf && (fl & 1))) ? 1 : 0);
+                            }
+                            if (m) ts1 += q;
+                            else ts0 += q;
+                            tq[e] = static_cast<int32_t>(q);
                         }
-                        if (m == 0) sum[0] += q;
-                        else sum[1] += q;
-                        uint32_t d0, d1, d2;
-                        digits3(static_cast<int>(q), d0, d1, d2);
-                        // k -> bit offset s, byte i, word w = 8 g + 2 tig + half
-                        const int s_ = k & 7, i = (k >> 3) & 3, w = k >> 5;
-                        const int g = w >> 3, tg = (w & 7) >> 1, hf = w & 1;
-                        const int ent = (s_ * mb.ng + g) * 32;
-                        bt[(ent + 4 * (3 * m + 0) + tg) * 8 + hf * 4 + i] = static_cast<unsigned char>(d0);
-                        bt[(ent + 4 * (3 * m + 1) + tg) * 8 + hf * 4 + i] = static_cast<unsigned char>(d1);
-                        bt[(ent + 4 * (3 * m + 2) + tg) * 8 + hf * 4 + i] = static_cast<unsigned char>(d2);
                     }
                 }
-#pragma unroll
-                for (int m = 0; m < kMaxM; ++m) {
-                    long long v = sum[m];
-                    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-                    if (lane == 0 && m < M && v != 0)
-                        atomicAdd(reinterpret_cast<unsigned long long*>(&s_tsum[l][m]), static_cast<unsigned long long>(v));
+                if (ctid < M) s_td[l][ctid] = ctid ? d1 : d0;
+                ts0 = group_sum(ts0, 32);
+                ts1 = group_sum(ts1, 32);
+                if (lane == 0) {
+                    atomicAdd(reinterpret_cast<unsigned long long*>(&s_tsum[l][0]), static_cast<unsigned long long>(ts0));
+                    if (M > 1) atomicAdd(reinterpret_cast<unsigned long long*>(&s_tsum[l][1]), static_cast<unsigned long long>(ts1));
                 }
+                consumers_sync();
+                // digit table: a task is (word w, bit offset s, batch row m) and writes whole
+                // words: byte i of column 3m + q holds digit q of t_q(32 w + s + 8 i)
+                uint32_t* bt = reinterpret_cast<uint32_t*>(gbase + mb.btab);
+                const int tasks = mb.nw * 8 * M;
+#pragma unroll 1
+                for (int e = ctid; e < tasks; e += kCT) {
+                    const int m = (e >= mb.nw * 8) ? 1 : 0, ws_ = e - m * mb.nw * 8;
+                    const int s_ = ws_ & 7, w = ws_ >> 3;
+                    uint32_t W0 = 0u, W1 = 0u, W2 = 0u;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int k = 32 * w + s_ + 8 * i;
+                        const int q = (k < mb.r) ? tq[m * mb.r + k] : 0;
+                        uint32_t a0, a1, a2;
+                        digits3(q, a0, a1, a2);
+                        W0 |= a0 << (8 * i);
+                        W1 |= a1 << (8 * i);
+                        W2 |= a2 << (8 * i);
+                    }
+                    const int g = w >> 3, tg = (w & 7) >> 1, hf = w & 1;
+                    uint32_t* dst = bt + 2 * ((s_ * mb.ng + g) * 32 + 12 * m + tg) + hf;
+                    dst[0] = W0;
+                    dst[8] = W1;   // column 3m + 1: four lanes on
+                    dst[16] = W2;  // column 3m + 2
+                }
+                consumers_sync();
             }
         }
         consumers_sync();
-        if (ctid == 0) {
-            __threadfence();
-            const unsigned long long old = atomicAdd(P.sync + 1, 1ull);
-            s_target2 = (old / G + 1) * G;
-        }
 
-        // ---- stage 2: each warp takes whole blocks of U rows
+        // ---- stage 2: all consumer warps work on each block.  For a pair of 16-row M-tiles,
+        // the 8 ng (word group, bit offset) units are split evenly over the warps; each warp's
+        // exact partial sums of P meet in shared memory.
         if (!s_abort) {
-            for (int b = cw; b < n2; b += kCW) {
+#pragma unroll 1
+            for (int b = 0; b < n2; ++b) {
                 const int i = n1 + b, s = i % ns;
-                // every lane observes the phase, which makes the TMA writes visible to it
-                const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(full(s), (i / ns) & 1, P.err));
-                if (!ok) {
-                    s_abort = 1;
-                    break;
-                }
+                if (!tc::mbar_wait(full(s), (i / ns) & 1, P.err)) s_abort = 1;
+                consumers_sync();
+                if (s_abort) break;
                 int l, rho;
                 block_of(b, l, rho);
                 const Member& mb = P.mem[l];
                 const uint32_t slot = slot_addr(s);
                 const uint32_t bt = base + static_cast<uint32_t>(mb.btab);
                 const int ng = mb.ng, BW = mb.BW;
+                const int u0 = (cw * 8 * ng) / kCW, u1 = ((cw + 1) * 8 * ng) / kCW;  // units g * 8 + s
+#pragma unroll 1
                 for (int pr = 0; pr < mb.R2 / 32; ++pr) {
                     const int row0 = rho * mb.R2 + 32 * pr;
                     if (row0 >= mb.d_out) break;
-                    int acc[8][2][4];
-#pragma unroll
-                    for (int s_ = 0; s_ < 8; ++s_)
-#pragma unroll
-                        for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) acc[s_][mt][e] = 0;
+                    int acc[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
                     // rows gid and gid + 8 of M-tiles 0 and 1 of the pair
                     const uint32_t r00 = slot + static_cast<uint32_t>(((32 * pr + gid) * BW + 2 * tig) * 4);
                     const uint32_t r01 = r00 + static_cast<uint32_t>(8 * BW * 4);
                     const uint32_t r10 = r00 + static_cast<uint32_t>(16 * BW * 4);
                     const uint32_t r11 = r00 + static_cast<uint32_t>(24 * BW * 4);
-                    for (int g = 0; g < ng; ++g) {
-                        const uint32_t go = static_cast<uint32_t>(32 * g);
-                        const uint2 u00 = lds64(r00 + go), u01 = lds64(r01 + go);
-                        const uint2 u10 = lds64(r10 + go), u11 = lds64(r11 + go);
-#pragma unroll
-                        for (int s_ = 0; s_ < 8; ++s_) {
-                            const uint32_t m8 = 0x01010101u << s_;
-                            const uint2 bb = lds64(bt + static_cast<uint32_t>(((s_ * ng + g) * 32 + lane) * 8));
-                            mma_u8s8(acc[s_][0], u00.x & m8, u01.x & m8, u00.y & m8, u01.y & m8, bb.x, bb.y);
-                            mma_u8s8(acc[s_][1], u10.x & m8, u11.x & m8, u10.y & m8, u11.y & m8, bb.x, bb.y);
+                    int gcur = -1;
+                    uint2 u00 = make_uint2(0u, 0u), u01 = u00, u10 = u00, u11 = u00;
+#pragma unroll 1
+                    for (int u = u0; u < u1; ++u) {
+                        const int g = u >> 3, s_ = u & 7;
+                        if (g != gcur) {
+                            const uint32_t go = static_cast<uint32_t>(32 * g);
+                            u00 = lds64(r00 + go);
+                            u01 = lds64(r01 + go);
+                            u10 = lds64(r10 + go);
+                            u11 = lds64(r11 + go);
+                            gcur = g;
                         }
+                        // the A bytes of offset s hold bit s: shifted down, every offset shares one
+                        // accumulator
+                        const uint32_t m1 = 0x01010101u;
+                        const uint2 bb = lds64(bt + static_cast<uint32_t>(((s_ * ng + g) * 32 + lane) * 8));
+                        mma_u8s8(acc[0], (u00.x >> s_) & m1, (u01.x >> s_) & m1, (u00.y >> s_) & m1, (u01.y >> s_) & m1, bb.x, bb.y);
+                        mma_u8s8(acc[1], (u10.x >> s_) & m1, (u11.x >> s_) & m1, (u10.y >> s_) & m1, (u11.y >> s_) & m1, bb.x, bb.y);
                     }
-                    // epilogue: y = s1 (2 P - sum t_q) 2^(d - Q), rounded once to bf16
+                    // this warp's partial P of each row, into its slice of the buffer
 #pragma unroll
                     for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
                         for (int rh = 0; rh < 2; ++rh) {
-                            int c_lo = 0, c_hi = 0;
-#pragma unroll
-                            for (int s_ = 0; s_ < 8; ++s_) {
-                                c_lo += acc[s_][mt][2 * rh] >> s_;
-                                c_hi += acc[s_][mt][2 * rh + 1] >> s_;
-                            }
                             long long P0, P1;
-                            combine_cols(c_lo, c_hi, tig, P0, P1);
-                            const int rl = 32 * pr + 16 * mt + 8 * rh + gid;
-                            const int row = rho * mb.R2 + rl;
-                            if (tig == 0 && row < mb.d_out) {
-                                const double s1v = static_cast<double>(f16_bits_to_float(s1s[b * P.R2max + rl]));
-                                for (int m = 0; m < M; ++m) {
-                                    const long long Pm = (m == 0) ? P0 : P1;
-                                    const long long val = 2 * Pm - s_tsum[l][m];
-                                    const double yv = s1v * static_cast<double>(val) * pow2_d(s_td[l][m] - s_Q[l][m]);
-                                    mb.y[static_cast<int64_t>(m) * mb.d_out + row] = __bfloat16_as_ushort(__double2bfloat16(yv));
-                                }
-                            }
+                            combine_cols(acc[mt][2 * rh], acc[mt][2 * rh + 1], tig, P0, P1);
+                            const int rl = 16 * mt + 8 * rh + gid;
+                            if (tig == 0) pbuf[2 * rl] = P0;
+                            if (tig == 1) pbuf[2 * rl + 1] = P1;
                         }
+                    consumers_sync();
+                    if (ctid < 32 * M) {
+                        // y = s1 (2 P - sum t_q) 2^(d - Q), rounded once to bf16
+                        const int rl = ctid & 31, m = ctid >> 5, row = row0 + rl;
+                        long long Pm = 0;
+                        const long long* pall = reinterpret_cast<const long long*>(gbase + P.off_dw);
+#pragma unroll
+                        for (int w = 0; w < kCW; ++w) Pm += pall[w * 64 * kMaxM + 2 * rl + m];
+                        if (row < mb.d_out) {
+                            const double s1v = static_cast<double>(f16_bits_to_float(s1s[b * P.R2max + 32 * pr + rl]));
+                            const long long val = 2 * Pm - s_tsum[l][m];
+                            const double yv = s1v * static_cast<double>(val) * pow2_d(s_td[l][m] - s_Q[l][m]);
+                            mb.y[static_cast<int64_t>(m) * mb.d_out + row] = __bfloat16_as_ushort(__double2bfloat16(yv));
+                        }
+                    }
+                    consumers_sync();
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive_cnt(empty(s), kCW);
+                if (ctid == 0) mbar_arrive_cnt(empty(s), kCW);
             }
-        }
-
-        // ---- every CTA has read t: clear this CTA's share of the accumulator
-        consumers_sync();
-        if (ctid == 0) {
-            const uint64_t t0 = tc::globaltimer_ns();
-            while (ld_acquire_u64(P.sync + 1) < s_target2) {
-                __nanosleep(64);
-                if (tc::globaltimer_ns() - t0 > tc::kWaitLimitNs) {
-                    flag_error(P.err, kErrTimeout);
-                    s_abort = 1;
-                    break;
-                }
-            }
-        }
-        consumers_sync();
-        if (!s_abort) {
-            long long* zone = P.mem[0].tacc;
-            const int e0 = static_cast<int>(static_cast<long long>(P.zero_elems) * cta / G);
-            const int e1 = static_cast<int>(static_cast<long long>(P.zero_elems) * (cta + 1) / G);
-            for (int e = e0 + ctid; e < e1; e += 32 * kCW) zone[e] = 0;
         }
     }
 
@@ -845,7 +929,6 @@ bool plan_stream(const nq_lrb_layer* const* Ls, int n, const uint16_t* x, uint16
         if (L->d_out > (1 << 30)) return false;
         const int nw = static_cast<int>(L->r / 32);
         if (nw > 248) return false;  // one U row must fit a TMA box (<= 256 words)
-        if (M * L->r > nq::ds::kTPer * 32 * nq::ds::kCW) return false;
         nch += (nw + nq::ds::kTileWords - 1) / nq::ds::kTileWords;
     }
     p.H1 = 64;
@@ -882,7 +965,7 @@ bool plan_stream(const nq_lrb_layer* const* Ls, int n, const uint16_t* x, uint16
         m.s1 = L->s1;
         m.s2 = L->s2;
         m.y = ys[l];
-        m.tacc = reinterpret_cast<long long*>(static_cast<char*>(ws) + kZoneOffset) + zone;
+        m.tacc = static_cast<int>(zone);
         zone += static_cast<size_t>(M) * m.rp;
         m.b2_bytes = static_cast<long long>(m.BW) * m.R2 * 4;
         if (!encode_u32_map(&m.tmV, L->V, L->d_in, m.nw, L->ldv, nq::ds::kTileWords, p.H1, true)) return false;
@@ -899,8 +982,8 @@ bool plan_stream(const nq_lrb_layer* const* Ls, int n, const uint16_t* x, uint16
     p.t1_off[n] = t1;
     p.t2_off[n] = t2;
     p.b2_cum[n] = b2;
-    if (zone * 8 > NQ_WS_ZONE_BYTES) return false;
-    p.zero_elems = static_cast<int>(zone);
+    if (zone > static_cast<size_t>(nq::ds::kZoneHalf)) return false;
+    p.zone = reinterpret_cast<long long*>(static_cast<char*>(ws) + kZoneOffset);
     p.sync = reinterpret_cast<unsigned long long*>(ws);
     p.err = nq_host::error_word();
     if (!p.err) return false;
@@ -942,7 +1025,10 @@ bool plan_stream(const nq_lrb_layer* const* Ls, int n, const uint16_t* x, uint16
         p.off_s2s = carve(static_cast<size_t>(p.n1max) * p.H1 * 2, 16);
         p.off_s1s = carve(static_cast<size_t>(p.n2max) * p.R2max * 2, 16);
         for (int l = 0; l < n; ++l) p.mem[l].btab = carve(static_cast<size_t>(8) * p.mem[l].ng * 32 * 8, 16);
-        p.off_dw = 0;
+        p.off_dw = carve(static_cast<size_t>(nq::ds::kCW) * 64 * nq::ds::kMaxM * 8, 16);
+        size_t tqb = 0;
+        for (int l = 0; l < n; ++l) tqb = std::max(tqb, static_cast<size_t>(M) * p.mem[l].r * 4);
+        p.off_tq = carve(tqb, 16);
         fixed = off;
     }
     const size_t slack = 1024;  // the kernel aligns the dynamic base to 1024 bytes
@@ -955,6 +1041,8 @@ bool plan_stream(const nq_lrb_layer* const* Ls, int n, const uint16_t* x, uint16
     p.off_zs += rebase;
     p.off_s2s += rebase;
     p.off_s1s += rebase;
+    p.off_dw += rebase;
+    p.off_tq += rebase;
     for (int l = 0; l < n; ++l) p.mem[l].btab += rebase;
     sp.smem = static_cast<size_t>(rebase) + fixed + slack;
     sp.grid = G;

@@ -9,8 +9,9 @@ blog), section 2, factorisation equation; section 4, "Inference Performance" (bi
   shapes, on this path and on the two-kernel path (M = 3).
 - Shapes whose stage-1 stretches cross column chunks inside one CTA, partial chunks and row
   blocks, and rows of very different magnitudes in one call.
-- The reserved workspace region: after any sequence of calls its accumulators are zero again
-  and its two counters sit at a multiple of the grid size (which also shows this path ran).
+- The reserved workspace region: after any sequence of calls the barrier counter has moved by
+  the grid size per single-launch call (which also shows this path ran), and the accumulator
+  half and bounds the next call will use are zero.
 """
 import numpy as np
 import pytest
@@ -31,10 +32,14 @@ def _sm_count():
 
 
 def _reserved_state(ws):
+    """Barrier counter, the bounds of both halves and the accumulator halves of the reserved
+    region: counters at bytes 0..7, bounds [2][4][2] int64 from byte 64, halves of 256 KiB each
+    from byte 4096."""
     head = ws[:RESERVED].cpu().numpy()
-    counters = head[:16].view(np.uint64)
-    zone = head[4096:].view(np.int64)
-    return int(counters[0]), int(counters[1]), zone
+    counter = int(head[:8].view(np.uint64)[0])
+    bounds = head[64:64 + 2 * 4 * 2 * 8].view(np.int64).reshape(2, 8)
+    halves = head[4096:].view(np.int64).reshape(2, -1)
+    return counter, bounds, halves
 
 
 def _outlier_input(d_in, M, seed, factors):
@@ -96,9 +101,10 @@ def test_rows_of_very_different_magnitude_and_zero_input():
     assert np.all(bf16_bits_to_f64(z) == 0.0)
 
 
-def test_reserved_region_is_restored_after_calls():
-    """After single, grouped and two-kernel calls on one workspace, the accumulators are zero
-    and each counter advanced by the grid size once per single-launch call."""
+def test_reserved_region_is_ready_after_calls():
+    """After single, grouped and two-kernel calls on one workspace, the barrier counter has
+    advanced by the grid size once per single-launch call, and the accumulator half and bounds
+    that the next call will use are zero."""
     need_gpu()
     G = _sm_count()
     projs = synth.make_workload("layer70b")
@@ -107,15 +113,17 @@ def test_reserved_region_is_restored_after_calls():
     ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
     x = upload_bf16(synth.make_input("layer70b", 8192, 2, key=2400))
     calls = 0
-    nq().layer_forward_group(layers[:3], x, ws=ws)      # q, k, v: one launch
-    calls += 1
-    nq().layer_forward(layers[3], x, ws=ws)             # o
-    calls += 1
-    nq().layer_forward(layers[3], x[:1], ws=ws)         # o at M = 1
-    calls += 1
-    x3 = upload_bf16(synth.make_input("layer70b", 8192, 3, key=2401))
-    nq().layer_forward(layers[3], x3, ws=ws)            # M = 3: the two-kernel path
-    nq().sync_status()
-    c0, c1, zone = _reserved_state(ws)
-    assert c0 == calls * G and c1 == calls * G
-    assert not zone.any()
+    for rep in range(2):
+        nq().layer_forward_group(layers[:3], x, ws=ws)      # q, k, v: one launch
+        calls += 1
+        nq().layer_forward(layers[3], x, ws=ws)             # o
+        calls += 1
+        nq().layer_forward(layers[3], x[:1], ws=ws)         # o at M = 1
+        calls += 1
+        x3 = upload_bf16(synth.make_input("layer70b", 8192, 3, key=2401))
+        nq().layer_forward(layers[3], x3, ws=ws)            # M = 3: the two-kernel path
+        nq().sync_status()
+        counter, bounds, halves = _reserved_state(ws)
+        assert counter == calls * G
+        nxt = calls & 1
+        assert not halves[nxt].any() and not bounds[nxt].any()
