@@ -104,16 +104,11 @@ NQ_API nq_status nq_pack_signs(const float* latent, int64_t rows, int64_t r, int
  * nq_workspace_bytes -- device scratch a call with M activation rows needs (for
  * nq_lrb_matvec, nq_lrb_matmul, nq_layer_forward, nq_lrb_transposed and
  * nq_lrb_scale_grads alike).  Returns 0 for an invalid layer or M.  The workspace must stay
- * untouched by other work while the call runs.
- * Its first NQ_WS_RESERVED_BYTES bytes belong to the single-launch decode path (two grid-barrier
- * counters and the exact int64 accumulators of t): zero-fill the workspace once before its
- * first use (cudaMemset to 0); every call leaves that region ready for the next one (the
- * accumulators back at zero, the counters at a multiple of the grid size).  After a call whose
- * bounded waits gave up (nq_sync_status returned NQ_ERR_TIMEOUT), zero it again.  The rest is
- * per-call scratch, fully written before it is read.  So one workspace serves consecutive calls
- * of any shape on the same stream.
+ * untouched by other work while the call runs.  Its first 4096 bytes are a reserved header
+ * that the kernels neither read nor write; the rest is per-call scratch, fully written
+ * before it is read.  So one workspace can be reused by consecutive calls of any shape on
+ * the same stream, with no initialisation.
  */
-#define NQ_WS_RESERVED_BYTES (4096 + 512 * 1024)
 NQ_API size_t nq_workspace_bytes(const nq_lrb_layer* L, int64_t M);
 
 /*
@@ -121,18 +116,11 @@ NQ_API size_t nq_workspace_bytes(const nq_lrb_layer* L, int64_t M);
  * Section 2 factorisation equation, evaluated as two streaming stages over the packed
  * words: t[m][k] = sum_j V_jk s2_j x[m][j], then y[m][i] = bf16(s1_i sum_k U_ik t[m][k]).
  *   x [M][d_in] bf16, y [M][d_out] bf16 (round to nearest even), ws = workspace of at
- *   least nq_workspace_bytes(L, M) bytes (16-byte aligned, reserved region zero-filled before
- *   first use, see nq_workspace_bytes).
- * Both stages sum exact integers of 23-bit fixed-point activations on the integer tensor path.
- *  - M <= 2, ldu and ldv multiples of 4 words, r <= 7936: one launch.  s2 x is quantised per
- *    stretch of rows that one CTA reduces for one 512-wide column block of V (shift from that
- *    stretch's maximum, at most 16 bits finer than the shift of max|s2| max|x|); the partial
- *    sums of t are added exactly as int64 at one common scale; t is re-quantised to 23 bits
- *    from its maximum (round to nearest even).
- *  - Otherwise: two launches.  s2 x is quantised per row slice of V, t per batch row (shift from
- *    an exact bound on |t|), and the partial sums are combined in fp64 in a fixed order.
- * Results are run-to-run deterministic.  Finite results need |s2_j x[m][j]| within the fp32
- * range.
+ *   least nq_workspace_bytes(L, M) bytes (16-byte aligned).
+ * Both stages sum exact integers: s2 x is quantised to 23-bit fixed point per row slice of V,
+ * t to 23-bit fixed point per batch row (the shift from an exact bound on |t|), and the
+ * partial sums are combined in fp64 in a fixed order.  Results are run-to-run deterministic.
+ * Finite results need |s2_j x[m][j]| within the fp32 range.
  */
 NQ_API nq_status nq_lrb_matvec(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y, int64_t M, void* ws,
                         size_t ws_bytes, void* stream);
@@ -229,10 +217,9 @@ NQ_API nq_status nq_lrb_sign_grads(const nq_lrb_layer* L, const uint16_t* x, con
  * nq_layer_forward_group -- y[l] = layer l applied to x, for 1 <= n <= NQ_MAX_GROUP projections
  * that share their input (a transformer's q, k, v, or its gate and up): every layer must have
  * the same d_in; d_out and r may differ.  For M <= NQ_MATVEC_MAX_M the group runs as one
- * launch (or, outside the single-launch path's reach, one launch of each decode stage) with the
- * layers' blocks side by side, which saves the fixed latency of a call per extra member;
- * numerics as nq_lrb_matvec, except that the stretches of rows over which x is quantised follow
- * the group's total size.  Larger M runs nq_lrb_matmul once
+ * launch of each decode stage (the layers' blocks side by side), which saves a kernel pair's
+ * fixed latency per extra member; numerics as nq_lrb_matvec, except that the row slices of V
+ * over which x is quantised follow the group's total size.  Larger M runs nq_lrb_matmul once
  * per layer.  y: array of n output pointers ([M][d_out_l] bf16 each); ws:
  * nq_group_workspace_bytes(layers, n, M) bytes (0 for an invalid group).
  */

@@ -1081,11 +1081,6 @@ size_t nq_decode_stage2_smem(int64_t r, int64_t M) {
 nq_status nq_launch_decode_group(const nq_lrb_layer* const* Ls, int n, const uint16_t* x, uint16_t* const* ys,
                                  int64_t M, void* ws, cudaStream_t stream, bool pdl, const uint16_t* cot,
                                  float* grad) {
-    if (!grad) {
-        // one launch for both stages when the layers allow it (decode_stream.cu)
-        const nq_status st = nq_launch_decode_stream(Ls, n, x, ys, M, ws, stream, pdl);
-        if (st != NQ_ERR_SHAPE) return st;
-    }
     const int m = static_cast<int>(M);
     if (n == 1) {
         switch (ntiles_for(M)) {

@@ -12,14 +12,9 @@
 #error "libnq is written for sm_100a (B200) only"
 #endif
 
-// Every workspace starts with a region that the single-launch decode kernel keeps in a fixed
-// state: the caller zero-fills it once, and every call leaves it zero again.  Its first
-// NQ_WS_SYNC_BYTES hold the kernel's grid-barrier counters, the next NQ_WS_ZONE_BYTES its exact
-// int64 accumulators of t.  The other kernels' per-call scratch starts after it.
-#define NQ_WS_SYNC_BYTES 4096
-#define NQ_WS_ZONE_BYTES (512 * 1024)
-#define NQ_WS_HEADER_BYTES (NQ_WS_SYNC_BYTES + NQ_WS_ZONE_BYTES)
-static_assert(NQ_WS_HEADER_BYTES == NQ_WS_RESERVED_BYTES, "nq.h states the reserved region's size");
+// Every workspace starts with this many reserved bytes, which the kernels neither read nor
+// write; the per-call scratch follows.
+#define NQ_WS_HEADER_BYTES 4096
 #define NQ_MAX_RANK NQ_MAX_RANK_LIMIT
 
 namespace nq {
@@ -79,10 +74,6 @@ nq_status nq_launch_decode_group(const nq_lrb_layer* const* Ls, int n, const uin
                                  int64_t M, void* ws, cudaStream_t stream, bool pdl, const uint16_t* cot = nullptr,
                                  float* grad = nullptr);
 size_t nq_decode_group_workspace_bytes(const nq_lrb_layer* const* Ls, int n, int64_t M);
-// The single-launch decode path (decode_stream.cu) for M <= 2 and layers whose packed rows TMA can
-// address; NQ_ERR_SHAPE (nothing launched) when the layers are outside its reach.
-nq_status nq_launch_decode_stream(const nq_lrb_layer* const* Ls, int n, const uint16_t* x, uint16_t* const* ys,
-                                  int64_t M, void* ws, cudaStream_t stream, bool pdl);
 // Prefill path (prefill.cu): Y = layer(x) on the tensor cores; with grad != nullptr it writes
 // grad[i] = sum_m cot[m][i] (T U^T)[m][i] instead of Y.
 nq_status nq_launch_prefill(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y, int64_t M, void* ws,
