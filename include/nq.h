@@ -254,19 +254,19 @@ NQ_API nq_status nq_selftest_bounded_wait(int64_t limit_us, void* stream);
 
 /*
  * nq_lrb_matvec_noalloc -- nq_lrb_matvec for callers that cannot allocate device memory.
- * The pages have no counterpart to this entry point; it exists for deployment.  Callers
- * that cannot hand over a workspace: plug-ins that an inference engine gives only their
- * input and output tensors, code issued while a stream is being captured into a CUDA graph
- * (cudaMalloc is not a stream operation and may synchronise the device), latency-critical
- * loops that cannot take an allocator round trip, plain C callers without an allocator.
- * Same operation, arguments and numerics as nq_lrb_matvec, minus the workspace: the
- * scratch (t's digit table and its sums) lives in one statically sized
- * array of NQ_NOALLOC_SCRATCH_BYTES inside libnq.so, which every GPU that loads the library
- * holds until the process exits.  A call whose scratch need (nq_workspace_bytes for the same
- * layer and M <= 8) exceeds that size returns NQ_ERR_SCRATCH_LIMIT without launching.
- * The first call on a device looks up the array's device address (set-up, once per
- * device, on the calling thread with that device current); make that first call before
- * any stream capture.
+ * The pages have no counterpart to this entry point; it exists for deployment.  Callers that
+ * cannot hand over a workspace: plug-ins that an inference engine gives only their input and
+ * output tensors, latency-critical loops that cannot take an allocator round trip, plain C
+ * callers without an allocator.
+ * Same operation, arguments, validation and numerics as nq_lrb_matvec, minus the workspace:
+ * the scratch (t's digit table and its sums) lives in one statically sized array of
+ * NQ_NOALLOC_SCRATCH_BYTES inside libnq.so, which every GPU that loads the library holds until
+ * the process exits.  A call whose scratch need (nq_workspace_bytes for the same layer and
+ * M <= 8) exceeds that size returns NQ_ERR_SCRATCH_LIMIT without launching.  The decode kernels
+ * write all of the scratch they read, so nothing in the array has to start at zero.
+ * The first call on a device looks up the array's device address (set-up, with that device
+ * current; a failed look-up returns NQ_ERR_LAUNCH and is tried again on the next call); make
+ * that first call before any stream capture.
  * All calls on a device share the one array: calls that can overlap on the GPU (different
  * streams, or the same stream without ordering) race and must be serialised by the caller.
  * Never calls cudaMalloc, cudaFree or any allocating routine.

@@ -100,6 +100,21 @@ nq_lrb_layer exchanged(const nq_lrb_layer* L) {
 
 namespace nq_host {
 
+bool pdl_on() { return pdl_enabled(); }
+
+nq_status check_decode_call(const nq_lrb_layer* L, int64_t M) {
+    nq_status st = check_layer(L);
+    if (st != NQ_OK) return st;
+    if (M < 1 || M > NQ_MATVEC_MAX_M) return NQ_ERR_SHAPE;
+    if (nq_decode_stage2_smem(L->r, M) > kMaxDecodeSmem) return NQ_ERR_SHAPE;
+    return NQ_OK;
+}
+
+bool device_ready() {
+    DeviceInfo* d = current_device();
+    return d && d->ok;
+}
+
 int sm_count() {
     DeviceInfo* d = current_device();
     return (d && d->sms > 0) ? d->sms : 148;
@@ -203,10 +218,8 @@ size_t nq_workspace_bytes(const nq_lrb_layer* L, int64_t M) {
 
 nq_status nq_lrb_matvec(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y, int64_t M, void* ws,
                         size_t ws_bytes, void* stream) {
-    nq_status st = check_layer(L);
+    nq_status st = nq_host::check_decode_call(L, M);
     if (st != NQ_OK) return st;
-    if (M < 1 || M > NQ_MATVEC_MAX_M) return NQ_ERR_SHAPE;
-    if (nq_decode_stage2_smem(L->r, M) > kMaxDecodeSmem) return NQ_ERR_SHAPE;
     if ((st = check_io(x, y, ws)) != NQ_OK) return st;
     if (ws_bytes < nq_decode_workspace_bytes(L->d_in, L->r, M)) return NQ_ERR_WORKSPACE;
     DeviceInfo* d = current_device();

@@ -55,6 +55,11 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 
 // Host-side launch plumbing shared by the translation units (defined in api.cu).
 namespace nq_host {
+bool pdl_on();                                    // programmatic dependent launch (off: NQ_DISABLE_PDL=1)
+// Validation shared by the decode entry points: the layer, 1 <= M <= NQ_MATVEC_MAX_M and the
+// shared memory stage 2 needs.  NQ_OK or the status the entry point returns.
+nq_status check_decode_call(const nq_lrb_layer* L, int64_t M);
+bool device_ready();                              // current device is sm_100 and set up
 int sm_count();                                   // multiprocessors of the current device
 unsigned int* error_word();                       // device address of the error word
 cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem, cudaStream_t s, void** args,
