@@ -261,8 +261,10 @@ NQ_API nq_status nq_selftest_bounded_wait(int64_t limit_us, void* stream);
  * Same operation, arguments, validation and numerics as nq_lrb_matvec, minus the workspace:
  * the scratch (t's digit table and its sums) lives in one statically sized array of
  * NQ_NOALLOC_SCRATCH_BYTES inside libnq.so, which every GPU that loads the library holds until
- * the process exits.  A call whose scratch need (nq_workspace_bytes for the same layer and
- * M <= 8) exceeds that size returns NQ_ERR_SCRATCH_LIMIT without launching.  The decode kernels
+ * the process exits.  Every shape that the decode kernels accept fits in it: stage 2's shared
+ * memory caps r (20224 at M <= 2, 11264 at M <= 5, 7680 at M <= 8), and the scratch such a
+ * layer needs stays under 256 KB.  Should a later layout need more than the array holds, the
+ * call returns NQ_ERR_SCRATCH_LIMIT without launching.  The decode kernels
  * write all of the scratch they read, so nothing in the array has to start at zero.
  * The first call on a device looks up the array's device address (set-up, with that device
  * current; a failed look-up returns NQ_ERR_LAUNCH and is tried again on the next call); make

@@ -13,7 +13,8 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "nq.h")
 
-NQ = dict(OK=0, NULL=1, SHAPE=2, ALIGN=3, WORKSPACE=4, DEVICE=5, LAUNCH=6, TIMEOUT=7)
+NQ = dict(OK=0, NULL=1, SHAPE=2, ALIGN=3, WORKSPACE=4, DEVICE=5, LAUNCH=6, TIMEOUT=7, SCRATCH_LIMIT=8)
+NOALLOC_SCRATCH_BYTES = 2 * 1024 * 1024  # NQ_NOALLOC_SCRATCH_BYTES in include/nq.h
 
 
 def declared_symbols():
@@ -214,6 +215,57 @@ def test_no_gpu_gives_device_error(nq):
     # valid arguments, no device: the call must refuse, not fall back to anything
     assert _call(nq, "nq_lrb_matvec", _layer(nq)) == NQ["DEVICE"]
     assert nq.raw_lib().nq_pack_signs(0x1000, 4, 64, 64, 0x2000, 2, None) == NQ["DEVICE"]
+
+
+def _noalloc(nq):
+    fn = nq.raw_lib().nq_lrb_matvec_noalloc
+    fn.restype = ctypes.c_int
+    fn.argtypes = [ctypes.POINTER(nq.nq_lrb_layer), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                   ctypes.c_void_p]
+    return lambda L, x=0x50000, y=0x60000, M=1: fn(ctypes.byref(L) if L is not None else None, x, y, M, None)
+
+
+def test_noalloc_validates_like_matvec(nq):
+    """The allocation-free entry point refuses what nq_lrb_matvec refuses, with the same status."""
+    na = _noalloc(nq)
+    cases = [
+        (None, {}), (_layer(nq, r=48), {}), (_layer(nq, ldu=1), {}), (_layer(nq, U=0), {}),
+        (_layer(nq, s2=0x40002), {}), (_layer(nq, d_out=0), {}),
+        (_layer(nq), dict(M=0)), (_layer(nq), dict(M=9)), (_layer(nq), dict(x=0)), (_layer(nq), dict(y=0)),
+        (_layer(nq), dict(x=0x50008)), (_layer(nq), dict(y=0x60002)),
+        (_layer(nq, r=1 << 17), dict(M=8)),
+    ]
+    for L, kw in cases:
+        want = _call(nq, "nq_lrb_matvec", L, **kw)
+        assert want != NQ["OK"]
+        assert na(L, **kw) == want, (L and (L.d_out, L.d_in, L.r), kw)
+
+
+def test_noalloc_scratch_covers_every_accepted_decode_shape(nq):
+    """For every M the decode path takes, the largest rank r it accepts (stage 2's shared
+    memory caps it) still fits the static scratch: the call gets past the scratch check to the
+    device check, and one step of r further both entry points refuse the shape."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present; accepted shapes would launch")
+    na = _noalloc(nq)
+    lib = nq.raw_lib()
+    for M in range(1, 9):
+        lo, hi = 32, 1 << 22  # lo accepted, hi refused
+        assert na(_layer(nq, r=lo), M=M) == NQ["DEVICE"]
+        assert na(_layer(nq, r=hi), M=M) == NQ["SHAPE"]
+        while hi - lo > 32:
+            mid = (lo + hi) // 64 * 32
+            if na(_layer(nq, r=mid), M=M) == NQ["SHAPE"]:
+                hi = mid
+            else:
+                lo = mid
+        L = _layer(nq, r=lo)
+        assert na(L, M=M) == NQ["DEVICE"], M  # not NQ_ERR_SCRATCH_LIMIT
+        assert _call(nq, "nq_lrb_matvec", L, M=M) == NQ["DEVICE"]
+        assert _call(nq, "nq_lrb_matvec", _layer(nq, r=hi), M=M) == NQ["SHAPE"]
+        need = lib.nq_workspace_bytes(ctypes.byref(_layer(nq, d_out=64, d_in=64, r=lo)), M)
+        assert 0 < need <= NOALLOC_SCRATCH_BYTES, (M, lo, need)
 
 
 def test_binding_refuses_host_tensors_before_any_call(nq):

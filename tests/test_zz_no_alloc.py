@@ -22,7 +22,7 @@ from tests.gpu_util import (REL, ABS, bf16_bits_to_f64, download_bf16_bits, half
 
 pytestmark = pytest.mark.gpu
 
-NQ_ERR_SCRATCH_LIMIT = 8
+NQ_ERR_SHAPE = 2
 
 
 def noalloc_fn():
@@ -63,19 +63,23 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls(workload, M):
         assert np.all(np.abs(got - y_ref) <= REL * S + ABS + half_ulp_bf16(y_ref)), "call %d vs the oracle" % call
 
 
-def test_noalloc_rejects_sizes_beyond_its_scratch():
+def test_noalloc_refuses_oversize_layers_like_matvec():
+    """A layer too large for the decode kernels (r = 131072 at M = 8: stage 2's digit table
+    of t alone would be 3 MiB) is refused by both entry points with the same status, before
+    anything is launched: y keeps its contents."""
     need_gpu()
     mod = nq()
     fn = noalloc_fn()
-    # M = 8 at r = 131072: stage 2's digit table of t alone is 8 bit offsets x 4096 words x 24
-    # columns x 4 B = 3 MiB, more than NQ_NOALLOC_SCRATCH_BYTES; the call must refuse before
-    # launching anything
     M = 8
     p = synth.make_projection("big", 64, 64, 131072, seed=501)
     L = upload_projection(p)
     x = upload_bf16(synth.acts_bf16(synth.rng_for(502), (M, p.d_in)))
-    y = upload_bf16(np.zeros((M, p.d_out), dtype=np.uint16))
-    assert L.workspace_bytes(M) > 2 * 1024 * 1024
+    fill = np.full((M, p.d_out), 0x3F80, dtype=np.uint16)  # bf16 1.0
+    y = upload_bf16(fill)
     st = fn(ctypes.byref(L.struct), x.data_ptr(), y.data_ptr(), M, None)
-    assert st == NQ_ERR_SCRATCH_LIMIT
-    assert "scratch" in mod.status_string(st)
+    assert st == NQ_ERR_SHAPE, mod.status_string(st)
+    with pytest.raises(mod.NQError) as err:
+        mod.lrb_matvec(L, x)
+    assert err.value.status == NQ_ERR_SHAPE
+    mod.sync_status()
+    assert np.array_equal(download_bf16_bits(y), fill)
