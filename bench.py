@@ -442,9 +442,9 @@ def _extra_block(torch, nq, stream, steps, warm, hbm_gbs, wl):
         blocks.append(projs)
     need = max(L.workspace_bytes(1) for bl in blocks for L in bl.values())
     for bl in blocks:
-        for names in (("q", "k", "v"), ("gate", "up")):
-            if all(n in bl for n in names):
-                need = max(need, nq.group_workspace_bytes([bl[n] for n in names], 1))
+        if all(n in bl for n in ("q", "k", "v")):
+            need = max(need, nq.group_workspace_bytes([bl[n] for n in ("q", "k", "v")], 1))
+        need = max(need, nq.mlp_gate_up_workspace_bytes(bl["gate"], bl["up"], 1))
     ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
     dmodel = shapes[0][2]
     x = torch.zeros((1, dmodel), dtype=torch.bfloat16, device="cuda").normal_()
@@ -462,8 +462,7 @@ def _extra_block(torch, nq, stream, steps, warm, hbm_gbs, wl):
                 xin = bufs["o"]
             else:
                 xin = xx
-            nq.layer_forward_group([bl["gate"], bl["up"]], xin, [bufs["gate"], bufs["up"]], ws=ws, stream=stream)
-            nq.silu_mul(bufs["gate"], bufs["up"], h, stream=stream)
+            nq.mlp_gate_up(bl["gate"], bl["up"], xin, h, ws=ws, stream=stream)
             nq.layer_forward(bl["down"], h, bufs["down"], ws=ws, stream=stream)
             xx = bufs["down"]
 
@@ -474,7 +473,8 @@ def _extra_block(torch, nq, stream, steps, warm, hbm_gbs, wl):
     return {"us_per_block": round(us, 3), "block_bytes": block_bytes, "GB_s": round(block_bytes / us / 1e3, 1),
             "frac_hbm": round(block_bytes / us / 1e3 / hbm_gbs, 4), "blocks_per_step": reps,
             "block": "+".join(n for (n, *_r) in shapes) + " + silu_mul",
-            "grouped": "q,k,v and gate,up each one nq_layer_forward_group call (shared input)"}
+            "grouped": ("q,k,v one nq_layer_forward_group call (shared input); " if shapes[0][0] == "q" else "")
+                       + "gate,up and SiLU.mul one nq_mlp_gate_up call"}
 
 
 def _extra_prefill(torch, nq, stream, steps, bf16_tf):
@@ -618,7 +618,7 @@ def _extra_model70b(torch, nq, stream, hbm_gbs, n_layers=80):
                        for (name, do, di, r) in shapes})
     need = max(L.workspace_bytes(1) for bl in layers for L in bl.values())
     need = max(need, nq.group_workspace_bytes([layers[0]["q"], layers[0]["k"], layers[0]["v"]], 1),
-               nq.group_workspace_bytes([layers[0]["gate"], layers[0]["up"]], 1))
+               nq.mlp_gate_up_workspace_bytes(layers[0]["gate"], layers[0]["up"], 1))
     ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
     dmodel = shapes[0][2]
     x = torch.zeros((1, dmodel), dtype=torch.bfloat16, device="cuda").normal_()
@@ -631,9 +631,7 @@ def _extra_model70b(torch, nq, stream, hbm_gbs, n_layers=80):
             nq.layer_forward_group([bl["q"], bl["k"], bl["v"]], xx, [bufs["q"], bufs["k"], bufs["v"]], ws=ws,
                                    stream=stream)
             nq.layer_forward(bl["o"], bufs["q"], bufs["o"], ws=ws, stream=stream)  # stands in for attention
-            nq.layer_forward_group([bl["gate"], bl["up"]], bufs["o"], [bufs["gate"], bufs["up"]], ws=ws,
-                                   stream=stream)
-            nq.silu_mul(bufs["gate"], bufs["up"], h, stream=stream)
+            nq.mlp_gate_up(bl["gate"], bl["up"], bufs["o"], h, ws=ws, stream=stream)
             nq.layer_forward(bl["down"], h, bufs["down"], ws=ws, stream=stream)
             xx = bufs["down"]
 
@@ -646,8 +644,8 @@ def _extra_model70b(torch, nq, stream, hbm_gbs, n_layers=80):
     return {"layers": n_layers, "weights_GB": round(wbytes / 1e9, 3), "us_per_token": round(us, 1),
             "tokens_per_s": round(1e6 / us, 1), "GB_s": round(alg / us / 1e3, 1),
             "frac_hbm": round(alg / us / 1e3 / hbm_gbs, 4),
-            "note": "LRB projections + SiLU.mul only; o takes q's output in place of attention; q,k,v and "
-                    "gate,up grouped"}
+            "note": "LRB projections + SiLU.mul only; o takes q's output in place of attention; q,k,v "
+                    "grouped; gate,up and SiLU.mul one fused call"}
 
 
 def _extra_pack(torch, nq, stream, steps, warm, hbm_gbs):

@@ -229,6 +229,24 @@ NQ_API nq_status nq_layer_forward_group(const nq_lrb_layer* const* layers, int n
                                         uint16_t* const* y, int64_t M, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * nq_mlp_gate_up -- h = bf16( silu(bf16(gate x)) * bf16(up x) ) for the gate and up projections
+ * of a Llama MLP block built from LRB layers (the pages quantise each projection on its own;
+ * the block around them is not part of the factorisation).  gate and up share x: equal d_in
+ * and equal d_out, r may differ.  The result equals, bit for bit, nq_layer_forward_group on
+ * {gate, up} followed by nq_silu_mul of its two outputs, but for M <= NQ_MATVEC_MAX_M the gate
+ * and up outputs never reach memory: stage 2 of the grouped decode computes both projections of
+ * a row in the same block and applies SiLU.mul in its epilogue, one launch fewer per MLP block.
+ * Larger M (or ranks whose two stage-2 tables do not fit on chip together) runs the unfused
+ * calls, with the two outputs kept in the workspace.  x [M][d_in], h [M][d_out] bf16, device,
+ * 16-byte aligned; ws: nq_mlp_gate_up_workspace_bytes(gate, up, M) bytes (0 for invalid
+ * layers or M < 1).  Errors: NQ_ERR_NULL, NQ_ERR_ALIGN, NQ_ERR_SHAPE (d_in or d_out differ,
+ * M < 1, a layer too large for the decode path), NQ_ERR_WORKSPACE, NQ_ERR_DEVICE.
+ */
+NQ_API size_t nq_mlp_gate_up_workspace_bytes(const nq_lrb_layer* gate, const nq_lrb_layer* up, int64_t M);
+NQ_API nq_status nq_mlp_gate_up(const nq_lrb_layer* gate, const nq_lrb_layer* up, const uint16_t* x, uint16_t* h,
+                                int64_t M, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * nq_silu_mul -- h[e] = bf16( silu(g[e]) * u[e] ), silu(g) = g / (1 + exp(-g)), fp32 math,
  * for the Llama MLP block built from LRB projections (gate, up -> h -> down).  Not part of
  * the factorisation itself.  g, u, h: n bf16 values each, device.

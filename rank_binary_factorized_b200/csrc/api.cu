@@ -16,6 +16,9 @@ size_t nq_decode_workspace_bytes(int64_t d_in, int64_t r, int64_t M);
 size_t nq_decode_stage2_smem(int64_t r, int64_t M);
 nq_status nq_launch_silu_mul(const uint16_t*, const uint16_t*, uint16_t*, int64_t, cudaStream_t, bool);
 size_t nq_prefill_workspace_bytes(const nq_lrb_layer*, int64_t M);
+size_t nq_decode_pair_smem(int64_t r0, int64_t r1, int64_t M);
+nq_status nq_launch_decode_gate_up(const nq_lrb_layer* gate, const nq_lrb_layer* up, const uint16_t* x, uint16_t* h,
+                                   int64_t M, void* ws, cudaStream_t stream, bool pdl);
 size_t nq_from_latent_ws(int64_t d_out, int64_t d_in, int64_t ldu, int64_t ldv);
 nq_status nq_launch_from_latent(const float* Uh, int64_t ld_uh, const float* Vh, int64_t ld_vh, int64_t d_out,
                                 int64_t d_in, int64_t r, uint32_t* U, int64_t ldu, uint32_t* V, int64_t ldv,
@@ -360,6 +363,53 @@ nq_status nq_lrb_from_latent(const float* Uh, int64_t ld_uh, const float* Vh, in
     if (!d || !d->ok) return NQ_ERR_DEVICE;
     return nq_launch_from_latent(Uh, ld_uh, Vh, ld_vh, d_out, d_in, r, U, ldu, V, ldv, s1, s2, eta, ws,
                                  static_cast<cudaStream_t>(stream));
+}
+
+namespace {
+// The unfused gate and up outputs ([M][d_out] bf16 each) follow the grouped workspace.
+size_t mlp_tmp_offset(const nq_lrb_layer* const* gu, int64_t M) {
+    return (nq_group_workspace_bytes(gu, 2, M) + 255) / 256 * 256;
+}
+size_t mlp_tmp_bytes(const nq_lrb_layer* gate, int64_t M) {
+    return (static_cast<size_t>(M) * gate->d_out * 2 + 255) / 256 * 256;
+}
+}  // namespace
+
+size_t nq_mlp_gate_up_workspace_bytes(const nq_lrb_layer* gate, const nq_lrb_layer* up, int64_t M) {
+    if (M < 1 || check_layer(gate) != NQ_OK || check_layer(up) != NQ_OK) return 0;
+    if (gate->d_in != up->d_in || gate->d_out != up->d_out) return 0;
+    const nq_lrb_layer* gu[2] = {gate, up};
+    return mlp_tmp_offset(gu, M) + 2 * mlp_tmp_bytes(gate, M);
+}
+
+nq_status nq_mlp_gate_up(const nq_lrb_layer* gate, const nq_lrb_layer* up, const uint16_t* x, uint16_t* h,
+                         int64_t M, void* ws, size_t ws_bytes, void* stream) {
+    nq_status st;
+    if ((st = check_layer(gate)) != NQ_OK || (st = check_layer(up)) != NQ_OK) return st;
+    if (M < 1 || gate->d_in != up->d_in || gate->d_out != up->d_out) return NQ_ERR_SHAPE;
+    if (M <= NQ_MATVEC_MAX_M && (nq_decode_stage2_smem(gate->r, M) > kMaxDecodeSmem ||
+                                 nq_decode_stage2_smem(up->r, M) > kMaxDecodeSmem))
+        return NQ_ERR_SHAPE;
+    if ((st = check_io(x, h, ws)) != NQ_OK) return st;
+    if (ws_bytes < nq_mlp_gate_up_workspace_bytes(gate, up, M)) return NQ_ERR_WORKSPACE;
+    DeviceInfo* d = current_device();
+    if (!d || !d->ok) return NQ_ERR_DEVICE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (M <= NQ_MATVEC_MAX_M && nq_decode_pair_smem(gate->r, up->r, M) <= kMaxDecodeSmem)
+        return nq_launch_decode_gate_up(gate, up, x, h, M, ws, s, pdl_enabled());
+    // unfused: both projections into the workspace, then SiLU.mul
+    const nq_lrb_layer* gu[2] = {gate, up};
+    char* tmp = static_cast<char*>(ws) + mlp_tmp_offset(gu, M);
+    uint16_t* g = reinterpret_cast<uint16_t*>(tmp);
+    uint16_t* u = reinterpret_cast<uint16_t*>(tmp + mlp_tmp_bytes(gate, M));
+    uint16_t* outs[2] = {g, u};
+    if (M <= NQ_MATVEC_MAX_M) {
+        if ((st = nq_launch_decode_group(gu, 2, x, outs, M, ws, s, pdl_enabled())) != NQ_OK) return st;
+    } else {
+        for (int l = 0; l < 2; ++l)
+            if ((st = nq_launch_prefill(gu[l], x, outs[l], M, ws, s, pdl_enabled())) != NQ_OK) return st;
+    }
+    return nq_launch_silu_mul(g, u, h, M * gate->d_out, s, pdl_enabled());
 }
 
 nq_status nq_silu_mul(const uint16_t* g, const uint16_t* u, uint16_t* h, int64_t n, void* stream) {

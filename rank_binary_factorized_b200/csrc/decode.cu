@@ -20,6 +20,7 @@
 #include <cooperative_groups.h>
 
 #include <algorithm>
+#include <cstdlib>
 
 #include "nq_common.cuh"
 
@@ -44,6 +45,11 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// Asks the copy engine to bring [src, src + bytes) into L2 (no completion to wait for);
+// src and bytes are multiples of 16.
+__device__ __forceinline__ void l2_prefetch_bulk(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 
 // The three balanced base-256 digits of a 23-bit signed integer v = a0 + 2^8 a1 + 2^16 a2,
 // each in [-128, 127], returned as s8 bytes.
@@ -124,6 +130,7 @@ struct S1Params {
     long long* tsum;
     int* tsh;
     int nwp;  // words per row padded to a multiple of 8 (the table's geometry)
+    int prefetch;  // prefetch the slice's rows of V into L2 (whole rows) before gathering strips
 };
 
 // Up to kMaxGroup projections that share their input x are launched as one grid: block
@@ -245,6 +252,25 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const __grid_const
     for (int i = 0; i < kS2Reg; ++i) {
         const int64_t j = j0 + tid + static_cast<int64_t>(i) * kS1Threads;
         s2r[i] = (s2reg && j < j1) ? f16_bits_to_float(__ldg(p.s2 + j)) : 0.0f;
+    }
+    if (warp == 0 && p.prefetch) {
+        // the slice's rows of V, whole rows, split among the blocks of this row slice: one
+        // contiguous range per block, prefetched into L2 by the copy engine, so that DRAM
+        // streams full lines while the blocks' 32-byte strips are gathered from L2
+        const int nc = grp.chunk_off[li + 1] - grp.chunk_off[li];
+        const int64_t rows = j1 - j0;
+        const int64_t r0 = j0 + (rows * chunk) / nc, r1 = j0 + (rows * (chunk + 1)) / nc;
+        if (r1 > r0) {
+            // from the 16-byte boundary at or below row r0 (V itself is 16-byte aligned) to the
+            // last row's r/32-th word, rounded up to 16 bytes
+            const uintptr_t b0 = reinterpret_cast<uintptr_t>(p.V + r0 * p.ldv);
+            const uintptr_t b1 = reinterpret_cast<uintptr_t>(p.V + (r1 - 1) * p.ldv + p.nw);
+            const char* a = reinterpret_cast<const char*>(b0 & ~static_cast<uintptr_t>(15));
+            const int64_t units = static_cast<int64_t>((b1 - (b0 & ~static_cast<uintptr_t>(15)) + 15) / 16);
+            constexpr int64_t kPiece = 2048;  // 16-byte units per prefetch (32 KB)
+            for (int64_t u = static_cast<int64_t>(lane) * kPiece; u < units; u += 32 * kPiece)
+                l2_prefetch_bulk(a + 16 * u, static_cast<uint32_t>(16 * min(kPiece, units - u)));
+        }
     }
     build_aws(j0);  // weights only: may overlap the previous grid
     pdl_launch_dependents();
@@ -607,53 +633,167 @@ struct S2Params {
     float* grad;
 };
 
-// Stage-2 blocks [cta_off[l], cta_off[l + 1]) work for member l of the group.
+// Stage-2 blocks [cta_off[l], cta_off[l + 1]) work for member l of the group.  In the paired
+// form (gate and up of an MLP block, equal d_out) every block works for both members on the
+// same rows and writes h = bf16(silu(bf16(gate)) * bf16(up)) to member 0's y.
 struct S2Group {
     S2Params p[kMaxGroup];
     int cta_off[kMaxGroup + 1];
     int n;
 };
 
-template <int NT, int TH, int GN>
+// h from the bf16 gate and up values: the same function as the elementwise SiLU.mul kernel
+__device__ __forceinline__ uint16_t silu_mul_bf16(uint16_t g, uint16_t u) {
+    const float gf = bf16_bits_to_float(g);
+    const float sg = gf / (1.0f + expf(-gf));
+    return float_to_bf16_bits(sg * bf16_bits_to_float(u));
+}
+
+// One member's share of stage 2 in shared memory: its digit table, the staged rows of U, the
+// per-row integer sums and the staged s1.
+struct S2Smem {
+    uint32_t* bt;    // 8 * nwp * NT*8 words (s2_bidx)
+    uint32_t* ublk;  // [chunk_mt*16][su]
+    int* red;        // [chunk_mt*16][NT*8]
+    float* s1_s;     // [chunk_mt*16]
+};
+
+template <int NT>
+__device__ __forceinline__ size_t s2_smem_words(const S2Params& p) {
+    return static_cast<size_t>(8) * p.nwp * NT * 8 + static_cast<size_t>(p.chunk_mt) * 16 * p.su +
+           static_cast<size_t>(p.chunk_mt) * 16 * NT * 8 + static_cast<size_t>(p.chunk_mt) * 16;
+}
+
+template <int NT>
+__device__ __forceinline__ S2Smem s2_carve(const S2Params& p, uint32_t* base) {
+    S2Smem m;
+    m.bt = base;
+    m.ublk = m.bt + 8 * p.nwp * NT * 8;
+    m.red = reinterpret_cast<int*>(m.ublk + p.chunk_mt * 16 * p.su);
+    m.s1_s = reinterpret_cast<float*>(m.red + p.chunk_mt * 16 * NT * 8);
+    return m;
+}
+
+// The MMAs of M-tiles [c0, c0 + nmt) of one member (rows staged in sm.ublk), added into sm.red:
+// each warp takes an equal, contiguous share of the (M-tile, word-group) pairs in M-tile-major
+// order and flushes its accumulators whenever its run leaves an M-tile.
+template <int NT, int kWarps>
+__device__ __forceinline__ void s2_mma_chunk(const S2Params& p, const S2Smem& sm, int nmt, int warp, int lane) {
+    const int gid = lane >> 2, tig = lane & 3;
+    const int ng = p.nwp / 8;
+    const int pairs = nmt * ng;
+    const int p_lo = (warp * pairs) / kWarps, p_hi = ((warp + 1) * pairs) / kWarps;
+    int pp = p_lo;
+    while (pp < p_hi) {
+        const int mtl = pp / ng;
+        const int g_lo = pp - mtl * ng;
+        const int g_hi = min(ng, g_lo + (p_hi - pp));
+        pp += g_hi - g_lo;
+        int acc[8][NT][4];
+#pragma unroll
+        for (int s_ = 0; s_ < 8; ++s_)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[s_][nt][e] = 0;
+        const uint32_t* u0 = sm.ublk + (mtl * 16 + gid) * p.su;
+        const uint32_t* u1 = u0 + 8 * p.su;
+        uint32_t w00 = u0[8 * g_lo + tig], w01 = u0[8 * g_lo + 4 + tig];
+        uint32_t w10 = u1[8 * g_lo + tig], w11 = u1[8 * g_lo + 4 + tig];
+        for (int g = g_lo; g < g_hi; ++g) {
+            const int wb = 8 * g;
+            // next group's words, loaded while this group's MMAs issue
+            const int wn = (g + 1 < g_hi) ? wb + 8 : wb;
+            const uint32_t n00 = u0[wn + tig], n01 = u0[wn + 4 + tig];
+            const uint32_t n10 = u1[wn + tig], n11 = u1[wn + 4 + tig];
+#pragma unroll
+            for (int s_ = 0; s_ < 8; ++s_) {
+                const uint32_t msk = 0x01010101u << s_;
+                const uint32_t a0 = w00 & msk, a1 = w10 & msk, a2 = w01 & msk, a3 = w11 & msk;
+                const uint2* b = reinterpret_cast<const uint2*>(sm.bt) + ((s_ * ng + g) * NT) * 32 + lane;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const uint2 bb = b[nt * 32];
+                    mma_u8s8(acc[s_][nt], a0, a1, a2, a3, bb.x, bb.y);
+                }
+            }
+            w00 = n00; w01 = n01; w10 = n10; w11 = n11;
+        }
+        // D[row][col]: e = 0,1 -> row gid, cols 2tig, 2tig+1; e = 2,3 -> row gid+8
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                int v = 0;
+#pragma unroll
+                for (int s_ = 0; s_ < 8; ++s_) v += acc[s_][nt][e] >> s_;
+                const int row = mtl * 16 + gid + ((e >> 1) << 3);
+                const int col = nt * 8 + 2 * tig + (e & 1);
+                atomicAdd(&sm.red[row * (NT * 8) + col], v);
+            }
+    }
+}
+
+// (U t_m) for staged row `row` as 2^-shift (2 P - Tsum), P = d0 + 2^8 d1 + 2^16 d2: exact
+// integers times a power of two
+template <int NT>
+__device__ __forceinline__ double s2_value(const S2Smem& sm, int row, int m, long long tsum, double dinv) {
+    const int* rr = sm.red + row * (NT * 8) + 3 * m;
+    const long long P = static_cast<long long>(rr[0]) + (static_cast<long long>(rr[1]) << 8) +
+                        (static_cast<long long>(rr[2]) << 16);
+    return static_cast<double>(2 * P - tsum) * dinv;
+}
+
+template <int NT, int TH, int GN, bool PAIR>
 __global__ void __launch_bounds__(TH, 1) decode_stage2_kernel(const __grid_constant__ S2Group grp) {
     constexpr int kS2Threads = TH;
     constexpr int kS2Warps = kS2Threads / 32;
+    constexpr int NM = PAIR ? 2 : 1;  // members this block works for
     extern __shared__ __align__(16) uint32_t smem2[];
-    int li = 0;  // the member of the group this block works for
-    if (GN > 1)
+    int li = 0;  // the (first) member of the group this block works for
+    if (GN > 1 && !PAIR)
         while (li + 1 < grp.n && static_cast<int>(blockIdx.x) >= grp.cta_off[li + 1]) ++li;
-    const S2Params& p = grp.p[li];
     const int bid = blockIdx.x - grp.cta_off[li];
     const int G = grp.cta_off[li + 1] - grp.cta_off[li];
-    uint32_t* bt = smem2;                                  // 8 * nwp * NT*8 words (s2_bidx)
-    uint32_t* ublk = bt + 8 * p.nwp * NT * 8;              // [chunk_mt*16][su]
-    int* red = reinterpret_cast<int*>(ublk + p.chunk_mt * 16 * p.su);  // [chunk_mt*16][NT*8]
-    float* s1_s = reinterpret_cast<float*>(red + p.chunk_mt * 16 * NT * 8);  // [chunk_mt*16]
-    __shared__ double s_dinv[NQ_MATVEC_MAX_M];  // 2^-shift: turns the exact integers into values
-    __shared__ unsigned long long s_tsum[NQ_MATVEC_MAX_M];
+    S2Smem sm[NM];
+    {
+        uint32_t* base = smem2;
+#pragma unroll
+        for (int k = 0; k < NM; ++k) {
+            sm[k] = s2_carve<NT>(grp.p[li + k], base);
+            base += s2_smem_words<NT>(grp.p[li + k]);
+        }
+    }
+    const S2Params& p = grp.p[li];  // rows, chunking and output of the block (member 0 of a pair)
+    __shared__ double s_dinv[NM][NQ_MATVEC_MAX_M];  // 2^-shift: turns the exact integers into values
+    __shared__ unsigned long long s_tsum[NM][NQ_MATVEC_MAX_M];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    if (tid < NQ_MATVEC_MAX_M) s_tsum[tid] = 0ull;
+    if (tid < NM * NQ_MATVEC_MAX_M) s_tsum[tid / NQ_MATVEC_MAX_M][tid % NQ_MATVEC_MAX_M] = 0ull;
     __syncthreads();
 
     const int mt0 = static_cast<int>((static_cast<int64_t>(bid) * p.mt_total) / G);
     const int mt1 = static_cast<int>((static_cast<int64_t>(bid + 1) * p.mt_total) / G);
 
-    // stage the rows of U of M-tiles [a, b) into ublk (row stride su); weights only, so this
-    // may run before the previous grid has finished
+    // stage the rows of U of M-tiles [a, b) into ublk (row stride su), for each member; weights
+    // only, so this may run before the previous grid has finished
     auto load_u = [&](int a, int b) {
-        const int64_t row0 = static_cast<int64_t>(a) * 16;
-        const int64_t row1 = min(static_cast<int64_t>(b) * 16, p.d_out);
-        const int rows = static_cast<int>(row1 - row0);
-        const bool even = ((p.ldu & 1) == 0) && ((p.nw & 1) == 0);
-        // one warp per row, lanes along the row
-        for (int rr = warp; rr < rows; rr += kS2Warps) {
-            const uint32_t* src = p.U + (row0 + rr) * p.ldu;
-            const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(ublk + rr * p.su));
-            if (even) {
-                for (int c = lane; c < p.nw / 2; c += 32) cp_async8(dst + 8u * c, src + 2 * c);
-            } else {
-                for (int c = lane; c < p.nw; c += 32) cp_async4(dst + 4u * c, src + c);
+#pragma unroll
+        for (int k = 0; k < NM; ++k) {
+            const S2Params& q = grp.p[li + k];
+            const int64_t row0 = static_cast<int64_t>(a) * 16;
+            const int64_t row1 = min(static_cast<int64_t>(b) * 16, q.d_out);
+            const int rows = static_cast<int>(row1 - row0);
+            const bool even = ((q.ldu & 1) == 0) && ((q.nw & 1) == 0);
+            // one warp per row, lanes along the row
+            for (int rr = warp; rr < rows; rr += kS2Warps) {
+                const uint32_t* src = q.U + (row0 + rr) * q.ldu;
+                const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(sm[k].ublk + rr * q.su));
+                if (even) {
+                    for (int c = lane; c < q.nw / 2; c += 32) cp_async8(dst + 8u * c, src + 2 * c);
+                } else {
+                    for (int c = lane; c < q.nw; c += 32) cp_async4(dst + 4u * c, src + c);
+                }
             }
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
@@ -661,9 +801,13 @@ __global__ void __launch_bounds__(TH, 1) decode_stage2_kernel(const __grid_const
 
     // s1 of the same rows (a weight), as fp32, for the epilogue
     auto load_s1 = [&](int a, int b) {
-        const int64_t row0 = static_cast<int64_t>(a) * 16;
-        const int rows = static_cast<int>(min(static_cast<int64_t>(b) * 16, p.d_out) - row0);
-        for (int i = tid; i < rows; i += kS2Threads) s1_s[i] = f16_bits_to_float(__ldg(p.s1 + row0 + i));
+#pragma unroll
+        for (int k = 0; k < NM; ++k) {
+            const S2Params& q = grp.p[li + k];
+            const int64_t row0 = static_cast<int64_t>(a) * 16;
+            const int rows = static_cast<int>(min(static_cast<int64_t>(b) * 16, q.d_out) - row0);
+            for (int i = tid; i < rows; i += kS2Threads) sm[k].s1_s[i] = f16_bits_to_float(__ldg(q.s1 + row0 + i));
+        }
     };
 
     if (mt0 < mt1) {
@@ -675,127 +819,86 @@ __global__ void __launch_bounds__(TH, 1) decode_stage2_kernel(const __grid_const
 
     // ---- t as stage 1 left it: the digit table goes to shared memory as it is (the chunk
     // loop's wait and barrier publish it), the shift and the sum of t_q come from the owners
-    {
-        const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(bt));
-        const int pieces = 2 * p.nwp * NT * 8;  // 16-byte pieces of 8 nwp NT 8 words
-        for (int c = tid; c < pieces; c += kS2Threads) cp_async16(dst + 16u * c, p.tab + 4 * c);
-        asm volatile("cp.async.commit_group;" ::: "memory");
-        // warp m adds row m's owner sums (exact integers), lane 0 keeps the result; each lane
-        // issues its loads four at a time, so the sums cost one round trip to L2
-        for (int m = warp; m < p.M; m += kS2Warps) {
-            const int sh = p.tsh[m];
-            long long v = 0;
-            for (int i0 = lane; i0 < p.tsum_n; i0 += 4 * 32) {
-                long long a[4];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int i = i0 + 32 * u;
-                    a[u] = (i < p.tsum_n) ? p.tsum[static_cast<int64_t>(i) * p.M + m] : 0ll;
-                }
-                v += (a[0] + a[1]) + (a[2] + a[3]);
+    for (int k = 0; k < NM; ++k) {
+        const S2Params& q = grp.p[li + k];
+        const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(sm[k].bt));
+        const int pieces = 2 * q.nwp * NT * 8;  // 16-byte pieces of 8 nwp NT 8 words
+        for (int c = tid; c < pieces; c += kS2Threads) cp_async16(dst + 16u * c, q.tab + 4 * c);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    // warp (k, m) adds member k's row-m owner sums (exact integers), lane 0 keeps the result;
+    // each lane issues its loads four at a time, so the sums cost one round trip to L2
+    for (int km = warp; km < NM * p.M; km += kS2Warps) {
+        const int k = km / p.M, m = km - k * p.M;
+        const S2Params& q = grp.p[li + k];
+        const int sh = q.tsh[m];
+        long long v = 0;
+        for (int i0 = lane; i0 < q.tsum_n; i0 += 4 * 32) {
+            long long a[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + 32 * u;
+                a[u] = (i < q.tsum_n) ? q.tsum[static_cast<int64_t>(i) * q.M + m] : 0ll;
             }
-            for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-            if (lane == 0) {
-                s_tsum[m] = static_cast<unsigned long long>(v);
-                s_dinv[m] = pow2_d(-sh);
-            }
+            v += (a[0] + a[1]) + (a[2] + a[3]);
+        }
+        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        if (lane == 0) {
+            s_tsum[k][m] = static_cast<unsigned long long>(v);
+            s_dinv[k][m] = pow2_d(-sh);
         }
     }
 
-    const int gid = lane >> 2, tig = lane & 3;
-    const int ng = p.nwp / 8;
     for (int c0 = mt0; c0 < mt1; c0 += p.chunk_mt) {
         const int c1 = min(mt1, c0 + p.chunk_mt);
         const int nmt = c1 - c0;
-        for (int e = tid; e < nmt * 16 * NT * 8; e += kS2Threads) red[e] = 0;
+#pragma unroll
+        for (int k = 0; k < NM; ++k)
+            for (int e = tid; e < nmt * 16 * NT * 8; e += kS2Threads) sm[k].red[e] = 0;
         cp_async_wait_all();
         __syncthreads();
-
-        // each warp takes an equal, contiguous share of the (M-tile, word-group) pairs in
-        // M-tile-major order and flushes its accumulators whenever its run leaves an M-tile
-        const int pairs = nmt * ng;
-        const int p_lo = (warp * pairs) / kS2Warps, p_hi = ((warp + 1) * pairs) / kS2Warps;
-        int pp = p_lo;
-        while (pp < p_hi) {
-            const int mtl = pp / ng;
-            const int g_lo = pp - mtl * ng;
-            const int g_hi = min(ng, g_lo + (p_hi - pp));
-            pp += g_hi - g_lo;
-            int acc[8][NT][4];
 #pragma unroll
-            for (int s_ = 0; s_ < 8; ++s_)
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) acc[s_][nt][e] = 0;
-            const uint32_t* u0 = ublk + (mtl * 16 + gid) * p.su;
-            const uint32_t* u1 = u0 + 8 * p.su;
-            uint32_t w00 = u0[8 * g_lo + tig], w01 = u0[8 * g_lo + 4 + tig];
-            uint32_t w10 = u1[8 * g_lo + tig], w11 = u1[8 * g_lo + 4 + tig];
-            for (int g = g_lo; g < g_hi; ++g) {
-                const int wb = 8 * g;
-                // next group's words, loaded while this group's MMAs issue
-                const int wn = (g + 1 < g_hi) ? wb + 8 : wb;
-                const uint32_t n00 = u0[wn + tig], n01 = u0[wn + 4 + tig];
-                const uint32_t n10 = u1[wn + tig], n11 = u1[wn + 4 + tig];
-#pragma unroll
-                for (int s_ = 0; s_ < 8; ++s_) {
-                    const uint32_t msk = 0x01010101u << s_;
-                    const uint32_t a0 = w00 & msk, a1 = w10 & msk, a2 = w01 & msk, a3 = w11 & msk;
-                    const uint2* b = reinterpret_cast<const uint2*>(bt) + ((s_ * ng + g) * NT) * 32 + lane;
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        const uint2 bb = b[nt * 32];
-                        mma_u8s8(acc[s_][nt], a0, a1, a2, a3, bb.x, bb.y);
-                    }
-                }
-                w00 = n00; w01 = n01; w10 = n10; w11 = n11;
-            }
-            // D[row][col]: e = 0,1 -> row gid, cols 2tig, 2tig+1; e = 2,3 -> row gid+8
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    int v = 0;
-#pragma unroll
-                    for (int s_ = 0; s_ < 8; ++s_) v += acc[s_][nt][e] >> s_;
-                    const int row = mtl * 16 + gid + ((e >> 1) << 3);
-                    const int col = nt * 8 + 2 * tig + (e & 1);
-                    atomicAdd(&red[row * (NT * 8) + col], v);
-                }
-        }
+        for (int k = 0; k < NM; ++k) s2_mma_chunk<NT, kS2Warps>(grp.p[li + k], sm[k], nmt, warp, lane);
         __syncthreads();
 
-        // epilogue: y = s1 * 2^-shift * (2 P - Tsum), P = d0 + 2^8 d1 + 2^16 d2
-        if (p.grad) {
-            // (U t_m)_i = 2^-shift (2 P - Tsum), weighted by the cotangent and summed over m in
-            // order, in fp64
+        if (PAIR) {
+            // h = silu(g) u from the bf16 gate and up outputs of the same row
+            for (int e = tid; e < nmt * 16 * p.M; e += kS2Threads) {
+                const int row = (p.M == 1) ? e : e / p.M, m = e - row * p.M;
+                const int64_t i = static_cast<int64_t>(c0) * 16 + row;
+                if (i < p.d_out) {
+                    const double gv = static_cast<double>(sm[0].s1_s[row]) *
+                                      s2_value<NT>(sm[0], row, m, static_cast<long long>(s_tsum[0][m]), s_dinv[0][m]);
+                    const double uv = static_cast<double>(sm[NM - 1].s1_s[row]) *
+                                      s2_value<NT>(sm[NM - 1], row, m, static_cast<long long>(s_tsum[NM - 1][m]),
+                                                   s_dinv[NM - 1][m]);
+                    p.y[static_cast<int64_t>(m) * p.d_out + i] =
+                        silu_mul_bf16(__bfloat16_as_ushort(__double2bfloat16(gv)), __bfloat16_as_ushort(__double2bfloat16(uv)));
+                }
+            }
+        } else if (p.grad) {
+            // (U t_m)_i weighted by the cotangent and summed over m in order, in fp64
             for (int row = tid; row < nmt * 16; row += kS2Threads) {
                 const int64_t i = static_cast<int64_t>(c0) * 16 + row;
                 if (i < p.d_out) {
                     double g = 0.0;
-                    for (int m = 0; m < p.M; ++m) {
-                        const int* rr = red + row * (NT * 8) + 3 * m;
-                        const long long P = static_cast<long long>(rr[0]) + (static_cast<long long>(rr[1]) << 8) +
-                                            (static_cast<long long>(rr[2]) << 16);
-                        const long long val = 2 * P - static_cast<long long>(s_tsum[m]);
+                    for (int m = 0; m < p.M; ++m)
                         g += static_cast<double>(bf16_bits_to_float(p.cot[static_cast<int64_t>(m) * p.d_out + i])) *
-                             (static_cast<double>(val) * s_dinv[m]);
-                    }
+                             s2_value<NT>(sm[0], row, m, static_cast<long long>(s_tsum[0][m]), s_dinv[0][m]);
                     p.grad[i] = static_cast<float>(g);
                 }
             }
-        }
-        for (int e = tid; e < (p.grad ? 0 : nmt * 16 * p.M); e += kS2Threads) {
-            const int row = (p.M == 1) ? e : e / p.M, m = e - row * p.M;
-            const int64_t i = static_cast<int64_t>(c0) * 16 + row;
-            if (i < p.d_out) {
-                const int* rr = red + row * (NT * 8) + 3 * m;
-                const long long P = static_cast<long long>(rr[0]) + (static_cast<long long>(rr[1]) << 8) +
-                                    (static_cast<long long>(rr[2]) << 16);
-                const long long val = 2 * P - static_cast<long long>(s_tsum[m]);
-                const double yv = static_cast<double>(s1_s[row]) * (static_cast<double>(val) * s_dinv[m]);
-                p.y[static_cast<int64_t>(m) * p.d_out + i] = __bfloat16_as_ushort(__double2bfloat16(yv));
+        } else {
+            // y = s1 * 2^-shift * (2 P - Tsum)
+            for (int e = tid; e < nmt * 16 * p.M; e += kS2Threads) {
+                const int row = (p.M == 1) ? e : e / p.M, m = e - row * p.M;
+                const int64_t i = static_cast<int64_t>(c0) * 16 + row;
+                if (i < p.d_out) {
+                    const double yv = static_cast<double>(sm[0].s1_s[row]) *
+                                      s2_value<NT>(sm[0], row, m, static_cast<long long>(s_tsum[0][m]), s_dinv[0][m]);
+                    p.y[static_cast<int64_t>(m) * p.d_out + i] = __bfloat16_as_ushort(__double2bfloat16(yv));
+                }
             }
         }
         __syncthreads();
@@ -877,25 +980,44 @@ TLayout t_layout(int64_t r, int64_t M) {
 
 size_t decode_ws_bytes(int64_t r, int64_t M) { return kWsHeader + t_layout(r, M).total; }
 
-template <int NT, int TH1, int TH2, int GN>
-void set_attrs_once() {
+// Stage 1 prefetches its rows of V into L2 (off with NQ_DECODE_PREFETCH=0).
+bool prefetch_v() {
+    static const bool on = [] {
+        const char* e = std::getenv("NQ_DECODE_PREFETCH");
+        return !(e && e[0] == '0');
+    }();
+    return on;
+}
+
+template <int NT, int TH, int GN>
+void set_stage1_attrs_once() {
     static std::atomic<bool> done[64];  // per device; setting an attribute twice is harmless
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || done[dev].load(std::memory_order_acquire)) return;
-    cudaFuncSetAttribute(nq::decode_stage1_kernel<NT, TH1, GN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(nq::decode_stage1_kernel<NT, TH, GN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(kStage1SmemBudget));
-    cudaFuncSetAttribute(nq::decode_stage1_kernel<NT, TH1, GN>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    cudaFuncSetAttribute(nq::decode_stage2_kernel<NT, TH2, GN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(nq::decode_stage1_kernel<NT, TH, GN>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    done[dev].store(true, std::memory_order_release);
+}
+
+template <int NT, int TH, int GN, bool PAIR>
+void set_stage2_attrs_once() {
+    static std::atomic<bool> done[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || done[dev].load(std::memory_order_acquire)) return;
+    cudaFuncSetAttribute(nq::decode_stage2_kernel<NT, TH, GN, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(kStage2SmemBudget));
     done[dev].store(true, std::memory_order_release);
 }
 
-// One launch of each stage for n projections that share x (n = 1: a single layer).
+// One launch of each stage for n projections that share x (n = 1: a single layer).  With
+// `pair` (n = 2, gate and up of equal d_out) stage 2 writes h = silu(gate x) * (up x) to ys[0].
 template <int NT, int GN>
 nq_status launch_decode_group_nt(const nq_lrb_layer* const* Ls, int n, const uint16_t* x, uint16_t* const* ys, int M,
                                  void* ws, const uint16_t* cot, float* grad, cudaStream_t stream, bool pdl,
-                                 float* t_only = nullptr) {
+                                 float* t_only = nullptr, bool pair = false) {
     // member l's share of the workspace (t's digit table, owner sums, shifts) follows the
     // earlier members'; with t_only (one layer), stage 1 alone runs and writes t in fp32 there
     char* base[nq::kMaxGroup];
@@ -929,6 +1051,7 @@ nq_status launch_decode_group_nt(const nq_lrb_layer* const* Ls, int n, const uin
                 q.tsh = reinterpret_cast<int*>(base[l] + tl[l].tsh);
             }
             q.nwp = static_cast<int>((L->r / 32 + 7) / 8 * 8);
+            q.prefetch = prefetch_v() ? 1 : 0;
             q.M = M;
             q.d_in = L->d_in;
             q.r = static_cast<int>(L->r);
@@ -944,15 +1067,16 @@ nq_status launch_decode_group_nt(const nq_lrb_layer* const* Ls, int n, const uin
         const bool wide = (NT <= 2) && sp.rows_per_slice >= 1024;
         const void* fn = wide ? reinterpret_cast<const void*>(nq::decode_stage1_kernel<NT, (NT <= 2 ? 512 : 256), GN>)
                               : reinterpret_cast<const void*>(nq::decode_stage1_kernel<NT, 256, GN>);
-        if (wide) set_attrs_once<NT, (NT <= 2 ? 512 : 256), 256, GN>();
-        else set_attrs_once<NT, 256, 256, GN>();
+        if (wide) set_stage1_attrs_once<NT, (NT <= 2 ? 512 : 256), GN>();
+        else set_stage1_attrs_once<NT, 256, GN>();
         if (nq_host::launch_ex(fn, dim3(acc, sp.CS), dim3(wide ? 512 : 256), sp.smem, stream, args, pdl, sp.CS) !=
             cudaSuccess)
             return NQ_ERR_LAUNCH;
     }
     if (t_only) return NQ_OK;
     {
-        // the SMs are shared among the members in proportion to their weight words
+        // the SMs are shared among the members in proportion to their weight words; a pair's
+        // blocks all work for both members
         const int sms = nq_host::sm_count();
         double wsum = 0.0;
         int mt[nq::kMaxGroup], nwp[nq::kMaxGroup];
@@ -963,11 +1087,10 @@ nq_status launch_decode_group_nt(const nq_lrb_layer* const* Ls, int n, const uin
         }
         nq::S2Group g{};
         g.n = n;
-        size_t smem = 0;
-        int min_per_cta = 1 << 30, acc = 0;
+        int acc = 0;
         for (int l = 0; l < n; ++l) {
             const nq_lrb_layer* L = Ls[l];
-            int gl = static_cast<int>(sms * (static_cast<double>(mt[l]) * nwp[l]) / wsum + 0.5);
+            int gl = pair ? sms : static_cast<int>(sms * (static_cast<double>(mt[l]) * nwp[l]) / wsum + 0.5);
             gl = std::max(1, std::min(gl, mt[l]));
             nq::S2Params& q = g.p[l];
             q.U = L->U;
@@ -987,27 +1110,53 @@ nq_status launch_decode_group_nt(const nq_lrb_layer* const* Ls, int n, const uin
             q.nwp = nwp[l];
             q.su = q.nwp + ((4 - q.nwp % 32) + 32) % 32;
             q.mt_total = mt[l];
-            const int per_cta = (q.mt_total + gl - 1) / gl;
-            min_per_cta = std::min(min_per_cta, per_cta);
-            const size_t bt_bytes = static_cast<size_t>(8) * q.nwp * NT * 8 * 4;
-            const size_t per_mt = static_cast<size_t>(16) * q.su * 4 + static_cast<size_t>(16) * NT * 8 * 4 + 16 * 4;
-            int chunk = per_cta;
-            if (bt_bytes + chunk * per_mt > kStage2SmemBudget)
-                chunk = static_cast<int>((kStage2SmemBudget - bt_bytes) / per_mt);
-            if (chunk < 1) return NQ_ERR_SHAPE;
-            q.chunk_mt = chunk;
-            const size_t smem2 = bt_bytes + chunk * per_mt;
-            smem = std::max(smem, smem2);
-            g.cta_off[l] = acc;
-            acc += gl;
+            g.cta_off[l] = pair ? 0 : acc;
+            if (!pair || l == 0) acc += gl;
         }
         g.cta_off[n] = acc;
+        if (pair) g.cta_off[1] = acc;
+        // M-tiles staged at a time: a block's whole share when it fits the shared memory
+        // (for a pair, both members' rows), else as many as fit
+        size_t smem = 0;
+        int min_per_cta = 1 << 30;
+        {
+            const int groups = pair ? 1 : n;
+            for (int gi = 0; gi < groups; ++gi) {
+                const int l0 = gi, l1 = pair ? n - 1 : gi;
+                const int G = g.cta_off[l0 + 1] - g.cta_off[l0];
+                const int per_cta = (mt[l0] + G - 1) / G;
+                min_per_cta = std::min(min_per_cta, per_cta);
+                size_t fixed = 0, per_mt = 0;
+                for (int l = l0; l <= l1; ++l) {
+                    const nq::S2Params& q = g.p[l];
+                    fixed += static_cast<size_t>(8) * q.nwp * NT * 8 * 4;
+                    per_mt += static_cast<size_t>(16) * q.su * 4 + static_cast<size_t>(16) * NT * 8 * 4 + 16 * 4;
+                }
+                int chunk = per_cta;
+                if (fixed + chunk * per_mt > kStage2SmemBudget)
+                    chunk = static_cast<int>((kStage2SmemBudget - std::min(fixed, kStage2SmemBudget)) / per_mt);
+                if (chunk < 1) return NQ_ERR_SHAPE;
+                for (int l = l0; l <= l1; ++l) g.p[l].chunk_mt = chunk;
+                smem = std::max(smem, fixed + chunk * per_mt);
+            }
+        }
         void* args[] = {&g};
         const bool wide = (NT == 1) && min_per_cta >= 6;
-        const void* fn = wide ? reinterpret_cast<const void*>(nq::decode_stage2_kernel<NT, (NT == 1 ? 512 : 256), GN>)
-                              : reinterpret_cast<const void*>(nq::decode_stage2_kernel<NT, 256, GN>);
-        if (wide) set_attrs_once<NT, 256, (NT == 1 ? 512 : 256), GN>();
-        else set_attrs_once<NT, 256, 256, GN>();
+        const void* fn = nullptr;
+        if constexpr (GN > 1) {
+            if (pair) {
+                fn = wide ? reinterpret_cast<const void*>(nq::decode_stage2_kernel<NT, (NT == 1 ? 512 : 256), GN, true>)
+                          : reinterpret_cast<const void*>(nq::decode_stage2_kernel<NT, 256, GN, true>);
+                if (wide) set_stage2_attrs_once<NT, (NT == 1 ? 512 : 256), GN, true>();
+                else set_stage2_attrs_once<NT, 256, GN, true>();
+            }
+        }
+        if (!fn) {
+            fn = wide ? reinterpret_cast<const void*>(nq::decode_stage2_kernel<NT, (NT == 1 ? 512 : 256), GN, false>)
+                      : reinterpret_cast<const void*>(nq::decode_stage2_kernel<NT, 256, GN, false>);
+            if (wide) set_stage2_attrs_once<NT, (NT == 1 ? 512 : 256), GN, false>();
+            else set_stage2_attrs_once<NT, 256, GN, false>();
+        }
         if (nq_host::launch_ex(fn, dim3(acc), dim3(wide ? 512 : 256), smem, stream, args, pdl, 1) != cudaSuccess)
             return NQ_ERR_LAUNCH;
     }
@@ -1053,8 +1202,8 @@ nq_status launch_stage1_pair_nt(const nq_lrb_layer* L0, const uint16_t* x0, floa
     const bool wide = (NT <= 2) && std::max(sp[0].rows_per_slice, sp[1].rows_per_slice) >= 1024;
     const void* fn = wide ? reinterpret_cast<const void*>(nq::decode_stage1_kernel<NT, (NT <= 2 ? 512 : 256), nq::kMaxGroup>)
                           : reinterpret_cast<const void*>(nq::decode_stage1_kernel<NT, 256, nq::kMaxGroup>);
-    if (wide) set_attrs_once<NT, (NT <= 2 ? 512 : 256), 256, nq::kMaxGroup>();
-    else set_attrs_once<NT, 256, 256, nq::kMaxGroup>();
+    if (wide) set_stage1_attrs_once<NT, (NT <= 2 ? 512 : 256), nq::kMaxGroup>();
+    else set_stage1_attrs_once<NT, 256, nq::kMaxGroup>();
     return nq_host::launch_ex(fn, dim3(acc, cs), dim3(wide ? 512 : 256), smem, stream, args, pdl, cs) == cudaSuccess
                ? NQ_OK
                : NQ_ERR_LAUNCH;
@@ -1094,6 +1243,24 @@ nq_status nq_launch_decode_group(const nq_lrb_layer* const* Ls, int n, const uin
         case 2: return launch_decode_group_nt<2, nq::kMaxGroup>(Ls, n, x, ys, m, ws, cot, grad, stream, pdl);
         default: return launch_decode_group_nt<3, nq::kMaxGroup>(Ls, n, x, ys, m, ws, cot, grad, stream, pdl);
     }
+}
+
+nq_status nq_launch_decode_gate_up(const nq_lrb_layer* gate, const nq_lrb_layer* up, const uint16_t* x, uint16_t* h,
+                                   int64_t M, void* ws, cudaStream_t stream, bool pdl) {
+    const nq_lrb_layer* Ls[2] = {gate, up};
+    uint16_t* ys[2] = {h, nullptr};
+    const int m = static_cast<int>(M);
+    switch (ntiles_for(M)) {
+        case 1: return launch_decode_group_nt<1, nq::kMaxGroup>(Ls, 2, x, ys, m, ws, nullptr, nullptr, stream, pdl, nullptr, true);
+        case 2: return launch_decode_group_nt<2, nq::kMaxGroup>(Ls, 2, x, ys, m, ws, nullptr, nullptr, stream, pdl, nullptr, true);
+        default: return launch_decode_group_nt<3, nq::kMaxGroup>(Ls, 2, x, ys, m, ws, nullptr, nullptr, stream, pdl, nullptr, true);
+    }
+}
+
+// Shared memory the paired stage 2 needs at the least: both digit tables and one M-tile of each.
+size_t nq_decode_pair_smem(int64_t r0, int64_t r1, int64_t M) {
+    const size_t a = nq_decode_stage2_smem(r0, M), b = nq_decode_stage2_smem(r1, M);
+    return (a > kStage2SmemBudget || b > kStage2SmemBudget || a + b > kStage2SmemBudget) ? kStage2SmemBudget + 1 : a + b;
 }
 
 nq_status nq_launch_decode(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y, int64_t M, void* ws,

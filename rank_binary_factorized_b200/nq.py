@@ -57,6 +57,11 @@ _lib.nq_from_latent_workspace_bytes.argtypes = [_i64, _i64, _i64, _i64, _i64]
 _lib.nq_lrb_from_latent.restype = ctypes.c_int
 _lib.nq_lrb_from_latent.argtypes = [_p, _i64, _p, _i64, _i64, _i64, _i64, _p, _i64, _p, _i64, _p, _p, _p, _p,
                                     ctypes.c_size_t, _p]
+_lib.nq_mlp_gate_up_workspace_bytes.restype = ctypes.c_size_t
+_lib.nq_mlp_gate_up_workspace_bytes.argtypes = [ctypes.POINTER(nq_lrb_layer), ctypes.POINTER(nq_lrb_layer), _i64]
+_lib.nq_mlp_gate_up.restype = ctypes.c_int
+_lib.nq_mlp_gate_up.argtypes = [ctypes.POINTER(nq_lrb_layer), ctypes.POINTER(nq_lrb_layer), _p, _p, _i64, _p,
+                                ctypes.c_size_t, _p]
 _lib.nq_group_workspace_bytes.restype = ctypes.c_size_t
 _lib.nq_group_workspace_bytes.argtypes = [ctypes.POINTER(ctypes.POINTER(nq_lrb_layer)), ctypes.c_int, _i64]
 _lib.nq_layer_forward_group.restype = ctypes.c_int
@@ -379,6 +384,32 @@ def layer_forward_group(layers, x: torch.Tensor, ys=None, ws=None, stream=None):
     _check("nq_layer_forward_group", _lib.nq_layer_forward_group(_layer_array(layers), len(layers), _ptr(x), yp, M,
                                                                  _ptr(ws), ws.numel(), _stream_ptr(stream)))
     return ys
+
+
+def mlp_gate_up_workspace_bytes(gate: Layer, up: Layer, M: int) -> int:
+    return int(_lib.nq_mlp_gate_up_workspace_bytes(ctypes.byref(gate.struct), ctypes.byref(up.struct), M))
+
+
+def mlp_gate_up(gate: Layer, up: Layer, x: torch.Tensor, h=None, ws=None, stream=None) -> torch.Tensor:
+    """h = bf16(silu(bf16(gate x)) * bf16(up x)) ([M][d_out] bf16), SiLU.mul fused into decode."""
+    dev = gate.U.device
+    if up.U.device != dev:
+        raise ValueError("gate, up: expected one device")
+    _need(x, "x", torch.bfloat16, device=dev)
+    M = int(x.shape[0]) if x.dim() == 2 else -1
+    _need(x, "x", torch.bfloat16, shape=(M, gate.d_in), device=dev)
+    if h is None:
+        h = torch.empty((M, gate.d_out), dtype=torch.bfloat16, device=dev)
+    _need(h, "h", torch.bfloat16, shape=(M, gate.d_out), device=dev)
+    if ws is None:
+        need = mlp_gate_up_workspace_bytes(gate, up, M)
+        if need == 0:
+            raise NQError("nq_mlp_gate_up_workspace_bytes", 2)
+        ws = torch.zeros(need, dtype=torch.uint8, device=dev)
+    _need_ws(ws, dev)
+    _check("nq_mlp_gate_up", _lib.nq_mlp_gate_up(ctypes.byref(gate.struct), ctypes.byref(up.struct), _ptr(x), _ptr(h),
+                                                 M, _ptr(ws), ws.numel(), _stream_ptr(stream)))
+    return h
 
 
 def silu_mul(g: torch.Tensor, u: torch.Tensor, h=None, stream=None) -> torch.Tensor:

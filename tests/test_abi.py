@@ -268,6 +268,39 @@ def test_noalloc_scratch_covers_every_accepted_decode_shape(nq):
         assert 0 < need <= NOALLOC_SCRATCH_BYTES, (M, lo, need)
 
 
+def test_mlp_gate_up_argument_errors(nq):
+    lib = nq.raw_lib()
+    fn = lib.nq_mlp_gate_up
+    fn.restype = ctypes.c_int
+    fn.argtypes = [ctypes.POINTER(nq.nq_lrb_layer), ctypes.POINTER(nq.nq_lrb_layer), ctypes.c_void_p, ctypes.c_void_p,
+                   ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    wsb = lib.nq_mlp_gate_up_workspace_bytes
+    wsb.restype = ctypes.c_size_t
+    wsb.argtypes = [ctypes.POINTER(nq.nq_lrb_layer), ctypes.POINTER(nq.nq_lrb_layer), ctypes.c_int64]
+    g, u = _layer(nq, d_out=64, d_in=96, r=64), _layer(nq, d_out=64, d_in=96, r=96)
+
+    def call(gl=g, ul=u, x=0x50000, h=0x60000, M=1, ws=0x70000, ws_bytes=1 << 30):
+        return fn(ctypes.byref(gl) if gl is not None else None, ctypes.byref(ul) if ul is not None else None,
+                  x, h, M, ws, ws_bytes, None)
+
+    assert call(gl=None) == NQ["NULL"]
+    assert call(ul=_layer(nq, d_out=64, d_in=97, r=64)) == NQ["SHAPE"]   # d_in differs
+    assert call(ul=_layer(nq, d_out=65, d_in=96, r=64)) == NQ["SHAPE"]   # d_out differs
+    assert call(M=0) == NQ["SHAPE"]
+    assert call(ul=_layer(nq, d_out=64, d_in=96, r=1 << 17)) == NQ["SHAPE"]  # too large for decode
+    assert call(x=0) == NQ["NULL"] and call(h=0) == NQ["NULL"] and call(ws=0) == NQ["NULL"]
+    assert call(x=0x50008) == NQ["ALIGN"]
+    assert call(ws_bytes=16) == NQ["WORKSPACE"]
+    assert wsb(ctypes.byref(g), ctypes.byref(_layer(nq, d_out=65, d_in=96, r=64)), 1) == 0
+    assert wsb(ctypes.byref(g), ctypes.byref(u), 0) == 0
+    for M in (1, 8, 9, 512):
+        need = wsb(ctypes.byref(g), ctypes.byref(u), M)
+        assert need >= 2 * M * 64 * 2  # room for the unfused gate and up outputs
+    import torch
+    if not torch.cuda.is_available():
+        assert call() == NQ["DEVICE"]
+
+
 def test_binding_refuses_host_tensors_before_any_call(nq):
     """The binding checks tensor arguments before their addresses reach the library (which
     reads device memory only): host tensors and wrong types raise, nothing is launched."""

@@ -78,3 +78,26 @@ def test_rows_of_very_different_magnitude_and_zero_input():
     y_ref, S = oracle.dense_packed(p.U, p.V, p.s1, p.s2, p.r, xb, rows=rows)
     check_tolerance(y[:, rows], y_ref, S, "row magnitudes 2^-40, 2^20")
     assert np.all(bf16_bits_to_f64(z) == 0.0)
+
+
+@pytest.mark.parametrize("d_out,d_in,r,M,align", [
+    (200, 64, 20224, 1, 4),     # largest rank at M = 1: a single chunk buffer
+    (3000, 96, 16384, 1, 4),    # two one-tile buffers, each block's chunks alternating in them
+    (60000, 64, 256, 1, 4),     # 26 M-tiles per block: the ring of six buffers wraps around
+    (60000, 64, 224, 2, 1),     # the same with rows of 7 words, copied in 4-byte pieces
+    (60001, 48, 320, 3, 1),     # 10 words (8-byte pieces), d_out odd: the last s1 half alone
+    (100, 64, 7168, 8, 4),      # largest rank at M = 8 (three B-table column tiles)
+])
+def test_stage2_ring_regimes(d_out, d_in, r, M, align):
+    """Stage 2 streams U through a ring of chunk buffers whose depth and chunk size depend on
+    r, M and d_out: these shapes cover a single buffer, buffers reused many times, and the
+    4- and 8-byte copy paths of unpadded strides, on sampled rows (first and last included)."""
+    need_gpu()
+    p = synth.make_projection("ring", d_out, d_in, r, seed=2300, key=d_out + r)
+    xb = synth.acts_bf16(synth.rng_for(2301, d_in, M), (M, d_in))
+    L = upload_projection(p, ld_align_words=align)
+    y = download_bf16_bits(nq().lrb_matvec(L, upload_bf16(xb)))
+    nq().sync_status()
+    rows = np.unique(np.concatenate([[0, 1, d_out - 2, d_out - 1], np.linspace(0, d_out - 1, 200).astype(np.int64)]))
+    y_ref, S = oracle.dense_packed(p.U, p.V, p.s1, p.s2, p.r, xb, rows=rows)
+    check_tolerance(y[:, rows], y_ref, S, "ring regime %r" % ((d_out, d_in, r, M, align),))

@@ -1,5 +1,6 @@
-"""SiLU-gated MLP block from three LRB projections (Llama-2 7B and 70B MLP shapes) and
-the nq_silu_mul kernel, against the CPU oracle."""
+"""SiLU-gated MLP block from three LRB projections (Llama-2 7B and 70B MLP shapes): the
+nq_silu_mul kernel and the fused gate/up call nq_mlp_gate_up, against the CPU oracle and, bit for
+bit, against the unfused calls they replace."""
 import numpy as np
 import pytest
 
@@ -28,23 +29,65 @@ def test_silu_mul_within_one_bf16_ulp():
     assert np.abs(gs - ws_).max() <= 1
 
 
+@pytest.mark.parametrize("fused", [False, True])
 @pytest.mark.parametrize("workload", ["mlp7b", "layer70b"])
-def test_mlp_block_decode(workload):
+def test_mlp_block_decode(workload, fused):
     """gate, up (shared x) -> h = silu(g) * u -> down, batch 1; down outputs vs the oracle's
-    MLP on a spread of rows, with S taken from the oracle's own h."""
+    MLP on a spread of rows, with S taken from the oracle's own h.  fused: h from
+    nq_mlp_gate_up instead of two projections and nq_silu_mul."""
     need_gpu()
     projs = {p.name: p for p in synth.make_workload(workload)}
     gate, up, down = projs["gate"], projs["up"], projs["down"]
     xb = synth.make_input(workload, gate.d_in, 1, key=31)
     Lg, Lu, Ld = (upload_projection(p) for p in (gate, up, down))
     x = upload_bf16(xb)
-    g = nq().layer_forward(Lg, x)
-    u = nq().layer_forward(Lu, x)
-    h = nq().silu_mul(g, u)
+    if fused:
+        h = nq().mlp_gate_up(Lg, Lu, x)
+    else:
+        g = nq().layer_forward(Lg, x)
+        u = nq().layer_forward(Lu, x)
+        h = nq().silu_mul(g, u)
     y = nq().layer_forward(Ld, h)
     nq().sync_status()
     # oracle: gate/up in the factored fp64 order, rounded to bf16, h, then the exact down
     rows = np.unique(np.concatenate([[0, down.d_out - 1], np.linspace(0, down.d_out - 1, 96).astype(np.int64)]))
     as_tuple = lambda p: (p.U, p.V, p.s1, p.s2, p.r)  # noqa: E731
     y_ref, S, _ = oracle.mlp(as_tuple(gate), as_tuple(up), as_tuple(down), xb, rows=rows, order="factored")
-    check_tolerance(download_bf16_bits(y)[:, rows], y_ref, S, workload + " MLP")
+    check_tolerance(download_bf16_bits(y)[:, rows], y_ref, S, workload + " MLP" + (" fused" if fused else ""))
+
+
+def _gate_up_pair(d_out, d_in, r_gate, r_up, seed):
+    gate = synth.make_projection("gate", d_out, d_in, r_gate, seed=seed, key=1)
+    up = synth.make_projection("up", d_out, d_in, r_up, seed=seed, key=2)
+    return gate, up
+
+
+@pytest.mark.parametrize("d_out,d_in,r_gate,r_up,M", [
+    (11008, 4096, 2368, 2368, 1),   # 7B MLP
+    (11008, 4096, 2368, 2368, 3),
+    (11008, 4096, 2368, 2368, 8),
+    (28672, 8192, 3520, 3520, 1),   # 70B MLP
+    (28672, 8192, 3520, 3520, 2),
+    (1000, 300, 96, 160, 1),        # ragged: d_out not a multiple of 16, different ranks
+    (1000, 300, 96, 160, 5),
+    (37, 64, 32, 64, 2),            # a single partial M-tile
+    (300, 64, 12000, 12000, 1),     # both stage-2 tables too large together: the unfused decode path
+    (2000, 512, 256, 320, 9),       # prefill path
+    (2000, 512, 256, 320, 64),
+])
+def test_mlp_gate_up_equals_unfused_calls(d_out, d_in, r_gate, r_up, M):
+    """nq_mlp_gate_up == nq_layer_forward_group({gate, up}) then nq_silu_mul, bit for bit, on
+    every element (the same integer sums and the same bf16 roundings of g and u)."""
+    need_gpu()
+    gate, up = _gate_up_pair(d_out, d_in, r_gate, r_up, seed=330 + M)
+    xb = synth.acts_bf16(synth.rng_for(331, d_in, M), (M, d_in))
+    Lg, Lu = upload_projection(gate), upload_projection(up)
+    x = upload_bf16(xb)
+    g, u = nq().layer_forward_group([Lg, Lu], x)
+    h_ref = nq().silu_mul(g, u)
+    h = nq().mlp_gate_up(Lg, Lu, x)
+    h2 = nq().mlp_gate_up(Lg, Lu, x)  # again, on the workspace the first call left behind
+    nq().sync_status()
+    want = download_bf16_bits(h_ref)
+    assert np.array_equal(download_bf16_bits(h), want)
+    assert np.array_equal(download_bf16_bits(h2), want)
