@@ -47,7 +47,7 @@ def parse_args():
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--headline-only", action="store_true", help="skip the other workloads")
     ap.add_argument("--only", default=None,
-                    help="run just these extra sections (comma list of attn7b_b8, mlp7b, layer70b, prefill, pack, "
+                    help="run just these extra sections (comma list of attn7b_b8, mlp7b, prefill, pack, "
                          "calib, signgrad, model70b) "
                          "after the headline; implies no CPU baseline")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU oracle sample budget")
@@ -350,6 +350,13 @@ def gpu_arm(args, rank, world, local):
     # the chain of layer_forward calls (captured once as a graph), D2H of the result
     result["e2e"] = e2e_measure(torch, nq, chain, stream, args, dist, world)
 
+    # ---- one public-API call on a cold L2: what the first layer of a decode step sees
+    result["latency_single_call"] = single_call_latency(torch, nq, chain, stream)
+    del chain
+
+    # ---- second headline: a Llama-2-70B decoder layer's projections at batch 1
+    result["headline_layer70b"] = headline_layer70b(torch, nq, stream, args, hbm_gbs, peak_src, local)
+
     if not args.headline_only or args.only is not None:
         result["extra"] = extras(torch, nq, stream, args, hbm_gbs, bf16_tf, bf16_tf_sus, peak_src)
 
@@ -357,6 +364,7 @@ def gpu_arm(args, rank, world, local):
         pass
     elif rank == 0 and world == 1:
         result["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+        result["parity_margins"] = parity_margins(torch, nq)
     elif rank == 0:
         result["cpu_baseline"] = None
 
@@ -364,6 +372,58 @@ def gpu_arm(args, rank, world, local):
         dist.barrier()
         dist.destroy_process_group()
     return result
+
+
+def single_call_latency(torch, nq, chain, stream, calls=50):
+    """One nq_layer_forward call of the headline layer through the Python binding, after a read
+    of 256 MB that leaves nothing of the layer in L2: host time from just before the call to
+    the end of a stream synchronise (argument checks, ctypes, launch, kernels, sync), and the
+    device time between CUDA events recorded around the call on its stream."""
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda").view(torch.int64)
+    flush.fill_(1)
+    y = torch.empty((chain.M, chain.layers[0].d_out), dtype=torch.bfloat16, device="cuda")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    host, dev = [], []
+    for i in range(calls + 3):
+        L = chain.layers[i % chain.n]
+        with torch.cuda.stream(stream):
+            torch.max(flush)  # reads 256 MB: L2 holds the flush buffer's clean lines afterwards
+        stream.synchronize()
+        t0 = time.perf_counter()
+        e0.record(stream)
+        nq.layer_forward(L, chain.x0, y, ws=chain.ws, stream=stream)
+        e1.record(stream)
+        stream.synchronize()
+        t1 = time.perf_counter()
+        if i >= 3:
+            host.append((t1 - t0) * 1e6)
+            dev.append(e0.elapsed_time(e1) * 1e3)
+    del flush
+    return {"host_us": round(statistics.median(host), 2), "device_us": round(statistics.median(dev), 2),
+            "calls": calls, "l2": "flushed before every call (a 256 MB read on the same stream)",
+            "note": "median of one nq_layer_forward call (7B attention projection, batch 1) through the Python "
+                    "binding: host time includes argument checks, the ctypes call, both launches and the "
+                    "synchronise"}
+
+
+def headline_layer70b(torch, nq, stream, args, hbm_gbs, peak_src, local):
+    """Batch-1 decode of a Llama-2-70B decoder layer's LRB projections (q, k, v grouped; o;
+    gate and up fused with SiLU.mul; down) over distinct layer instances (> 3x L2 per step)."""
+    sampler = ClockSampler(nvml_index(local))
+    r = _extra_block(torch, nq, stream, max(10, args.steps // 2), max(3, args.warmup), hbm_gbs, "layer70b", sampler)
+    alg = r["block_bytes"]
+    return {"workload": "Llama-2-70B decoder layer: q,o 8192x8192 r=2240; k,v 1024x8192 r=512; gate,up "
+                        "28672x8192 and down 8192x28672 r=3520; decode batch 1",
+            "value": r["us_per_block"], "unit": "us/layer", "steps": r["steps"], "layers_per_step": r["blocks_per_step"],
+            "grouped": r["grouped"],
+            "roofline": {"bound": "hbm", "kernel": "decode layer (8 stage kernels, PDL-chained)",
+                         "achieved": r["GB_s"], "peak": hbm_gbs,
+                         "peak_source": peak_src + " (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else peak_src,
+                         "unit": "GB/s", "frac": r["frac_hbm"], "traffic": profile_traffic("decode_layer70b_b1"),
+                         "algorithmic_bytes_per_launch": alg},
+            "clocks": sampler.summary(),
+            "l2": "no flush: %d distinct layers per step, %.0f MB > 3x L2" % (r["blocks_per_step"],
+                                                                            r["blocks_per_step"] * alg / 1e6)}
 
 
 def e2e_measure(torch, nq, chain, stream, args, dist, world):
@@ -400,9 +460,8 @@ def extras(torch, nq, stream, args, hbm_gbs, bf16_tf, bf16_tf_sus, peak_src):
     (_, d_out, d_in, r), = synth.WORKLOADS[HEADLINE]
     if on("attn7b_b8"):
         out.update(_extra_b8(torch, nq, stream, steps, warm, hbm_gbs, d_out, d_in, r))
-    for wl in ("mlp7b", "layer70b"):
-        if on(wl):
-            out[wl] = _extra_block(torch, nq, stream, steps, warm, hbm_gbs, wl)
+    if on("mlp7b"):
+        out["mlp7b"] = _extra_block(torch, nq, stream, steps, warm, hbm_gbs, "mlp7b")
     if on("prefill"):
         out["prefill70b_gate"] = _extra_prefill(torch, nq, stream, steps, bf16_tf)
     if on("pack"):
@@ -428,7 +487,7 @@ def _extra_b8(torch, nq, stream, steps, warm, hbm_gbs, d_out, d_in, r):
                           "frac_hbm": round(lb / us / 1e3 / hbm_gbs, 4)}}
 
 
-def _extra_block(torch, nq, stream, steps, warm, hbm_gbs, wl):
+def _extra_block(torch, nq, stream, steps, warm, hbm_gbs, wl, sampler=None):
     """A 7B MLP block or a 70B decoder layer's projections (+ SiLU.mul), decode batch 1."""
     shapes = synth.WORKLOADS[wl]
     block_bytes = sum(decode_bytes(do, di, r, 1) for (_, do, di, r) in shapes)
@@ -467,11 +526,11 @@ def _extra_block(torch, nq, stream, steps, warm, hbm_gbs, wl):
             xx = bufs["down"]
 
     g = graph_of(torch, run_blocks, stream)
-    ms = timed_replays(torch, g, stream, steps, warm)
+    ms = timed_replays(torch, g, stream, steps, warm, sampler=sampler)
     us = ms * 1e3 / (steps * reps)
     del g, blocks
     return {"us_per_block": round(us, 3), "block_bytes": block_bytes, "GB_s": round(block_bytes / us / 1e3, 1),
-            "frac_hbm": round(block_bytes / us / 1e3 / hbm_gbs, 4), "blocks_per_step": reps,
+            "frac_hbm": round(block_bytes / us / 1e3 / hbm_gbs, 4), "blocks_per_step": reps, "steps": steps,
             "block": "+".join(n for (n, *_r) in shapes) + " + silu_mul",
             "grouped": ("q,k,v one nq_layer_forward_group call (shared input); " if shapes[0][0] == "q" else "")
                        + "gate,up and SiLU.mul one nq_mlp_gate_up call"}
@@ -488,8 +547,8 @@ def _extra_prefill(torch, nq, stream, steps, bf16_tf):
         y = torch.empty((M, do), dtype=torch.bfloat16, device="cuda")
         ws = L.workspace(M)
         g = graph_of(torch, lambda: nq.lrb_matmul(L, x, y, ws=ws, stream=stream), stream)
-        psteps = 3 if M >= 512 else steps
-        ms = timed_replays(torch, g, stream, psteps, 2)
+        psteps = max(20, steps)
+        ms = timed_replays(torch, g, stream, psteps, 3)
         us = ms * 1e3 / psteps
         flops = 2.0 * M * r * (di + do)
         pre["M%d" % M] = {"us": round(us, 2), "TFLOP_s": round(flops / us / 1e6, 2),
@@ -585,8 +644,8 @@ def _extra_sign_grads(torch, nq, stream, steps, warm, hbm_gbs, bf16_tf):
         ybar = torch.zeros((M, do), dtype=torch.bfloat16, device="cuda").normal_()
         ws = torch.empty(nq.sign_grads_workspace_bytes(L70, M), dtype=torch.uint8, device="cuda")
         g = graph_of(torch, lambda: nq.lrb_sign_grads(L70, x, ybar, gU=gU, gV=gV, ws=ws, stream=stream), stream)
-        ms = timed_replays(torch, g, stream, 3, 2)
-        us = ms * 1e3 / 3
+        ms = timed_replays(torch, g, stream, 20, 3)
+        us = ms * 1e3 / 20
         flops = 4.0 * M * r * (di + do)  # two GEMM 1 passes and the two outer products
         wbytes = 4 * r * (do + di)
         out["sign_grads_prefill70b_gate_M%d" % M] = {
@@ -679,6 +738,37 @@ def cpu_baseline(budget_s: float):
     return {"value": round(us, 1), "unit": "us/layer", "cores": 1, "kind": "oracle",
             "sample": "%d forwards of the factored fp64 oracle (s1 (.) U (V^T (s2 (.) x))) on one 4096x4096 r=2048 "
                       "layer at batch 1, single thread, median" % len(times)}
+
+
+def parity_margins(torch, nq, nrows=64):
+    """Parity headroom per configuration on sampled rows (the first, the last and a spread): the
+    CPU oracle's exact forward against the GPU's bf16 output, as the largest |err| / bound for
+    the stated bound 2e-3 S + 1e-5 (S = sum of |terms|) and for that bound plus half a bf16 unit
+    of y (the rounding of the output itself).  Runs in the CPU-baseline leg (rank 0, N = 1)."""
+    import oracle
+    cases = [("attn7b", 0, 1), ("attn7b", 0, 8), ("mlp7b", 0, 1), ("layer70b", 4, 1), ("layer70b", 6, 1),
+             ("prefill70b", 0, 64)]
+    out = {}
+    for wl, idx, M in cases:
+        p = synth.make_workload(wl)[idx]
+        xb = synth.make_input(wl, p.d_in, M, key=4242)
+        L = nq.Layer.from_host(p.U, p.V, p.s1, p.s2, p.r)
+        x = torch.from_numpy(np.ascontiguousarray(xb).view(np.int16)).cuda().view(torch.bfloat16)
+        y = nq.layer_forward(L, x)
+        nq.sync_status()
+        yb = y.view(torch.int16).cpu().numpy().view(np.uint16)
+        rows = np.unique(np.concatenate([[0, p.d_out - 1], np.linspace(0, p.d_out - 1, nrows).astype(np.int64)]))
+        y_ref, S = oracle.dense_packed(p.U, p.V, p.s1, p.s2, p.r, xb, rows=rows)
+        got = (yb[:, rows].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        err = np.abs(got - y_ref)
+        bound = 2e-3 * S + 1e-5
+        _, e = np.frexp(np.abs(y_ref))
+        half_ulp = np.ldexp(0.5, np.maximum(np.where(y_ref == 0, -125, e), -125) - 8)
+        out["%s/%s M=%d" % (wl, p.name, M)] = {"strict": round(float((err / bound).max()), 4),
+                                                "with_bf16_rounding": round(float((err / (bound + half_ulp)).max()), 4),
+                                                "rows": int(rows.size)}
+        del L, x, y
+    return out
 
 
 def reference_arm(args):
