@@ -46,6 +46,9 @@ def parse_args():
     ap.add_argument("--impl", choices=["nq", "reference"], default="nq")
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--headline-only", action="store_true", help="skip the other workloads")
+    ap.add_argument("--layer70b-only", action="store_true",
+                    help="run only the 70B decoder-layer section (for profiling: its first launches are the "
+                         "first layer's kernels); prints its figures alone")
     ap.add_argument("--only", default=None,
                     help="run just these extra sections (comma list of attn7b_b8, mlp7b, prefill, pack, "
                          "calib, signgrad, model70b) "
@@ -291,6 +294,11 @@ def gpu_arm(args, rank, world, local):
         dist = tdist
     hbm_gbs, bf16_tf, bf16_tf_sus, peak_src = measured_peaks()
     stream = torch.cuda.Stream()
+
+    if args.layer70b_only:
+        return {"metric": METRIC, "value": None, "unit": "us/layer", "n_gpus": world,
+                "note": "70B decoder-layer section alone (profiling run); no headline",
+                "headline_layer70b": headline_layer70b(torch, nq, stream, args, hbm_gbs, peak_src, local)}
 
     # ---- headline: 7B attention projection, batch M, chain of distinct instances
     (_, d_out, d_in, r), = synth.WORKLOADS[HEADLINE]
