@@ -127,10 +127,14 @@ NQ_API nq_status nq_lrb_matvec(const nq_lrb_layer* L, const uint16_t* x, uint16_
 
 /*
  * nq_lrb_matmul -- prefill path on the tensor cores (tcgen05), any M >= 1 (tuned for
- * M >= 64).  Same operation as nq_lrb_matvec.  The activations are scaled by s2 and
- * rounded to fp16, the packed signs are expanded to fp16 +-1 on chip, both products
- * accumulate in fp32 (TMEM), the intermediate t is rounded to fp16, and y is rounded to
- * bf16.  Finite results require |x_j s2_j| and |t_k| below the fp16 range (65504).
+ * M >= 64).  Same operation as nq_lrb_matvec.  The activations are scaled by s2 and by one
+ * power of two 2^-e_m per row m, chosen so that sum_j |2^-e_m x_mj s2_j| <= 2^14, and rounded
+ * to fp16; the packed signs are expanded to fp16 +-1 on chip; both products accumulate in fp32
+ * (TMEM); the intermediate t (|t| <= 2^14 by the choice of e_m) is rounded to fp16; y is scaled
+ * back by 2^e_m and s1 and rounded to bf16.  So no finite bf16 input overflows fp16 on the way,
+ * rows of very small values keep fp16's full precision, and y is finite whenever its value
+ * lies in the bf16 range.  The powers of two are exact: rows that stay inside fp16's normal
+ * range either way give the same bits as without them.  The workspace holds e_m.
  */
 NQ_API nq_status nq_lrb_matmul(const nq_lrb_layer* L, const uint16_t* x, uint16_t* y, int64_t M, void* ws,
                         size_t ws_bytes, void* stream);
@@ -205,7 +209,9 @@ NQ_API nq_status nq_lrb_scale_grads(const nq_lrb_layer* L, const uint16_t* x, co
  *   M <= NQ_MATVEC_MAX_M: t and u from the decode stage 1 (exact integer sums of the 23-bit
  *   quantised activations, fp32), the sum over m in fp32 on the CUDA cores.  Larger M: t and u
  *   from the tensor-core GEMM 1 (fp16 operands s2 . x and s1 . ybar, fp16 t, u), the sum over
- *   m on the tensor cores (fp16 operands, fp32 accumulation).
+ *   m on the tensor cores (fp16 operands, fp32 accumulation).  That sum runs over the rows,
+ *   so they share one scale: finite results here need |x_j s2_j|, |ybar_i s1_i|, |t_k| and
+ *   |u_k| below the fp16 range (65504).
  *   ws: nq_sign_grads_workspace_bytes(L, M) bytes (0 for an invalid layer or M < 1).
  */
 NQ_API size_t nq_sign_grads_workspace_bytes(const nq_lrb_layer* L, int64_t M);

@@ -5,9 +5,11 @@
 // The factorisation equation of section 2 is evaluated right to left as two dense products
 // whose weight operand is +-1:
 //
-//   Z = fp16(x (.) s2)                      [M][d_in]   (scale_convert_kernel)
+//   Z = fp16(2^-e x (.) s2)                 [M][d_in]   (scale_convert_rows_kernel)
 //   T = fp16(Z V)        V in {+-1}^{d_in x r}          (umma kernel, mode V)
-//   Y = bf16(s1 (.) (T U^T))  U in {+-1}^{d_out x r}    (umma kernel, mode U)
+//   Y = bf16(2^e s1 (.) (T U^T))  U in {+-1}^{d_out x r} (umma kernel, mode U)
+// with one power of two e per token that keeps Z and T inside fp16's range (the sign-gradient
+// path, which sums over tokens, uses e = 0: scale_convert_kernel).
 //
 // Both products run in one persistent warp-specialised kernel, D[w][n] = sum_K A[w][K] B[n][K]:
 //   * A (the weights, MMA M = 128 rows of U, or of V^T) is expanded on chip from the packed
@@ -59,6 +61,7 @@ struct PrefillArgs {
     void* out;             // mode V: T fp16 [M][ldo]; mode U: Y bf16 [M][ldo]
     int64_t ldo;
     const uint16_t* s1;    // mode U
+    const int* row_exp;    // mode U: token m's activations were scaled by 2^-row_exp[m] (none if null)
     unsigned int* err;
     int bits_tma;          // packed signs arrive by TMA (row stride a multiple of 16 bytes)
     // gradient mode (mode U, gpart != nullptr): no Y; for every token tile tn and row w,
@@ -395,6 +398,17 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             float* part = (ksplit > 1) ? args.partial + static_cast<int64_t>(u % ksplit) * args.M * args.ldo : nullptr;
             const int acc = tc_count & 1;
             const uint32_t aph = (tc_count >> 1) & 1u;
+            // does any token of this tile carry a power of two?  (loads issued before the wait
+            // for the accumulator, so their latency hides behind it; almost always none)
+            bool tile_scaled = false;
+            if (MODE == kModeU && args.row_exp != nullptr) {
+#pragma unroll
+                for (int c = 0; c < 256; c += 32) {
+                    const int64_t tk = static_cast<int64_t>(tn) * tile_n + c + lane;
+                    if (c + lane < tile_n && tk < args.M && args.row_exp[tk] != 0) tile_scaled = true;
+                }
+                tile_scaled = __any_sync(__activemask(), tile_scaled);
+            }
             if (!(ok = tc::mbar_wait(acc_full(acc), aph, err))) break;
             tc::tc_fence_after();
             const int64_t wrow = static_cast<int64_t>(tw) * kTileW + rl;
@@ -406,22 +420,50 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             for (int c0 = 0; c0 < tile_n; c0 += 32) {
                 uint32_t v[32];
                 tc::tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * 256 + c0, v);
+                // the exponents of these 32 tokens: lane l loads token c0 + l's; almost always
+                // all zero (rows inside fp16's range keep e = 0), and then the plain loop runs
+                int el = 0;
+                if (tile_scaled) {
+                    const int64_t tk = static_cast<int64_t>(tn) * tile_n + c0 + lane;
+                    el = (c0 + lane < tile_n && tk < args.M) ? args.row_exp[tk] : 0;
+                }
+                const bool scaled = tile_scaled && __any_sync(__activemask(), el != 0);
                 tc::tmem_wait_ld();
-                if (row_ok) {
+                if (!scaled) {
+                    if (row_ok) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const int64_t tok = static_cast<int64_t>(tn) * tile_n + c0 + j;
+                            if (c0 + j < tile_n && tok < args.M) {
+                                const float f = __uint_as_float(v[j]);
+                                if (grad) {
+                                    g += static_cast<double>(bf16_bits_to_float(args.cot[tok * args.ldcot + wrow])) * f;
+                                } else if (MODE == kModeU) {
+                                    static_cast<uint16_t*>(args.out)[tok * args.ldo + wrow] = float_to_bf16_bits(scale * f);
+                                } else if (part) {
+                                    part[tok * args.ldo + wrow] = f;
+                                } else {
+                                    static_cast<uint16_t*>(args.out)[tok * args.ldo + wrow] =
+                                        __half_as_ushort(__float2half_rn(f));
+                                }
+                            }
+                        }
+                    }
+                } else if (MODE == kModeU) {
+                    // token j's values times 2^e_j (exact powers of two), e_j from lane j
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
+                        const int e = __shfl_sync(__activemask(), el, j);
                         const int64_t tok = static_cast<int64_t>(tn) * tile_n + c0 + j;
-                        if (c0 + j < tile_n && tok < args.M) {
+                        if (row_ok && c0 + j < tile_n && tok < args.M) {
                             const float f = __uint_as_float(v[j]);
                             if (grad) {
-                                g += static_cast<double>(bf16_bits_to_float(args.cot[tok * args.ldcot + wrow])) * f;
-                            } else if (MODE == kModeU) {
-                                static_cast<uint16_t*>(args.out)[tok * args.ldo + wrow] = float_to_bf16_bits(scale * f);
-                            } else if (part) {
-                                part[tok * args.ldo + wrow] = f;
+                                g += static_cast<double>(bf16_bits_to_float(args.cot[tok * args.ldcot + wrow])) *
+                                     (static_cast<double>(f) * __longlong_as_double(static_cast<long long>(1023 + e) << 52));
                             } else {
-                                static_cast<uint16_t*>(args.out)[tok * args.ldo + wrow] =
-                                    __half_as_ushort(__float2half_rn(f));
+                                const float sf = scale * f;
+                                const float o = (e >= -126 && e <= 127) ? sf * __int_as_float((e + 127) << 23) : ldexpf(sf, e);
+                                static_cast<uint16_t*>(args.out)[tok * args.ldo + wrow] = float_to_bf16_bits(o);
                             }
                         }
                     }
@@ -501,6 +543,179 @@ __global__ void __launch_bounds__(256) scale_convert_kernel(const uint16_t* __re
     }
 }
 
+// 2^k as a float for -126 <= k <= 127
+__device__ __forceinline__ float pow2f(int k) { return __int_as_float((k + 127) << 23); }
+
+// Row m of Z = fp16(2^-e_m x[m] (.) s2), with one power of two e_m per row: e_m = 0 while the row
+// fits fp16 (L = sum_j |x_j s2_j| <= 2^14, and L / d_in >= 2^-10 so that typical values sit well
+// inside fp16's normal range), else chosen so that 2^-e_m L <= 2^14.  Then every |Z| and every
+// |T[m][k]| = |sum_j Z[m][j] V[j][k]| stays below fp16's largest value (65504) for any finite
+// bf16 x and fp16 s2, and rows of small values keep their significant bits instead of falling
+// into fp16's subnormals.  e_m goes to row_exp[m]; the epilogue of GEMM 2 multiplies by 2^e_m.
+// Scaling by powers of two commutes with the roundings (bf16 x times fp16 s2 is exact in fp32;
+// fp16 and fp32 round the same relative way wherever both values are normal).
+// One block per row.  Pass 1 takes the largest |x| and L in fp32 (fixed order: per thread,
+// then a tree).  Where that sum overflowed or fell below 2^-100 (rows of extreme magnitude), a
+// second pass takes it again after scaling x by 2^-ex (2^ex <= max |x| < 2^(ex + 1)); values
+// more than 2^126 below the row's largest flush to zero there, far below fp16's resolution of
+// the row anyway.  The last pass converts.  Rows of up to 2048 kRowVecs values stay in
+// registers; longer ones are read again from L2 for each pass.
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+__device__ __forceinline__ float f16_lo(uint32_t h) { return f16_bits_to_float(static_cast<uint16_t>(h & 0xFFFFu)); }
+__device__ __forceinline__ float f16_hi(uint32_t h) { return f16_bits_to_float(static_cast<uint16_t>(h >> 16)); }
+
+template <int kRowVecs>
+__global__ void __launch_bounds__(256) scale_convert_rows_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ s2,
+                                                                uint16_t* __restrict__ z, int* __restrict__ row_exp,
+                                                                int64_t M, int64_t d_in, int64_t ldz) {
+    constexpr int kRowChunk = 256 * kRowVecs;  // vectors (of 8 values) per chunk
+    pdl_wait();
+    __shared__ unsigned int s_max[8];
+    __shared__ float s_sum[8];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const bool vec = (d_in & 7) == 0;  // rows of whole 16-byte vectors (else one value at a time)
+    const int64_t nvec = vec ? d_in / 8 : 0;
+    const int64_t nchunk = vec ? (nvec + kRowChunk - 1) / kRowChunk : 0;
+    const int lg = 64 - __clzll(static_cast<unsigned long long>(d_in - 1));  // ceil(log2 d_in)
+    for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
+        const uint16_t* xr = x + m * d_in;
+        uint16_t* zr = z + m * ldz;
+        uint4 xv[kRowVecs], sv[kRowVecs];
+        auto load = [&](int64_t c) {
+#pragma unroll
+            for (int u = 0; u < kRowVecs; ++u) {
+                const int64_t v = c * kRowChunk + u * 256 + tid;
+                if (v < nvec) {
+                    xv[u] = __ldg(reinterpret_cast<const uint4*>(xr) + v);
+                    sv[u] = __ldg(reinterpret_cast<const uint4*>(s2) + v);
+                } else {
+                    xv[u] = make_uint4(0u, 0u, 0u, 0u);
+                    sv[u] = make_uint4(0u, 0u, 0u, 0u);
+                }
+            }
+        };
+        // ---- pass 1: the largest |x| (as bf16 bits, ordered like the magnitudes) and L
+        unsigned int mx = 0u;
+        float l1 = 0.0f;
+        if (vec) {
+            for (int64_t c = 0; c < nchunk; ++c) {
+                load(c);
+#pragma unroll
+                for (int u = 0; u < kRowVecs; ++u) {
+                    const uint32_t w[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
+                    const uint32_t h[4] = {sv[u].x, sv[u].y, sv[u].z, sv[u].w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        mx = max(mx, max(w[q] & 0x7FFFu, (w[q] >> 16) & 0x7FFFu));
+                        l1 += fabsf(bf16_lo(w[q]) * f16_lo(h[q])) + fabsf(bf16_hi(w[q]) * f16_hi(h[q]));
+                    }
+                }
+            }
+        } else {
+            for (int64_t j = tid; j < d_in; j += 256) {
+                mx = max(mx, static_cast<unsigned int>(xr[j] & 0x7FFFu));
+                l1 += fabsf(bf16_bits_to_float(xr[j]) * f16_bits_to_float(s2[j]));
+            }
+        }
+        mx = __reduce_max_sync(0xffffffffu, mx);
+        for (int off = 16; off > 0; off >>= 1) l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+        if (lane == 0) {
+            s_max[warp] = mx;
+            s_sum[warp] = l1;
+        }
+        __syncthreads();
+        mx = 0u;
+        l1 = 0.0f;
+        for (int w = 0; w < 8; ++w) {
+            mx = max(mx, s_max[w]);
+            l1 += s_sum[w];
+        }
+        __syncthreads();  // s_max and s_sum are written again below or by the next row
+        const bool finite_row = mx != 0u && mx < 0x7F80u;  // neither all zero nor inf/NaN
+        // the conversion multiplies x by f1 f2, then by s2, then by fs (exact powers of two)
+        float f1 = 1.0f, f2 = 1.0f, fs = 1.0f;
+        int e = 0;
+        if (finite_row && l1 > 0.0f) {
+            if (l1 <= 3.0e38f && l1 >= 0x1p-100f) {
+                int c = 0;
+                frexpf(l1, &c);  // L < 2^c
+                const bool fits = (c <= 14) && (c - 1 - lg >= -10);
+                if (!fits) {
+                    e = c - 14;  // |e| <= 114
+                    fs = pow2f(-e);
+                }
+            } else {
+                // ---- pass 2 (rows of extreme magnitude): L after scaling x by 2^-ex
+                const int ex = (mx >= 0x80u) ? static_cast<int>(mx >> 7) - 127 : (31 - __clz(mx)) - 133;
+                f1 = pow2f((-ex) / 2);
+                f2 = pow2f(-ex - (-ex) / 2);  // 2^-ex = f1 f2, each a normal float
+                float l2 = 0.0f;
+                if (vec) {
+                    for (int64_t c = 0; c < nchunk; ++c) {
+                        if (nchunk > 1) load(c);
+#pragma unroll
+                        for (int u = 0; u < kRowVecs; ++u) {
+                            const uint32_t w[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
+                            const uint32_t h[4] = {sv[u].x, sv[u].y, sv[u].z, sv[u].w};
+#pragma unroll
+                            for (int q = 0; q < 4; ++q)
+                                l2 += fabsf(bf16_lo(w[q]) * f1 * f2 * f16_lo(h[q])) + fabsf(bf16_hi(w[q]) * f1 * f2 * f16_hi(h[q]));
+                        }
+                    }
+                } else {
+                    for (int64_t j = tid; j < d_in; j += 256)
+                        l2 += fabsf(bf16_bits_to_float(xr[j]) * f1 * f2 * f16_bits_to_float(s2[j]));
+                }
+                for (int off = 16; off > 0; off >>= 1) l2 += __shfl_xor_sync(0xffffffffu, l2, off);
+                if (lane == 0) s_sum[warp] = l2;
+                __syncthreads();
+                l2 = 0.0f;
+                for (int w = 0; w < 8; ++w) l2 += s_sum[w];
+                __syncthreads();
+                if (l2 > 0.0f) {
+                    int c = 0;
+                    frexpf(l2, &c);  // l2 < 2^c <= 2^38 (d_in values of |2^-ex x| < 2, |s2| <= 65504)
+                    const int sh = min(14 - c, 127);  // a smaller sh keeps the bound (sums below 2^-113 only)
+                    e = ex - sh;
+                    fs = pow2f(sh);
+                } else {
+                    f1 = f2 = 1.0f;  // nothing survived the scaling: the row converts as it is
+                }
+            }
+        }
+        if (tid == 0) row_exp[m] = e;
+        // ---- conversion: z = fp16(((x f1 f2) s2) fs)
+        if (vec) {
+            for (int64_t c = 0; c < nchunk; ++c) {
+                if (nchunk > 1) load(c);
+#pragma unroll
+                for (int u = 0; u < kRowVecs; ++u) {
+                    const int64_t v = c * kRowChunk + u * 256 + tid;
+                    if (v < nvec) {
+                        const uint32_t w[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
+                        const uint32_t h[4] = {sv[u].x, sv[u].y, sv[u].z, sv[u].w};
+                        uint32_t o[4];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const float a = (bf16_lo(w[q]) * f1 * f2) * f16_lo(h[q]) * fs;
+                            const float b = (bf16_hi(w[q]) * f1 * f2) * f16_hi(h[q]) * fs;
+                            o[q] = static_cast<uint32_t>(__half_as_ushort(__float2half_rn(a))) |
+                                   (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(b))) << 16);
+                        }
+                        reinterpret_cast<uint4*>(zr)[v] = make_uint4(o[0], o[1], o[2], o[3]);
+                    }
+                }
+            }
+        } else {
+            for (int64_t j = tid; j < d_in; j += 256) {
+                const float v = (bf16_bits_to_float(xr[j]) * f1 * f2) * f16_bits_to_float(s2[j]) * fs;
+                zr[j] = __half_as_ushort(__float2half_rn(v));
+            }
+        }
+    }
+}
+
 // T[m][k] = fp16( sum over splits s = 0 .. S-1, in order, of partial[s][m][k] ) for k < r;
 // four k per thread (r % 32 == 0 and ldt % 8 == 0: 16-byte loads, 8-byte stores).
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restrict__ partial, int S, int64_t M,
@@ -554,7 +769,7 @@ struct PrefillPlan {
     int64_t ldz, ldt;
     int tile_n1, tile_n2;  // token tiles of GEMM 1 and GEMM 2
     int ksplit1;           // K splits of GEMM 1 (when its packed signs arrive by TMA)
-    size_t off_z, off_t, off_p, off_g, total;
+    size_t off_z, off_t, off_p, off_g, off_e, total;
 };
 
 // K splits for a GEMM of `tiles` output tiles over nkb k blocks: the fewest k-block steps on
@@ -613,7 +828,8 @@ PrefillPlan plan_prefill(const nq_lrb_layer* L, int64_t M) {
     p.off_g = p.off_p + (p.ksplit1 > 1 ? align256(static_cast<size_t>(p.ksplit1) * M * p.ldt * 4) : 0);
     // gradient mode: fp64 partial per (token tile of GEMM 2, row)
     const int64_t n_tn2 = (M + p.tile_n2 - 1) / p.tile_n2;
-    p.total = p.off_g + align256(static_cast<size_t>(n_tn2 * L->d_out) * sizeof(double));
+    p.off_e = p.off_g + align256(static_cast<size_t>(n_tn2 * L->d_out) * sizeof(double));
+    p.total = p.off_e + align256(static_cast<size_t>(M) * sizeof(int));  // per-token exponents
     return p;
 }
 
@@ -723,11 +939,21 @@ namespace {
 
 // Z = fp16(x . s2) and T = fp16(Z V) of layer L into the workspace ws, laid out by plan p.
 nq_status launch_stage1(const nq_lrb_layer* L, const uint16_t* x, int64_t M, void* ws, const PrefillPlan& p,
-                        cudaStream_t stream, bool pdl) {
+                        cudaStream_t stream, bool pdl, int* row_exp = nullptr) {
     uint16_t* z = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + p.off_z);
     uint16_t* t = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + p.off_t);
     unsigned int* err = nq_host::error_word();
-    {  // Z = fp16(x * s2)
+    if (row_exp) {  // Z = fp16(2^-e_m x * s2), one exponent per token
+        const unsigned blocks = static_cast<unsigned>(std::min<int64_t>(M, 65535));
+        const uint16_t* s2 = L->s2;
+        int64_t d_in = L->d_in, ldz = p.ldz;
+        void* args[] = {&x, &s2, &z, &row_exp, &M, &d_in, &ldz};
+        // four vectors per thread: rows of up to 8192 values stay in registers, longer ones are
+        // read again (from L2) by the later passes; a small footprint keeps several blocks per SM
+        const void* fn = reinterpret_cast<const void*>(nq::scale_convert_rows_kernel<4>);
+        if (nq_host::launch_pdl(fn, dim3(blocks), dim3(256), 0, stream, args, pdl) != cudaSuccess)
+            return NQ_ERR_LAUNCH;
+    } else {  // Z = fp16(x * s2)
         // four vectors per thread once the job has enough of them for 2 blocks per SM at that
         // depth; one otherwise (more, smaller blocks for few rows)
         const int64_t per_row = (L->d_in % 8 == 0) ? L->d_in / 8 : L->d_in;  // work items per row
@@ -806,7 +1032,8 @@ nq_status nq_launch_prefill(const nq_lrb_layer* L, const uint16_t* x, uint16_t* 
     const PrefillPlan p = plan_prefill(L, M);
     uint16_t* t = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + p.off_t);
     unsigned int* err = nq_host::error_word();
-    nq_status st0 = launch_stage1(L, x, M, ws, p, stream, pdl);
+    int* row_exp = reinterpret_cast<int*>(static_cast<char*>(ws) + p.off_e);
+    nq_status st0 = launch_stage1(L, x, M, ws, p, stream, pdl, row_exp);
     if (st0 != NQ_OK) return st0;
     {  // Y = bf16(s1 * (T U^T)): weights = U (M-extent d_out, K = r), B = T
         const int tile_n = p.tile_n2;
@@ -826,6 +1053,7 @@ nq_status nq_launch_prefill(const nq_lrb_layer* L, const uint16_t* x, uint16_t* 
         a.out = y;
         a.ldo = L->d_out;
         a.s1 = L->s1;
+        a.row_exp = row_exp;
         a.err = err;
         double* gpart = reinterpret_cast<double*>(static_cast<char*>(ws) + p.off_g);
         if (grad) {

@@ -15,7 +15,8 @@ import torch
 
 import oracle
 from rank_binary_factorized_b200 import synth
-from tests.gpu_util import (check_tolerance, download_bf16_bits, need_gpu, nq, upload_bf16, upload_projection)
+from tests.gpu_util import (ABS, REL, bf16_bits_to_f64, check_tolerance, download_bf16_bits, half_ulp_bf16, need_gpu, nq,
+                            upload_bf16, upload_projection)
 
 pytestmark = pytest.mark.gpu
 
@@ -140,3 +141,77 @@ def test_one_workspace_shared_by_decode_and_prefill():
     for xb, y in outs:
         y_ref, S = oracle.dense_packed(p.U, p.V, p.s1, p.s2, p.r, xb)
         check_tolerance(download_bf16_bits(y), y_ref, S, "shared workspace M=%d" % xb.shape[0])
+
+
+def _rows_scaled(xb, exps):
+    """bf16 rows multiplied by 2^e (exact; e = None gives an all-zero row)."""
+    xf = (np.asarray(xb, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    for m, e in enumerate(exps):
+        xf[m] = 0.0 if e is None else np.ldexp(xf[m], e)
+    return oracle.round_bf16(xf)
+
+
+@pytest.mark.parametrize("d_out,d_in,r", [(300, 2048, 256), (129, 1000, 96)])
+def test_rows_beyond_and_below_fp16_range(d_out, d_in, r):
+    """Each row gets its own power of two before the fp16 conversion: rows scaled by 2^-120 up to
+    2^124 (|x s2| far above 65504, sums of |x s2| beyond fp32's range, and values far below fp16's
+    smallest normal) and an all-zero row, in one call, each within its own tolerance and finite;
+    the zero row is zero."""
+    need_gpu()
+    p = synth.make_projection("range", d_out, d_in, r, seed=2400, key=d_out)
+    exps = [-120, -30, 0, 20, 80, None, 40, -60, 124, 10]  # M = 10 > 8: the tensor-core path
+    xb = _rows_scaled(synth.acts_bf16(synth.rng_for(2401, d_in), (len(exps), d_in)), exps)
+    y = gpu_matmul(p, xb)
+    y_ref, S = oracle.dense_packed(p.U, p.V, p.s1, p.s2, p.r, xb)
+    assert np.all(np.isfinite(y_ref))
+    got = bf16_bits_to_f64(y)
+    assert np.all(np.isfinite(got))
+    for m, e in enumerate(exps):
+        if e is None:
+            assert np.all(y[m] & 0x7FFF == 0)
+            continue
+        # row m is a base row times 2^e, so is everything it produces: the absolute part of the
+        # bound scales with it (else it would hide any error of a tiny row)
+        tol = REL * S[m] + ABS * 2.0 ** e + half_ulp_bf16(y_ref[m])
+        err = np.abs(got[m] - y_ref[m])
+        assert np.all(err <= tol), "row 2^%d: max err/tol %.3g" % (e, float((err / tol).max()))
+
+
+def test_intermediate_beyond_fp16_range():
+    """Unit scales and |x| around 1000: every z fits fp16 but the sums t over 8192 rows reach
+    about 10^5, beyond 65504; the per-row power of two keeps t in range."""
+    need_gpu()
+    d_out, d_in, r, M = 512, 8192, 256, 12
+    p = synth.make_projection("trange", d_out, d_in, r, seed=2402)
+    p.s1 = np.full(d_out, 0x3C00, dtype=np.uint16)
+    p.s2 = np.full(d_in, 0x3C00, dtype=np.uint16)
+    xb = _rows_scaled(synth.acts_bf16(synth.rng_for(2403, d_in), (M, d_in)), [10] * M)
+    # the premise, by numpy alone: t = V^T x with V's unpacked signs (unit s2)
+    vbits = np.unpackbits(np.ascontiguousarray(p.V, dtype="<u4").view(np.uint8), axis=1, bitorder="little")[:, :r]
+    xf = (xb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    t = xf @ (2.0 * vbits - 1.0)
+    assert np.abs(xf).max() < 65504 and np.abs(t).max() > 65504
+    y = gpu_matmul(p, xb)
+    y_ref, S = oracle.dense_packed(p.U, p.V, p.s1, p.s2, p.r, xb)
+    check_tolerance(y, y_ref, S, "prefill |t| > 65504")
+
+
+def test_scale_grads_prefill_rows_beyond_fp16_range():
+    """The scale gradients' tensor-core path sums over rows in fp64 after undoing each row's
+    power of two: rows at 2^40 and 2^-40 in one call match the oracle's gradients."""
+    need_gpu()
+    d_out, d_in, r = 200, 512, 128
+    p = synth.make_projection("gscale", d_out, d_in, r, seed=2404)
+    exps = [40, 0, -40, 10, 0, -10, 20, 0, 5, -5]
+    xb = _rows_scaled(synth.acts_bf16(synth.rng_for(2405, d_in), (len(exps), d_in)), exps)
+    yb = synth.acts_bf16(synth.rng_for(2406, d_out), (len(exps), d_out))
+    L = upload_projection(p)
+    g1, g2 = nq().lrb_scale_grads(L, upload_bf16(xb), upload_bf16(yb))
+    nq().sync_status()
+    ref1, S1, ref2, S2 = oracle.scale_grads_packed(p.U, p.V, p.s1, p.s2, p.r, xb, yb)
+    g1 = g1.cpu().numpy().astype(np.float64)
+    g2 = g2.cpu().numpy().astype(np.float64)
+    assert np.all(np.isfinite(g1)) and np.all(np.isfinite(g2))
+    # fp32 outputs: the stated bound plus the output rounding (2^-24 relative)
+    assert np.all(np.abs(g1 - ref1) <= 2e-3 * S1 + 1e-5 + 2.0 ** -24 * np.abs(ref1))
+    assert np.all(np.abs(g2 - ref2) <= 2e-3 * S2 + 1e-5 + 2.0 ** -24 * np.abs(ref2))
