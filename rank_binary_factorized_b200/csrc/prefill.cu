@@ -398,18 +398,19 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             float* part = (ksplit > 1) ? args.partial + static_cast<int64_t>(u % ksplit) * args.M * args.ldo : nullptr;
             const int acc = tc_count & 1;
             const uint32_t aph = (tc_count >> 1) & 1u;
-            // does any token of this tile carry a power of two?  (loads issued before the wait
-            // for the accumulator, so their latency hides behind it; almost always none)
-            bool tile_scaled = false;
-            if (MODE == kModeU && args.row_exp != nullptr) {
+            // does any token of this tile carry a power of two?  The exponents are loaded before
+            // the wait for the accumulator and first used after it, so their latency hides
+            // behind the wait; almost always none is set.
+            int tev[8];
+            const bool has_exp = (MODE == kModeU) && args.row_exp != nullptr;
 #pragma unroll
-                for (int c = 0; c < 256; c += 32) {
-                    const int64_t tk = static_cast<int64_t>(tn) * tile_n + c + lane;
-                    if (c + lane < tile_n && tk < args.M && args.row_exp[tk] != 0) tile_scaled = true;
-                }
-                tile_scaled = __any_sync(__activemask(), tile_scaled);
+            for (int c = 0; c < 8; ++c) {
+                const int64_t tk = static_cast<int64_t>(tn) * tile_n + 32 * c + lane;
+                tev[c] = (has_exp && 32 * c + lane < tile_n && tk < args.M) ? args.row_exp[tk] : 0;
             }
             if (!(ok = tc::mbar_wait(acc_full(acc), aph, err))) break;
+            const bool tile_scaled =
+                has_exp && __any_sync(__activemask(), ((tev[0] | tev[1] | tev[2] | tev[3]) | (tev[4] | tev[5] | tev[6] | tev[7])) != 0);
             tc::tc_fence_after();
             const int64_t wrow = static_cast<int64_t>(tw) * kTileW + rl;
             const bool row_ok = wrow < args.rows_w;
