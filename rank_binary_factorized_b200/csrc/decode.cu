@@ -784,15 +784,21 @@ __global__ void __launch_bounds__(TH, 1) decode_stage2_kernel(const __grid_const
             const int64_t row0 = static_cast<int64_t>(a) * 16;
             const int64_t row1 = min(static_cast<int64_t>(b) * 16, q.d_out);
             const int rows = static_cast<int>(row1 - row0);
-            const bool even = ((q.ldu & 1) == 0) && ((q.nw & 1) == 0);
-            // one warp per row, lanes along the row
+            // one warp per row, lanes along the row: 16-byte pieces when the row stride allows
+            // (reading up to 4 ceil(nw / 4) <= ldu words), else 8- or 4-byte pieces
+            const int mode = ((q.ldu & 3) == 0) ? 16 : (((q.ldu & 1) == 0 && (q.nw & 1) == 0) ? 8 : 4);
+            const int pieces = mode == 16 ? (q.nw + 3) >> 2 : (mode == 8 ? q.nw >> 1 : q.nw);
+            const uint32_t dst0 = static_cast<uint32_t>(__cvta_generic_to_shared(sm[k].ublk));
+            const uint32_t* src0 = q.U + row0 * q.ldu;
             for (int rr = warp; rr < rows; rr += kS2Warps) {
-                const uint32_t* src = q.U + (row0 + rr) * q.ldu;
-                const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(sm[k].ublk + rr * q.su));
-                if (even) {
-                    for (int c = lane; c < q.nw / 2; c += 32) cp_async8(dst + 8u * c, src + 2 * c);
+                const uint32_t* src = src0 + rr * q.ldu;
+                const uint32_t dst = dst0 + 4u * static_cast<uint32_t>(rr * q.su);
+                if (mode == 16) {
+                    for (int c = lane; c < pieces; c += 32) cp_async16(dst + 16u * c, src + 4 * c);
+                } else if (mode == 8) {
+                    for (int c = lane; c < pieces; c += 32) cp_async8(dst + 8u * c, src + 2 * c);
                 } else {
-                    for (int c = lane; c < q.nw; c += 32) cp_async4(dst + 4u * c, src + c);
+                    for (int c = lane; c < pieces; c += 32) cp_async4(dst + 4u * c, src + c);
                 }
             }
         }
