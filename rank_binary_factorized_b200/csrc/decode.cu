@@ -439,25 +439,40 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const __grid_const
         if (warp_active) {
             const int w = wcol;
             const int kb_lo = (khalf * nkb) / kKSplit, kb_hi = ((khalf + 1) * nkb) / kKSplit;
-            for (int kb2 = kb_lo; kb2 < kb_hi; kb2 += 2) {
+            // operands of K step kb: the A words of both 16-output halves and the B digits;
+            // the next step's are loaded from shared memory while this step's MMAs issue
+            const uint32_t* abase = aws + w * (nkb * 32 + 4) + tig * 4;
+            const uint32_t* zbase = zq + tig * SWZ + gid;
+            struct Ops {
+                uint4 a[2];
+                uint32_t b[NT][2];
+            };
+            auto fetch = [&](int kb, Ops& o) {
 #pragma unroll
-                for (int par = 0; par < 2; ++par) {
-                    const int kb = kb2 + par;
-                    if (kb < kb_hi) {
-                        uint32_t bf[NT][2];
+                for (int h = 0; h < 2; ++h) o.a[h] = *reinterpret_cast<const uint4*>(abase + (kb * 2 + h) * 16);
 #pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) {
-                            bf[nt][0] = zq[(8 * kb + tig) * SWZ + nt * 8 + gid];
-                            bf[nt][1] = zq[(8 * kb + 4 + tig) * SWZ + nt * 8 + gid];
-                        }
+                for (int nt = 0; nt < NT; ++nt) {
+                    o.b[nt][0] = zbase[(8 * kb) * SWZ + nt * 8];
+                    o.b[nt][1] = zbase[(8 * kb + 4) * SWZ + nt * 8];
+                }
+            };
+            auto issue = [&](const Ops& o, int (&ac)[2][NT][4]) {
 #pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            const uint4 a = *reinterpret_cast<const uint4*>(aws + w * (nkb * 32 + 4) + ((kb * 2 + h) * 4 + tig) * 4);
+                for (int h = 0; h < 2; ++h)
 #pragma unroll
-                            for (int nt = 0; nt < NT; ++nt)
-                                mma_u8s8(acc[par][h][nt], a.x & msk, a.y & msk, a.z & msk, a.w & msk, bf[nt][0], bf[nt][1]);
-                        }
-                    }
+                    for (int nt = 0; nt < NT; ++nt)
+                        mma_u8s8(ac[h][nt], o.a[h].x & msk, o.a[h].y & msk, o.a[h].z & msk, o.a[h].w & msk, o.b[nt][0],
+                                 o.b[nt][1]);
+            };
+            Ops cur, nxt;
+            if (kb_lo < kb_hi) fetch(kb_lo, cur);
+            // two accumulator sets, even and odd K steps, for two independent MMA chains per tile
+            for (int kb = kb_lo; kb < kb_hi; kb += 2) {
+                if (kb + 1 < kb_hi) fetch(kb + 1, nxt);
+                issue(cur, acc[0]);
+                if (kb + 1 < kb_hi) {
+                    if (kb + 2 < kb_hi) fetch(kb + 2, cur);
+                    issue(nxt, acc[1]);
                 }
             }
         }
