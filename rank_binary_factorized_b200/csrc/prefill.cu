@@ -94,6 +94,35 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
                  : "memory");
 }
 
+// One 32-token chunk of GEMM 2's epilogue when some token carries a power of two (rare: rows
+// outside fp16's range): the chunk is read from TMEM again and token j's values are multiplied
+// by 2^e_j, e_j handed across the warp from lane j.  Kept out of line so that the plain loop
+// stays compact.  Returns the chunk's share of the gradient partial (gradient mode).
+__device__ __noinline__ double scaled_chunk(const PrefillArgs& args, uint32_t taddr, int tn, int tile_n, int c0,
+                                            int64_t wrow, bool row_ok, float scale, bool grad, int el) {
+    uint32_t v[32];
+    tc::tmem_ld_32x32b_x32(taddr, v);
+    tc::tmem_wait_ld();
+    double g = 0.0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        const int e = __shfl_sync(__activemask(), el, j);
+        const int64_t tok = static_cast<int64_t>(tn) * tile_n + c0 + j;
+        if (row_ok && c0 + j < tile_n && tok < args.M) {
+            const float f = __uint_as_float(v[j]);
+            if (grad) {
+                g += static_cast<double>(bf16_bits_to_float(args.cot[tok * args.ldcot + wrow])) *
+                     (static_cast<double>(f) * __longlong_as_double(static_cast<long long>(1023 + e) << 52));
+            } else {
+                const float sf = scale * f;
+                const float o = (e >= -126 && e <= 127) ? sf * __int_as_float((e + 127) << 23) : ldexpf(sf, e);
+                static_cast<uint16_t*>(args.out)[tok * args.ldo + wrow] = float_to_bf16_bits(o);
+            }
+        }
+    }
+    return g;
+}
+
 // SPLIT: the launch splits tiles over K (mode V); without it the unit of work is the tile and
 // the unit bookkeeping folds away at compile time.
 template <int MODE, bool SPLIT>
@@ -451,23 +480,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                         }
                     }
                 } else if (MODE == kModeU) {
-                    // token j's values times 2^e_j (exact powers of two), e_j from lane j
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int e = __shfl_sync(__activemask(), el, j);
-                        const int64_t tok = static_cast<int64_t>(tn) * tile_n + c0 + j;
-                        if (row_ok && c0 + j < tile_n && tok < args.M) {
-                            const float f = __uint_as_float(v[j]);
-                            if (grad) {
-                                g += static_cast<double>(bf16_bits_to_float(args.cot[tok * args.ldcot + wrow])) *
-                                     (static_cast<double>(f) * __longlong_as_double(static_cast<long long>(1023 + e) << 52));
-                            } else {
-                                const float sf = scale * f;
-                                const float o = (e >= -126 && e <= 127) ? sf * __int_as_float((e + 127) << 23) : ldexpf(sf, e);
-                                static_cast<uint16_t*>(args.out)[tok * args.ldo + wrow] = float_to_bf16_bits(o);
-                            }
-                        }
-                    }
+                    g += scaled_chunk(args, tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * 256 + c0, tn,
+                                      tile_n, c0, wrow, row_ok, scale, grad, el);
                 }
             }
             if (grad && row_ok) args.gpart[static_cast<int64_t>(tn) * args.rows_w + wrow] = g;
