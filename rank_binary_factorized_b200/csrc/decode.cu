@@ -109,6 +109,7 @@ __device__ __forceinline__ int s2_bidx(int s_, int w, int col, int ng) {
 // under programmatic dependent launch; the host picks 512 only for long slices and NT <= 2.
 constexpr int kS1Words = 8;            // words (of 32 outputs) per cluster chunk
 constexpr int kS1Outs = kS1Words * 32;  // outputs k per chunk
+constexpr int kS1PartCap = kS1Outs + 16;  // inbox doubles per batch row: ceil(256 / CS) CS <= 271
 
 struct S1Params {
     const uint32_t* V;
@@ -190,7 +191,7 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const __grid_const
     uint32_t* zq = aws + kS1Words * (nkb * 32 + 4);  // [nq_rows][SWZ]
     int* red = reinterpret_cast<int*>(zq + nq_rows * SWZ);               // [256][NT*8]
     double* part = reinterpret_cast<double*>(red + kS1Outs * NT * 8);   // inbox [M][per][CS]
-    float* zs_s = reinterpret_cast<float*>(part + p.M * (kS1Outs + 16));  // [M][zld] when p.zstage
+    float* zs_s = reinterpret_cast<float*>(part + p.M * (kS1PartCap + 16));  // [M][zld] when p.zstage
     const int zld = p.rows_per_slice + p.rows_per_slice / 32;             // one pad word per 32
     __shared__ float s_mul[NQ_MATVEC_MAX_M];
     __shared__ double s_dinv[NQ_MATVEC_MAX_M];  // 2^-shift: turns the exact integers into values
@@ -515,22 +516,24 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const __grid_const
     // block of rank k / per; every block stores its fp64 partial for k into slot [rank of
     // the sender] of the owner's inbox (distributed shared memory), one cluster barrier
     // publishes the stores, and each owner sums its slots in a fixed order.
-    // CS is a power of two (1 .. 16), so is the share per owner; the exact integer times the
-    // power of two 2^-shift is exact in fp64
-    const int lg_per = 8 - (31 - __clz(CS));  // log2(kS1Outs / CS)
-    const int per = 1 << lg_per;
+    // The share per owner is ceil(256 / CS) outputs (the last owner's may run short); the
+    // exact integer times the power of two 2^-shift is exact in fp64.
+    const int per = (kS1Outs + CS - 1) / CS;
+    // a power-of-two CS (the usual case) splits by shifts: no division on this critical path
+    const bool per_pow2 = (CS & (CS - 1)) == 0;
+    const int lg_per = per_pow2 ? 8 - (31 - __clz(CS)) : 0;
     for (int e = tid; e < p.M * kS1Outs; e += kS1Threads) {
         const int m = e / kS1Outs, kl = e - m * kS1Outs;
         const int* rr = red + kl * (NT * 8) + 3 * m;
         const long long P = static_cast<long long>(rr[0]) + (static_cast<long long>(rr[1]) << 8) +
                             (static_cast<long long>(rr[2]) << 16);
         const long long val = 2 * P - static_cast<long long>(s_zsum[m]);
-        const int owner = kl >> lg_per, ko = kl & (per - 1);
+        const int owner = per_pow2 ? (kl >> lg_per) : kl / per, ko = kl - owner * per;
         double* dst = cluster.map_shared_rank(part, owner);
         dst[(m * per + ko) * CS + q] = static_cast<double>(val) * s_dinv[m];
     }
     // the slice's bound on its share of |t| (exact), into every owner's inbox after the partials
-    double* bound = part + p.M * kS1Outs;  // [M][CS]
+    double* bound = part + p.M * kS1PartCap;  // [M][CS]
     if (p.tab)
         for (int e = tid; e < p.M * CS; e += kS1Threads) {
             const int m = e / CS, owner = e - m * CS;
@@ -560,7 +563,8 @@ __global__ void __launch_bounds__(TH, 1) decode_stage1_kernel(const __grid_const
 #pragma unroll
         for (int m = 0; m < MG; ++m) tqacc[m] = 0;
         for (int e = tid; e < p.M * per; e += kS1Threads) {
-            const int m = e >> lg_per, ko = e & (per - 1);
+            const int m = per_pow2 ? (e >> lg_per) : e / per, ko = e - m * per;
+            if (k_lo + ko >= kS1Outs) continue;  // past the chunk: the last owner's share runs short
             const int64_t k = static_cast<int64_t>(wglob0) * 32 + k_lo + ko;
             double sum = 0.0;
             if (k < p.r) {
@@ -945,6 +949,8 @@ constexpr size_t kStage2SmemBudget = 200 * 1024;
 
 int ntiles_for(int64_t M) { return static_cast<int>((3 * M + 7) / 8); }
 
+int stage1_max_clusters(int cs);
+
 struct S1Plan {
     int n_chunks, CS, rows_per_slice, jc_rows, zstage;
     size_t smem;
@@ -953,24 +959,36 @@ struct S1Plan {
 int chunks_of(int64_t r) { return static_cast<int>((r / 32 + nq::kS1Words - 1) / nq::kS1Words); }
 
 // Stage-1 shape for a grid of `total_chunks` word chunks over d_in rows: the cluster size CS
-// (row slices per chunk) shrinks as the chunk count grows, so that the grid stays near one
-// block per SM; rows per slice and the staging pass follow.
+// (row slices per chunk, up to 16) is a power of two that keeps the grid near one block per SM,
+// raised to any larger size for which the whole grid fits the SMs in one wave with every cluster
+// resident at once (the hardware's count of co-resident clusters of that size, one block per
+// SM); rows per slice and the staging pass follow.
 // A given cluster size (force_cs > 0) replaces the choice, for members of one grid.
 S1Plan plan_stage1(int64_t d_in, int total_chunks, int64_t M, int force_cs = 0) {
     S1Plan p{};
     p.n_chunks = total_chunks;
-    int cs = total_chunks <= 8 ? 16 : (total_chunks <= 18 ? 8 : (total_chunks <= 37 ? 4 : 2));
-    while (cs > 1 && static_cast<int64_t>(cs) * 32 > d_in) cs >>= 1;
     // more than 8 output columns (M > 2): blocks too register-heavy to share an SM with the
     // previous grid's, so a cluster waits for that many free SMs of one GPC; 8 keeps the wait
     // short (7B attention, M = 8: 30.8 -> 19.1 us per layer against 16)
-    if (ntiles_for(M) >= 2 && cs > 8) cs = 8;
+    const int cap = ntiles_for(M) >= 2 ? 8 : 16;
+    // the power of two that keeps the grid near one block per SM, and then any larger size for
+    // which the grid still fits the SMs in one wave with every cluster resident at once
+    int cs = total_chunks <= 8 ? 16 : (total_chunks <= 18 ? 8 : (total_chunks <= 37 ? 4 : 2));
+    while (cs > 1 && static_cast<int64_t>(cs) * 32 > d_in) cs >>= 1;
+    if (cs > cap) cs = cap;
+    for (int c = cap; c > cs; --c) {
+        if (static_cast<int64_t>(c) * 32 > d_in) continue;                               // slices of >= 32 rows
+        if (static_cast<int64_t>(c) * total_chunks > nq_host::sm_count()) continue;  // one wave
+        if (stage1_max_clusters(c) < total_chunks) continue;  // all clusters resident at once
+        cs = c;
+        break;
+    }
     if (force_cs > 0) cs = force_cs;
     p.CS = cs;
     p.rows_per_slice = static_cast<int>(((d_in + cs - 1) / cs + 31) / 32 * 32);
     const int nt = ntiles_for(M);
     const int swz = nt == 1 ? 8 : 24;
-    const size_t fixed = static_cast<size_t>(nq::kS1Outs) * nt * 8 * 4 + static_cast<size_t>(M) * (nq::kS1Outs + 16) * 8 +
+    const size_t fixed = static_cast<size_t>(nq::kS1Outs) * nt * 8 * 4 + static_cast<size_t>(M) * (nq::kS1PartCap + 16) * 8 +
                          nq::kS1Words * 16;
     int64_t jc = static_cast<int64_t>((kStage1SmemBudget - fixed) / (32 + swz)) / 32 * 32;
     if (jc > p.rows_per_slice) jc = p.rows_per_slice;
@@ -1031,6 +1049,37 @@ void set_stage2_attrs_once() {
     cudaFuncSetAttribute(nq::decode_stage2_kernel<NT, TH, GN, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(kStage2SmemBudget));
     done[dev].store(true, std::memory_order_release);
+}
+
+// Clusters of cs stage-1 blocks (each holding an SM's shared-memory budget) that can be
+// resident at once on this device, from the occupancy query; cached per device and size.
+int stage1_max_clusters(int cs) {
+    static std::atomic<int> cache[64][17];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || cs < 1 || cs > 16) return 0;
+    int v = cache[dev][cs].load(std::memory_order_acquire);
+    if (v > 0) return v - 1;
+    set_stage1_attrs_once<1, 256, 1>();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1, cs);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = kStage1SmemBudget;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = static_cast<unsigned>(cs);
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void*>(nq::decode_stage1_kernel<1, 256, 1>), &cfg) !=
+        cudaSuccess) {
+        cudaGetLastError();  // leave no error behind; the query is retried on the next call
+        return 0;
+    }
+    cache[dev][cs].store(n + 1, std::memory_order_release);
+    return n;
 }
 
 // One launch of each stage for n projections that share x (n = 1: a single layer).  With
