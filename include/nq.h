@@ -26,7 +26,8 @@
  * - Packed sign layout: row i of a [rows][ld] uint32 matrix holds element k of that row at
  *   bit (k % 32) of word (k / 32), least significant bit first; bit 1 means +1, bit 0
  *   means -1.  r must be a multiple of 32.  Words r/32 .. ld-1 of a row are padding: pack
- *   writes them as 0 and no reader looks at them.
+ *   writes them as 0, and their values never affect a result (the decode kernels may copy
+ *   them along with the row).
  * - fp16 values (s1, s2) and bf16 values (x, y) are passed as uint16_t bit patterns.
  * - Activations are row-major: x is [M][d_in], y is [M][d_out], contiguous.
  * - Alignment: every pointer must be 16-byte aligned (NQ_ERR_ALIGN otherwise).
@@ -37,6 +38,10 @@
  *   layer's weights in the kernel launched immediately before a call that reads them
  *   without a stream/event synchronisation in between.  Activations and workspace are
  *   only touched after that wait.
+ * - Environment: NQ_DISABLE_PDL=1 launches every kernel without programmatic dependent
+ *   launch (each waits for the previous grid in full); NQ_DECODE_PREFETCH=0 stops the decode
+ *   stage 1 from asking the copy engine to prefetch its rows of V into L2.  Both are read once
+ *   per process and change timing only, never a result.
  */
 #ifndef NQ_H_
 #define NQ_H_
