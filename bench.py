@@ -799,7 +799,8 @@ def reference_arm(args):
     return {"impl": "reference", "metric": METRIC, "value": round(v, 1), "unit": "us/layer", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(v / 1e3, 3), "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "Llama-2-7B attention projection d_out=d_in=4096 r=2048, decode batch %d" % args.batch,
+            "config": {"workload": "Llama-2-7B attention projection d_out=d_in=4096 r=2048 (1.0 bit/weight), decode batch %d"
+                                   % args.batch,
                        "batch": args.batch, "layers_per_step": 1},
             "cpu_baseline": {**base, "value": round(v, 1)},
             "e2e": {"value": round(v, 1), "unit": "us/layer", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
