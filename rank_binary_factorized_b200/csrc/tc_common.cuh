@@ -1,5 +1,5 @@
 // tc_common.cuh -- thin inline-PTX wrappers for the sm_100a tensor-core machinery used by
-// the prefill kernels: mbarriers, TMA tile loads (no multicast), tcgen05 MMA / TMEM.
+// the prefill kernels: mbarriers, TMA tile loads (each CTA loads its own tiles), tcgen05 MMA / TMEM.
 // Written from the public PTX ISA descriptions of these instructions.
 #pragma once
 
@@ -70,7 +70,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigne
     return mbar_wait_for(bar, parity, err, kWaitLimitNs);
 }
 
-// ------------------------------------------------------------------ TMA (tile mode, no multicast)
+// ------------------------------------------------------------------ TMA (tile mode, one CTA per copy)
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
